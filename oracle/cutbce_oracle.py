@@ -1,0 +1,251 @@
+"""Float64 CPU oracle for the exact fused large-vocabulary BCE loss and its gradient.
+
+TEST INFRASTRUCTURE. Only tests/, __graft_entry__.smoke() and bench.py's CPU
+baseline leg may import this module. The product path (the CUDA library and
+its Python binding) never imports it, and it imports nothing from the product.
+
+What it computes follows "Cut Binary Cross Entropy: Efficient Large-Vocabulary
+Loss and Gradient Kernels for Sequential Recommendation" (Li, Ning, Hammad):
+
+  * section III-A, Eq. (1): standard BCE of logit x and target y,
+        l(x, y) = -y log s(x) - (1 - y) log(1 - s(x)),  s = logistic sigmoid;
+  * section III-A, Eq. (2): the same value in the stable form
+        l(x, y) = max(x, 0) + log(1 + exp(-|x|)) - y x = l(x, 0) - y x;
+  * section III-A, Eq. (3): the loss of one position sums Eq. (2) over the whole
+    vocabulary (with a 1/V factor);
+  * section III-B, Eq. (4): dl/dx = s(x) - y, so with G = s(X) - Y,
+        grad_A = G E  and  grad_E = G^T A,
+    rows of A (here H) being the B*N flattened positions; averaging over the
+    positions adds 1/(BN), padding positions excluded.
+
+The logits X = A E^T are formed here chunk by chunk over the vocabulary (the
+"vocabulary chunking" idea of section III-A), densely, in float64, with a
+dense multi-hot Y inside the element loss (the Eq. (1)/(2) form), so that this
+file is a plain restatement and shares no arithmetic with the GPU design.
+
+Readings where the pages are silent (each is listed in the design doc):
+  * normalisation: MEAN_VALID_POSITIONS (default) divides the summed loss by the
+    number of valid positions; SUM does not divide; MEAN_ELEMENTS divides by
+    n_valid * V (Eq. (3)'s 1/V times section III-B's 1/BN);
+  * duplicate ids in a row count once (Y is multi-hot, y in {0, 1});
+  * -1 marks an empty slot; an id < -1 or >= V in a valid row is an error;
+    id 0 is an ordinary item;
+  * the per-position `weights` of the pages' API is read as a {0, 1} mask: a
+    masked row adds no loss, gets a zero dH row and adds nothing to dE; its ids
+    are ignored entirely (not even range-checked);
+  * the upstream gradient is one scalar g (default 1) multiplying dH and dE;
+  * with no valid position the loss and both gradients are 0.
+
+Every function here is pinned by tests/test_oracle_pins.py against identities,
+closed forms, finite differences and torch's own BCE-with-logits.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Sequence
+
+import numpy as np
+
+MEAN_VALID_POSITIONS = 0
+SUM = 1
+MEAN_ELEMENTS = 2
+
+LN2 = float(np.log(2.0))
+
+
+class TargetRangeError(ValueError):
+    """An id < -1 or >= V sits in a valid row."""
+
+
+@dataclasses.dataclass
+class Targets:
+    """The positive sets P_t and the validity of each position (section III-B, sparse ids)."""
+    valid: np.ndarray            # bool [T]
+    sets: list                   # per row: sorted int64 array of distinct ids (empty if masked)
+
+    @property
+    def n_valid(self) -> int:
+        return int(self.valid.sum())
+
+    @property
+    def row_counts(self) -> np.ndarray:
+        return np.array([len(s) for s in self.sets], dtype=np.int64)
+
+    @property
+    def n_pairs(self) -> int:
+        return int(self.row_counts.sum())
+
+
+def positive_sets(targets: np.ndarray, mask: Optional[np.ndarray], V: int) -> Targets:
+    """Apply the mask and the id rules: P_t = set of ids >= 0 in a valid row."""
+    targets = np.asarray(targets)
+    T = targets.shape[0]
+    valid = np.ones(T, dtype=bool) if mask is None else (np.asarray(mask) != 0)
+    sets = []
+    for t in range(T):
+        if not valid[t]:
+            sets.append(np.zeros(0, dtype=np.int64))
+            continue
+        row = targets[t].astype(np.int64)
+        if np.any(row < -1) or np.any(row >= V):
+            raise TargetRangeError(f"row {t}: id outside [-1, {V})")
+        sets.append(np.unique(row[row >= 0]))
+    return Targets(valid=valid, sets=sets)
+
+
+def sigmoid(x: np.ndarray) -> np.ndarray:
+    """Logistic sigmoid, two-branch form that never overflows."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-x[pos]))
+    ex = np.exp(x[~pos])
+    out[~pos] = ex / (1.0 + ex)
+    return out
+
+
+def bce_eq1(x: np.ndarray, y: np.ndarray) -> np.ndarray:
+    """Eq. (1): -y log s(x) - (1-y) log(1 - s(x)), evaluated literally (moderate |x| only)."""
+    x = np.asarray(x, dtype=np.float64)
+    y = np.asarray(y, dtype=np.float64)
+    p = 1.0 / (1.0 + np.exp(-x))
+    return -y * np.log(p) - (1.0 - y) * np.log(1.0 - p)
+
+
+def bce_eq2(x: np.ndarray, y: np.ndarray) -> np.ndarray:
+    """Eq. (2): max(x, 0) + log(1 + exp(-|x|)) - y x."""
+    x = np.asarray(x, dtype=np.float64)
+    y = np.asarray(y, dtype=np.float64)
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x))) - y * x
+
+
+def scale_factor(reduction: int, n_valid: int, V: int) -> float:
+    """Normalisation s applied to the summed loss and to both gradients."""
+    if n_valid == 0:
+        return 0.0
+    if reduction == MEAN_VALID_POSITIONS:
+        return 1.0 / n_valid
+    if reduction == SUM:
+        return 1.0
+    if reduction == MEAN_ELEMENTS:
+        return 1.0 / (float(n_valid) * float(V))
+    raise ValueError(f"unknown reduction {reduction}")
+
+
+def _multi_hot(sets_valid: Sequence[np.ndarray], c0: int, c1: int) -> np.ndarray:
+    Y = np.zeros((len(sets_valid), c1 - c0), dtype=np.float64)
+    for r, ids in enumerate(sets_valid):
+        sel = ids[(ids >= c0) & (ids < c1)]
+        Y[r, sel - c0] = 1.0
+    return Y
+
+
+@dataclasses.dataclass
+class Result:
+    loss: float
+    dH: Optional[np.ndarray]
+    dE: Optional[np.ndarray]
+    sum_loss: float              # unnormalised sum of Eq. (2) over valid rows and all items
+    n_valid: int
+    n_pairs: int
+    row_counts: np.ndarray
+
+
+def forward_backward(H: np.ndarray, E: np.ndarray, targets: np.ndarray,
+                     mask: Optional[np.ndarray] = None, reduction: int = MEAN_VALID_POSITIONS,
+                     grad_loss: float = 1.0, chunk: int = 8192, want_grad: bool = True) -> Result:
+    """Loss and gradients of the fused BCE, computed densely chunk by chunk over V.
+
+    H [T, D] and E [V, D] are taken as given (the exact input values, widened to
+    float64); targets [T, K] int ids with -1 empty; mask [T] (nonzero = valid).
+    """
+    H64 = np.asarray(H, dtype=np.float64)
+    E64 = np.asarray(E, dtype=np.float64)
+    T, D = H64.shape
+    V = E64.shape[0]
+    tg = positive_sets(targets, mask, V)
+    rows = np.nonzero(tg.valid)[0]
+    Hv = H64[rows]
+    sets_v = [tg.sets[t] for t in rows]
+
+    total = 0.0
+    dHv = np.zeros_like(Hv) if want_grad else None
+    dE = np.zeros((V, D), dtype=np.float64) if want_grad else None
+    if len(rows):
+        for c0 in range(0, V, chunk):
+            c1 = min(V, c0 + chunk)
+            Ec = E64[c0:c1]
+            Z = Hv @ Ec.T                                  # chunk logits, then discarded
+            Y = _multi_hot(sets_v, c0, c1)
+            total += float(bce_eq2(Z, Y).sum())            # Eq. (2), summed as in Eq. (3)
+            if want_grad:
+                G = sigmoid(Z) - Y                         # Eq. (4)
+                dHv += G @ Ec
+                dE[c0:c1] = G.T @ Hv
+    s = scale_factor(reduction, len(rows), V)
+    dH = None
+    if want_grad:
+        dH = np.zeros((T, D), dtype=np.float64)
+        dH[rows] = grad_loss * s * dHv
+        dE *= grad_loss * s
+    return Result(loss=s * total, dH=dH, dE=dE, sum_loss=total, n_valid=len(rows),
+                  n_pairs=tg.n_pairs, row_counts=tg.row_counts)
+
+
+def dE_rows(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np.ndarray],
+            items: Sequence[int], reduction: int = MEAN_VALID_POSITIONS,
+            grad_loss: float = 1.0) -> np.ndarray:
+    """Selected rows of grad_E (Eq. (4)), each from its own logit column X[:, v]."""
+    H64 = np.asarray(H, dtype=np.float64)
+    V = E.shape[0]
+    tg = positive_sets(targets, mask, V)
+    rows = np.nonzero(tg.valid)[0]
+    Hv = H64[rows]
+    s = scale_factor(reduction, len(rows), V)
+    out = np.zeros((len(items), H64.shape[1]), dtype=np.float64)
+    for i, v in enumerate(items):
+        z = Hv @ np.asarray(E[v], dtype=np.float64)
+        y = np.array([1.0 if np.any(tg.sets[t] == v) else 0.0 for t in rows])
+        out[i] = grad_loss * s * ((sigmoid(z) - y) @ Hv)
+    return out
+
+
+def dH_rows(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np.ndarray],
+            positions: Sequence[int], reduction: int = MEAN_VALID_POSITIONS,
+            grad_loss: float = 1.0, chunk: int = 1 << 20) -> np.ndarray:
+    """Selected rows of grad_A = grad_H (Eq. (4)), each from its own logit row X[t, :]."""
+    V = E.shape[0]
+    tg = positive_sets(targets, mask, V)
+    s = scale_factor(reduction, tg.n_valid, V)
+    out = np.zeros((len(positions), H.shape[1]), dtype=np.float64)
+    for i, t in enumerate(positions):
+        if not tg.valid[t]:
+            continue
+        h = np.asarray(H[t], dtype=np.float64)
+        acc = np.zeros(H.shape[1], dtype=np.float64)
+        for c0 in range(0, V, chunk):
+            c1 = min(V, c0 + chunk)
+            Ec = np.asarray(E[c0:c1], dtype=np.float64)
+            z = Ec @ h
+            y = np.zeros(c1 - c0)
+            ids = tg.sets[t]
+            y[ids[(ids >= c0) & (ids < c1)] - c0] = 1.0
+            acc += (sigmoid(z) - y) @ Ec
+        out[i] = grad_loss * s * acc
+    return out
+
+
+def loss_sum_slice(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np.ndarray],
+                   v0: int, v1: int, chunk: int = 8192) -> float:
+    """Unnormalised Eq. (2) sum restricted to the items [v0, v1) (all valid rows)."""
+    V = E.shape[0]
+    tg = positive_sets(targets, mask, V)
+    rows = np.nonzero(tg.valid)[0]
+    Hv = np.asarray(H, dtype=np.float64)[rows]
+    sets_v = [tg.sets[t] for t in rows]
+    total = 0.0
+    for c0 in range(v0, v1, chunk):
+        c1 = min(v1, c0 + chunk)
+        Z = Hv @ np.asarray(E[c0:c1], dtype=np.float64).T
+        total += float(bce_eq2(Z, _multi_hot(sets_v, c0, c1)).sum())
+    return total
