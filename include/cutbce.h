@@ -1,0 +1,170 @@
+/*
+ * cutbce.h -- C ABI of the exact fused large-vocabulary binary cross-entropy
+ * loss and its gradient, for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one defined in "Cut Binary Cross Entropy: Efficient
+ * Large-Vocabulary Loss and Gradient Kernels for Sequential Recommendation"
+ * (Li, Ning, Hammad):
+ *
+ *   logits      x_tv = h_t . e_v                           (section I-A, X = A E^T)
+ *   element     l(x, y) = max(x,0) + log(1 + e^-|x|) - y x  (section III-A, Eq. (2))
+ *   loss        s * sum_{valid t} sum_{v < V} l(x_tv, y_tv)   (Eq. (3), averaging of III-B)
+ *   gradients   G = sigmoid(X) - Y,  dH = g s G E,  dE = g s G^T H   (section III-B, Eq. (4))
+ *
+ * where y_tv = 1 iff item v is one of the (distinct) positive ids of
+ * position t, s is the normalisation chosen by `reduction`, and g is the
+ * upstream gradient.  The [T, V] logits and their gradient are never written
+ * to device memory (section III-B, Table I of the paper): every logit tile is
+ * formed on chip, in tensor memory, and consumed there.
+ *
+ * Conventions shared by every entry point:
+ *  - T = B * N flattened positions (section III-A, footnote 1), V items,
+ *    D feature width, K target slots per position.
+ *  - H is [T, D] and E is [V, D], row-major, dense, device memory.  bf16
+ *    (CUTBCE_BF16, the fast path) or fp32 (CUTBCE_F32, a plain CUDA-core path
+ *    meant for small checks).  For bf16, D must be a multiple of 8 and at most
+ *    256, and H, E must be 16-byte aligned.
+ *  - targets is int32 [T, K], device memory.  -1 marks an empty slot; an id in
+ *    [0, V) is a positive item; repeated ids in one row count once.  Any other
+ *    id in a valid row is a data error (CUTBCE_ERR_TARGET_RANGE, reported
+ *    through the workspace status word, see cutbce_read_status).
+ *  - mask is uint8 [T] (1 = valid position, 0 = padding), device memory, or
+ *    NULL for "all valid".  A masked position contributes no loss, receives a
+ *    zero dH row and contributes nothing to dE; its ids are ignored entirely.
+ *  - Every output and the workspace are owned by the caller.  The library
+ *    never allocates or frees device memory and keeps no state between calls
+ *    apart from cached device attributes.
+ *  - All compute calls are asynchronous on `stream`.  Errors a host can see
+ *    (NULL pointers, sizes <= 0, unsupported D or dtype, a workspace that is
+ *    too small, a device that is not sm_100) are returned before anything is
+ *    launched.  Data-dependent errors (an id out of range, a bounded wait in a
+ *    kernel that ran out) are written to the workspace status word; when it is
+ *    nonzero the outputs of that call are unspecified.
+ *  - dH and dE are overwritten, not accumulated.  The loss is double.
+ *  - Results are deterministic: no floating-point atomics are used, and every
+ *    reduction runs in a fixed order that does not depend on the GPU's SM count.
+ */
+#ifndef CUTBCE_H
+#define CUTBCE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st* cutbce_stream_t;
+
+typedef enum {
+  CUTBCE_OK = 0,
+  CUTBCE_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, misaligned pointer */
+  CUTBCE_ERR_UNSUPPORTED = 2,   /* D, K or dtype outside the supported set; not an sm_100 device */
+  CUTBCE_ERR_WORKSPACE = 3,     /* workspace smaller than cutbce_workspace_size() */
+  CUTBCE_ERR_TARGET_RANGE = 4,  /* an id < -1 or >= V in a valid row (device-detected) */
+  CUTBCE_ERR_TIMEOUT = 5,       /* a bounded wait inside a kernel ran out (device-detected) */
+  CUTBCE_ERR_CUDA = 6           /* a CUDA runtime call failed */
+} cutbce_status;
+
+typedef enum { CUTBCE_BF16 = 0, CUTBCE_F32 = 1 } cutbce_dtype;
+
+/* Normalisation s of the summed loss (and of both gradients):
+ *  MEAN_VALID_POSITIONS: 1 / n_valid  (positions averaged, padding excluded; section III-B)
+ *  SUM:                  1
+ *  MEAN_ELEMENTS:        1 / (n_valid * V)  (Eq. (3)'s 1/V and section III-B's 1/BN)
+ * With n_valid = 0 the loss and both gradients are 0. */
+typedef enum {
+  CUTBCE_MEAN_VALID_POSITIONS = 0,
+  CUTBCE_SUM = 1,
+  CUTBCE_MEAN_ELEMENTS = 2
+} cutbce_reduction;
+
+/* Problem statement, after the paper's cut_binary_cross_entropy(activations,
+ * embeddings, targets, weights) (section III-C, Listing 1), flattened to T rows. */
+typedef struct {
+  int64_t T;                 /* positions (B*N), >= 1 */
+  int64_t V;                 /* items, >= 1, < 2^31 */
+  int64_t D;                 /* feature width, >= 1 */
+  int64_t K;                 /* target slots per position, 1..128 */
+  int32_t dtype;             /* cutbce_dtype of H and E */
+  int32_t reduction;         /* cutbce_reduction */
+  const void* H;             /* [T, D] activations (device) */
+  const void* E;             /* [V, D] item embeddings (device) */
+  const int32_t* targets;    /* [T, K] positive ids, -1 empty (device) */
+  const uint8_t* mask;       /* [T] 1 = valid, or NULL = all valid (device) */
+} cutbce_problem;
+
+/* Bytes of device workspace that a compute call on this problem needs.  The
+ * size has no T*V term: it is O(T*K + S*T*D + V/128) for a split count S <= 64
+ * chosen from T.  Host-only; launches nothing.  Returns INVALID_ARG or
+ * UNSUPPORTED for a problem the compute calls would reject. */
+cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes);
+
+/* Loss only (section III-A).  loss: device double, written with the
+ * normalised loss.  ws: device workspace of ws_bytes bytes (>= workspace size),
+ * 256-byte aligned. */
+cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_bytes,
+                             double* loss, cutbce_stream_t stream);
+
+/* Gradients only (section III-B, Eq. (4)), recomputing the logits.
+ * grad_loss: device float scalar g, or NULL for g = 1.
+ * dH: device float [T, D]; dE: device float [V, D]; either may be NULL to skip it. */
+cutbce_status cutbce_backward(const cutbce_problem* prob, const float* grad_loss,
+                              float* dH, float* dE, void* ws, size_t ws_bytes,
+                              cutbce_stream_t stream);
+
+/* Loss and both gradients in one pass over the logits for the loss and dE and
+ * a second pass for dH.  loss may be NULL to skip it; dH or dE may be NULL. */
+cutbce_status cutbce_forward_backward(const cutbce_problem* prob, const float* grad_loss,
+                                      double* loss, float* dH, float* dE,
+                                      void* ws, size_t ws_bytes, cutbce_stream_t stream);
+
+/* Bytes of device memory that cutbce_forward_backward_host needs in dev_buf. */
+cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes);
+
+/* The fused call for callers whose buffers live in host memory: prob's H, E,
+ * targets and mask are HOST pointers (pinned memory makes the copies
+ * asynchronous), grad_loss is a host value, and loss / dH / dE are host
+ * outputs (dH, dE may be NULL).  dev_buf (>= cutbce_host_buffer_size bytes,
+ * 256-byte aligned, caller-owned device memory) holds the device copies and the
+ * workspace.  The call copies the inputs in, runs cutbce_forward_backward,
+ * copies the results out and synchronises `stream`; on return the host outputs
+ * are valid and the returned status includes the device status word. */
+cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float grad_loss,
+                                           double* loss, float* dH, float* dE,
+                                           void* dev_buf, size_t dev_bytes,
+                                           cutbce_stream_t stream);
+
+/* Synchronises `stream` and returns the device status word of the last call
+ * that used this workspace (CUTBCE_OK, TARGET_RANGE or TIMEOUT). */
+cutbce_status cutbce_read_status(const void* ws, cutbce_stream_t stream);
+
+/* Synchronises `stream` and reads the integer side results of the last call on
+ * this workspace: the number of valid positions, the number of distinct
+ * (position, positive item) pairs, and, if row_counts is not NULL, the number of
+ * distinct positive ids of each position (host int32 [T], 0 for masked rows). */
+cutbce_status cutbce_read_counts(const cutbce_problem* prob, const void* ws,
+                                 int64_t* n_valid, int64_t* n_pairs, int32_t* row_counts,
+                                 cutbce_stream_t stream);
+
+/* Number of kernels one call of the given entry (0 forward, 1 backward,
+ * 2 forward_backward) launches for this problem (for launch accounting). */
+int cutbce_kernel_launches(const cutbce_problem* prob, int entry);
+
+/* Human-readable name of a status code (static storage). */
+const char* cutbce_status_string(cutbce_status status);
+
+/* Self-test of the bounded-wait machinery the kernels use: launches one CTA
+ * that waits on a shared-memory barrier nothing will ever signal, with a
+ * limit of limit_ns nanoseconds.  The wait gives up, writes CUTBCE_ERR_TIMEOUT
+ * to *status_dev (device int32) and the kernel returns normally: the context
+ * stays usable.  limit_ns must be in (0, 10^10]. */
+cutbce_status cutbce_selftest_wait_timeout(int64_t limit_ns, int32_t* status_dev,
+                                           cutbce_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CUTBCE_H */

@@ -1,0 +1,180 @@
+"""GPU vs float64 oracle, element by element, on seeded inputs (small sizes
+spanning several tiles with ragged tails in both T and V, every supported
+feature width, the three normalisations, and the method's edge cases)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import cutbce_oracle as O
+from vocabulary_label_bce_b200 import binding as B
+from vocabulary_label_bce_b200 import workloads as W
+from gpu_util import GRAD_RTOL, LOSS_RTOL, check_against_oracle, rel_fro, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    dict(T=300, V=1000, D=64, K=5),     # 3 position tiles, 8 item tiles, both ragged
+    dict(T=257, V=2047, D=128, K=8),
+    dict(T=200, V=777, D=256, K=16),    # streamed tiles of 64 rows
+    dict(T=130, V=515, D=192, K=6),
+    dict(T=100, V=300, D=32, K=4),      # feature width padded to 64 by the TMA box
+    dict(T=129, V=640, D=96, K=3),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"T{s['T']}_V{s['V']}_D{s['D']}")
+def test_fused_matches_oracle(shape):
+    p = W.draw(**shape, dtype="bf16", seed=1, ids="zipf", zipf_s=1.1, mask="random", mask_frac=0.1)
+    got = run_gpu(p, "mean")
+    _, rep = check_against_oracle(p, got, "mean")
+    print(shape, rep)
+
+
+@pytest.mark.parametrize("reduction", ["sum", "mean", "mean_elements"])
+def test_reductions_and_upstream_gradient(reduction):
+    p = W.draw(T=333, V=1500, D=64, K=4, dtype="bf16", seed=2, mask="random", mask_frac=0.2)
+    got = run_gpu(p, reduction, grad_loss=0.37)
+    check_against_oracle(p, got, reduction, grad_loss=0.37)
+
+
+def test_tiny_f32_config():
+    p = W.draw_config("tiny_f32")
+    got = run_gpu(p, "mean")
+    _, rep = check_against_oracle(p, got, "mean", loss_rtol=1e-6, grad_rtol=1e-5)
+    print(rep)
+
+
+def test_small_catalog_config_full():
+    p = W.draw_config("small_catalog")
+    got = run_gpu(p, "mean")
+    _, rep = check_against_oracle(p, got, "mean")
+    print(rep)
+
+
+def test_forward_and_backward_entries():
+    p = W.draw(T=200, V=900, D=64, K=5, dtype="bf16", seed=3, ids="zipf", mask="random", mask_frac=0.1)
+    t = to_device(p)
+    fused = run_gpu(p, "mean", tensors=t)
+    fwd = run_gpu(p, "mean", entry="forward", tensors=t)
+    bwd = run_gpu(p, "mean", entry="backward", tensors=t)
+    assert fwd["status"] == 0 and bwd["status"] == 0
+    assert fwd["loss"] == fused["loss"]          # same kernels, same order
+    check_against_oracle(p, fwd, "mean")
+    check_against_oracle(p, bwd, "mean")
+    assert rel_fro(bwd["dE"], fused["dE"]) < 1e-3 and rel_fro(bwd["dH"], fused["dH"]) < 1e-3
+
+
+def test_deterministic_bits():
+    p = W.draw(T=400, V=3000, D=64, K=8, dtype="bf16", seed=4, ids="zipf", mask="random", mask_frac=0.1)
+    t = to_device(p)
+    a = run_gpu(p, "mean", tensors=t)
+    b = run_gpu(p, "mean", tensors=t)
+    assert a["loss"] == b["loss"]
+    assert np.array_equal(a["dH"], b["dH"]) and np.array_equal(a["dE"], b["dE"])
+
+
+def test_all_masked():
+    p = W.draw(T=150, V=400, D=64, K=3, dtype="bf16", seed=5)
+    p.mask[:] = 0
+    got = run_gpu(p, "mean")
+    assert got["status"] == 0
+    assert got["loss"] == 0.0 and np.all(got["dH"] == 0) and np.all(got["dE"] == 0)
+
+
+def test_single_position_single_item():
+    p = W.draw(T=1, V=1, D=64, K=2, dtype="bf16", seed=6, mask="none")
+    got = run_gpu(p, "sum")
+    check_against_oracle(p, got, "sum")
+
+
+def test_no_positive_ids():
+    p = W.draw(T=140, V=700, D=64, K=4, dtype="bf16", seed=7)
+    p.targets[:] = -1
+    got = run_gpu(p, "mean")
+    check_against_oracle(p, got, "mean")
+
+
+def test_duplicates_padding_and_masked_garbage():
+    p = W.draw(T=260, V=1300, D=64, K=6, dtype="bf16", seed=8, ids="zipf", mask="random", mask_frac=0.25)
+    p.targets[:, 5] = p.targets[:, 0]            # repeated ids
+    p.targets[::7, 2] = -1                        # holes
+    masked = np.nonzero(p.mask == 0)[0]
+    p.targets[masked, 1] = 10**6                  # out of range, but in masked rows: ignored
+    got = run_gpu(p, "mean")
+    check_against_oracle(p, got, "mean")
+
+
+def test_out_of_range_id_sets_status():
+    p = W.draw(T=64, V=500, D=64, K=3, dtype="bf16", seed=9, mask="none")
+    p.targets[10, 1] = 500
+    got = run_gpu(p, "mean")
+    assert got["status"] == B.ERR_TARGET_RANGE
+    p.targets[10, 1] = -5
+    got = run_gpu(p, "mean")
+    assert got["status"] == B.ERR_TARGET_RANGE
+
+
+def test_zero_activations_closed_form():
+    p = W.draw(T=190, V=1100, D=64, K=5, dtype="bf16", seed=10, mask="random", mask_frac=0.1)
+    p.H[:] = 0
+    p.H_bits[:] = 0
+    got = run_gpu(p, "sum")
+    tg = O.positive_sets(p.targets, p.mask, p.V)
+    assert got["loss"] == pytest.approx(tg.n_valid * p.V * math.log(2.0), rel=1e-6)
+    assert np.all(got["dE"] == 0.0)
+    check_against_oracle(p, got, "sum")
+
+
+def test_paper_stress_distribution():
+    # A, E ~ N(0, I), D=128, L=8 uniform ids (mini-benchmark inputs): saturated logits
+    p = W.draw(T=256, V=2000, D=128, K=8, dtype="bf16", seed=11, e_std=1.0, ids="uniform", mask="none")
+    got = run_gpu(p, "mean")
+    _, rep = check_against_oracle(p, got, "mean")
+    print(rep)
+
+
+def test_host_buffer_entry_matches_device_entry():
+    p = W.draw(T=300, V=1200, D=64, K=5, dtype="bf16", seed=12, ids="zipf", mask="random", mask_frac=0.1)
+    dev = run_gpu(p, "mean", grad_loss=1.5)
+    Hh = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Eh = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    th = torch.from_numpy(p.targets).pin_memory()
+    mh = torch.from_numpy(p.mask).pin_memory()
+    prob = B.make_problem(Hh, Eh, th, mh, "mean")
+    buf = torch.empty(B.cutbce_host_buffer_size(prob), dtype=torch.uint8, device="cuda")
+    loss = torch.zeros((), dtype=torch.float64).pin_memory()
+    dH = torch.zeros((p.T, p.D), dtype=torch.float32).pin_memory()
+    dE = torch.zeros((p.V, p.D), dtype=torch.float32).pin_memory()
+    B.cutbce_forward_backward_host(prob, 1.5, loss, dH, dE, buf)
+    assert float(loss) == dev["loss"]
+    assert np.array_equal(dH.numpy(), dev["dH"].astype(np.float32))
+    assert np.array_equal(dE.numpy(), dev["dE"].astype(np.float32))
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    st = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    B.cutbce_selftest_wait_timeout(20_000_000, st)    # 20 ms on a barrier nothing signals
+    torch.cuda.synchronize()
+    assert int(st.item()) == B.ERR_TIMEOUT
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0                   # the context is still usable
+
+
+def test_autograd_wrapper():
+    from vocabulary_label_bce_b200.api import cut_bce
+    p = W.draw(T=180, V=800, D=64, K=4, dtype="bf16", seed=13, mask="random", mask_frac=0.1)
+    H, E, tg, m = to_device(p)
+    Hf = H.float().requires_grad_(True)
+    Ef = E.float().requires_grad_(True)
+    # bf16 leaves with autograd: compute through the kernel, gradients come back in the leaf dtype
+    Hb = H.clone().requires_grad_(True)
+    Eb = E.clone().requires_grad_(True)
+    loss = cut_bce(Hb, Eb, tg, m)
+    (2.0 * loss).backward()
+    ref = O.forward_backward(p.H, p.E, p.targets, p.mask, grad_loss=2.0)
+    assert abs(float(loss) - ref.loss) / abs(ref.loss) < LOSS_RTOL
+    assert rel_fro(Hb.grad.float().cpu().numpy(), ref.dH) < GRAD_RTOL + 4e-3   # bf16 output rounding
+    assert rel_fro(Eb.grad.float().cpu().numpy(), ref.dE) < GRAD_RTOL + 4e-3
+    del Hf, Ef

@@ -1,0 +1,194 @@
+"""ctypes binding of libcutbce (include/cutbce.h): argument marshalling only.
+
+Every step of the loss and its gradient runs in the library's CUDA kernels;
+this module only turns torch tensors into pointers and sizes, takes the
+current CUDA stream, and allocates outputs and the workspace through torch.
+There is no CPU fallback: if the library is missing, importing a function that
+needs it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "CutBCEError", "cutbce_problem", "load_library", "library_path", "declared_functions",
+    "cutbce_workspace_size", "cutbce_forward", "cutbce_backward", "cutbce_forward_backward",
+    "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
+    "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
+    "cutbce_selftest_wait_timeout", "REDUCTIONS",
+]
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TARGET_RANGE, ERR_TIMEOUT, ERR_CUDA = range(7)
+BF16, F32 = 0, 1
+REDUCTIONS = {"mean": 0, "sum": 1, "mean_elements": 2}
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_HEADER = os.path.join(os.path.dirname(_PKG), "include", "cutbce.h")
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libcutbce.so")
+
+
+class cutbce_problem(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int64), ("V", ctypes.c_int64), ("D", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("dtype", ctypes.c_int32), ("reduction", ctypes.c_int32),
+        ("H", ctypes.c_void_p), ("E", ctypes.c_void_p), ("targets", ctypes.c_void_p), ("mask", ctypes.c_void_p),
+    ]
+
+
+class CutBCEError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        msg = _LIB.cutbce_status_string(self.status).decode() if _LIB is not None else str(status)
+        super().__init__(f"{where}: {msg} (status {self.status})" if where else f"{msg} (status {self.status})")
+
+
+_LIB: Optional[ctypes.CDLL] = None
+_P = ctypes.POINTER(cutbce_problem)
+_vp, _sz, _i32, _i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
+_SIGS = {
+    "cutbce_workspace_size": (_i32, [_P, ctypes.POINTER(_sz)]),
+    "cutbce_forward": (_i32, [_P, _vp, _sz, _vp, _vp]),
+    "cutbce_backward": (_i32, [_P, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cutbce_forward_backward": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cutbce_host_buffer_size": (_i32, [_P, ctypes.POINTER(_sz)]),
+    "cutbce_forward_backward_host": (_i32, [_P, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cutbce_read_status": (_i32, [_vp, _vp]),
+    "cutbce_read_counts": (_i32, [_P, _vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), _vp, _vp]),
+    "cutbce_kernel_launches": (ctypes.c_int, [_P, ctypes.c_int]),
+    "cutbce_status_string": (ctypes.c_char_p, [_i32]),
+    "cutbce_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
+}
+
+
+def load_library() -> ctypes.CDLL:
+    """Load the in-tree libcutbce.so (built by `python -m vocabulary_label_bce_b200.build`)."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m vocabulary_label_bce_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions include/cutbce.h declares."""
+    text = open(_HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cutbce_[a-z_]+)\s*\(", text)))
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise CutBCEError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_problem(H: torch.Tensor, E: torch.Tensor, targets: torch.Tensor, mask: Optional[torch.Tensor] = None,
+                 reduction: str | int = "mean") -> cutbce_problem:
+    """Describe tensors already on the device.  H [T, D], E [V, D] bf16 or fp32, targets int32 [T, K]."""
+    if H.dim() != 2 or E.dim() != 2 or targets.dim() != 2:
+        raise ValueError("H, E, targets must be 2-D")
+    if H.dtype != E.dtype or H.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("H and E must share dtype bf16 or fp32")
+    if targets.dtype != torch.int32:
+        raise ValueError("targets must be int32")
+    for t in (H, E, targets) + ((mask,) if mask is not None else ()):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if mask is not None and mask.dtype not in (torch.uint8, torch.bool):
+        raise ValueError("mask must be uint8 or bool")
+    red = REDUCTIONS[reduction] if isinstance(reduction, str) else int(reduction)
+    return cutbce_problem(H.shape[0], E.shape[0], H.shape[1], targets.shape[1],
+                          BF16 if H.dtype == torch.bfloat16 else F32, red,
+                          H.data_ptr(), E.data_ptr(), targets.data_ptr(),
+                          mask.data_ptr() if mask is not None else None)
+
+
+# ---------------------------------------------------------------- one function per C entry point
+def cutbce_workspace_size(prob: cutbce_problem) -> int:
+    n = _sz(0)
+    _check(load_library().cutbce_workspace_size(ctypes.byref(prob), ctypes.byref(n)), "cutbce_workspace_size")
+    return int(n.value)
+
+
+def cutbce_forward(prob, ws: torch.Tensor, loss: torch.Tensor, stream=None) -> None:
+    _check(load_library().cutbce_forward(ctypes.byref(prob), ws.data_ptr(), ws.numel(), loss.data_ptr(),
+                                         _stream(stream)), "cutbce_forward")
+
+
+def cutbce_backward(prob, grad_loss: Optional[torch.Tensor], dH: Optional[torch.Tensor],
+                    dE: Optional[torch.Tensor], ws: torch.Tensor, stream=None) -> None:
+    _check(load_library().cutbce_backward(
+        ctypes.byref(prob), grad_loss.data_ptr() if grad_loss is not None else None,
+        dH.data_ptr() if dH is not None else None, dE.data_ptr() if dE is not None else None,
+        ws.data_ptr(), ws.numel(), _stream(stream)), "cutbce_backward")
+
+
+def cutbce_forward_backward(prob, grad_loss: Optional[torch.Tensor], loss: Optional[torch.Tensor],
+                            dH: Optional[torch.Tensor], dE: Optional[torch.Tensor], ws: torch.Tensor,
+                            stream=None) -> None:
+    _check(load_library().cutbce_forward_backward(
+        ctypes.byref(prob), grad_loss.data_ptr() if grad_loss is not None else None,
+        loss.data_ptr() if loss is not None else None, dH.data_ptr() if dH is not None else None,
+        dE.data_ptr() if dE is not None else None, ws.data_ptr(), ws.numel(), _stream(stream)),
+        "cutbce_forward_backward")
+
+
+def cutbce_host_buffer_size(prob: cutbce_problem) -> int:
+    n = _sz(0)
+    _check(load_library().cutbce_host_buffer_size(ctypes.byref(prob), ctypes.byref(n)), "cutbce_host_buffer_size")
+    return int(n.value)
+
+
+def cutbce_forward_backward_host(prob, grad_loss: float, loss: torch.Tensor, dH: Optional[torch.Tensor],
+                                 dE: Optional[torch.Tensor], dev_buf: torch.Tensor, stream=None) -> None:
+    """prob's pointers and loss/dH/dE are host (CPU, ideally pinned) tensors; dev_buf is device memory."""
+    _check(load_library().cutbce_forward_backward_host(
+        ctypes.byref(prob), float(grad_loss), loss.data_ptr(), dH.data_ptr() if dH is not None else None,
+        dE.data_ptr() if dE is not None else None, dev_buf.data_ptr(), dev_buf.numel(), _stream(stream)),
+        "cutbce_forward_backward_host")
+
+
+def cutbce_read_status(ws: torch.Tensor, stream=None) -> int:
+    return int(load_library().cutbce_read_status(ws.data_ptr(), _stream(stream)))
+
+
+def cutbce_read_counts(prob, ws: torch.Tensor, row_counts: Optional[torch.Tensor] = None, stream=None):
+    nv, npairs = _i64(0), _i64(0)
+    _check(load_library().cutbce_read_counts(ctypes.byref(prob), ws.data_ptr(), ctypes.byref(nv),
+                                             ctypes.byref(npairs),
+                                             row_counts.data_ptr() if row_counts is not None else None,
+                                             _stream(stream)), "cutbce_read_counts")
+    return int(nv.value), int(npairs.value)
+
+
+def cutbce_kernel_launches(prob, entry: int) -> int:
+    return int(load_library().cutbce_kernel_launches(ctypes.byref(prob), int(entry)))
+
+
+def cutbce_status_string(status: int) -> str:
+    return load_library().cutbce_status_string(int(status)).decode()
+
+
+def cutbce_selftest_wait_timeout(limit_ns: int, status_dev: torch.Tensor, stream=None) -> None:
+    _check(load_library().cutbce_selftest_wait_timeout(int(limit_ns), status_dev.data_ptr(), _stream(stream)),
+           "cutbce_selftest_wait_timeout")

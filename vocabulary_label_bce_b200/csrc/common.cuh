@@ -1,0 +1,64 @@
+// Shared definitions: status codes, the workspace header, tile geometry.
+#pragma once
+#include <cstdint>
+#include <cstddef>
+
+namespace cutbce {
+
+enum : int {
+  kOk = 0,
+  kErrInvalidArg = 1,
+  kErrUnsupported = 2,
+  kErrWorkspace = 3,
+  kErrTargetRange = 4,
+  kErrTimeout = 5,
+  kErrCuda = 6,
+};
+
+enum : int { kMeanValidPositions = 0, kSum = 1, kMeanElements = 2 };
+
+constexpr int kMaxK = 128;            // target slots per position
+constexpr int kMaxDim = 256;          // feature width
+constexpr int kTileM = 128;           // stationary rows per tile = TMEM lanes
+constexpr int kGroupRows = 64;        // rows per group of v-sorted pairs
+constexpr int kMaxCtas = 256;         // upper bound of a persistent grid
+constexpr int kMaxSplits = 64;        // dH partial splits over the vocabulary
+constexpr int kTileThreads = 384;     // 12 warps: TMA, MMA, fix-up, idle, 8 epilogue
+constexpr int kEpiWarp0 = 4;
+constexpr int kNumEpiWarps = 8;
+
+// First 256 bytes of the workspace.
+struct WsHeader {
+  int status;          // first device-detected error, 0 = none
+  int n_valid;         // valid positions
+  int n_pairs;         // distinct (position, positive item) pairs
+  int pad0;
+  double loss_scale;   // s
+  float grad_scale;    // g * s
+  float pad1;
+};
+
+// Geometry of the tcgen05 tile engine for one padded feature width DP.
+template <int DP>
+struct TileCfg {
+  static_assert(DP % 64 == 0 && DP >= 64 && DP <= 256, "DP must be 64, 128, 192 or 256");
+  static constexpr int BN = DP <= 128 ? 128 : 64;          // streamed rows per tile (Z columns)
+  static constexpr int NKB = DP / 64;                        // 128-byte column blocks per row
+  static constexpr int NX = DP == 64 ? 4 : 3;                // stages of the streamed-operand ring
+  static constexpr uint32_t S_BYTES = kTileM * DP * 2;       // stationary tile
+  static constexpr uint32_t X_BYTES = BN * DP * 2;           // streamed tile
+  static constexpr uint32_t G_BYTES = kTileM * BN * 2;       // bf16 sigmoid tile
+  static constexpr int ACC_COL = 2 * BN;                     // TMEM column of the gradient accumulator
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int NUM_BARS = 2 + 2 * NX + 2 * 5 + 3;    // see the kernel for the list
+  static constexpr uint32_t SMEM_BYTES =
+      1024 + S_BYTES + NX * X_BYTES + 2 * G_BYTES + NUM_BARS * 8 + 16 + 64;
+  static_assert(ACC_COL + DP <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(SMEM_BYTES > 232448 / 2, "one CTA per SM keeps the TMEM allocation uncontended");
+};
+
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+}  // namespace cutbce

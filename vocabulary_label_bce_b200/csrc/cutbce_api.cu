@@ -1,0 +1,515 @@
+// Host side of libcutbce: argument checks, the planner (tile geometry,
+// vocabulary splits, workspace layout), TMA descriptors and the launch
+// sequence on one stream.  Everything here is plain C++ over the CUDA runtime;
+// the library allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "cutbce.h"
+#include "common.cuh"
+#include "prep_finish.cuh"
+#include "tile_engine.cuh"
+
+namespace {
+using namespace cutbce;
+
+constexpr long long kDefaultTimeoutNs = 2000000000LL;  // 2 s per wait: far above any tile's latency
+constexpr int64_t kSplitItemsTarget = 16 * 148;        // about 16 dH work items per SM of a 148-SM part
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Plan {
+  int64_t T, V, D, K;
+  int dtype, reduction;
+  int DP, BN;
+  int64_t Tpad, ngroups_max, n_vitems, n_gather_blocks;
+  int S, tps, n_vtiles_bn;
+  size_t elem;
+  size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_grp_t, o_grp_v, o_hc, o_lpart,
+      o_cpart, o_cursor, o_dhpart, total;
+};
+
+cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
+  if (p == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  if (p->T <= 0 || p->V <= 0 || p->D <= 0 || p->K <= 0) return CUTBCE_ERR_INVALID_ARG;
+  if (p->dtype != CUTBCE_BF16 && p->dtype != CUTBCE_F32) return CUTBCE_ERR_UNSUPPORTED;
+  if (p->reduction < 0 || p->reduction > 2) return CUTBCE_ERR_INVALID_ARG;
+  if (p->K > kMaxK || p->D > kMaxDim) return CUTBCE_ERR_UNSUPPORTED;
+  if (p->dtype == CUTBCE_BF16 && (p->D % 8) != 0) return CUTBCE_ERR_UNSUPPORTED;
+  if (p->V >= (int64_t(1) << 31) || p->T >= (int64_t(1) << 30) || p->T * p->K >= (int64_t(1) << 31))
+    return CUTBCE_ERR_UNSUPPORTED;
+  if (need_data) {
+    if (p->H == nullptr || p->E == nullptr || p->targets == nullptr) return CUTBCE_ERR_INVALID_ARG;
+    if (p->dtype == CUTBCE_BF16 &&
+        ((reinterpret_cast<uintptr_t>(p->H) | reinterpret_cast<uintptr_t>(p->E)) & 15) != 0)
+      return CUTBCE_ERR_INVALID_ARG;
+  }
+  return CUTBCE_OK;
+}
+
+void make_plan(const cutbce_problem* p, Plan& pl) {
+  pl.T = p->T;
+  pl.V = p->V;
+  pl.D = p->D;
+  pl.K = p->K;
+  pl.dtype = p->dtype;
+  pl.reduction = p->reduction;
+  const bool bf16 = p->dtype == CUTBCE_BF16;
+  pl.DP = bf16 ? static_cast<int>(round_up(p->D, 64)) : static_cast<int>(p->D);
+  pl.BN = (bf16 && pl.DP > 128) ? 64 : 128;
+  pl.elem = bf16 ? 2 : 4;
+  pl.Tpad = round_up(p->T, kTileM);
+  pl.ngroups_max = ceil_div(p->T, kGroupRows);
+  pl.n_vitems = ceil_div(p->V, kTileM);
+  pl.n_gather_blocks = ceil_div(pl.Tpad, 8);
+  if (bf16) {
+    pl.n_vtiles_bn = static_cast<int>(ceil_div(p->V, pl.BN));
+    const int64_t nTmax = ceil_div(p->T, kTileM);
+    int64_t s0 = ceil_div(kSplitItemsTarget, nTmax);
+    s0 = std::max<int64_t>(1, std::min<int64_t>({s0, kMaxSplits, pl.n_vtiles_bn}));
+    pl.tps = static_cast<int>(ceil_div(pl.n_vtiles_bn, s0));
+    pl.S = static_cast<int>(ceil_div(pl.n_vtiles_bn, pl.tps));  // every split is non-empty
+  } else {
+    pl.n_vtiles_bn = 0;
+    pl.tps = 0;
+    pl.S = 1;
+  }
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  const size_t TK = static_cast<size_t>(p->T) * p->K;
+  pl.o_hdr = take(256);
+  pl.o_cidx = take(4 * p->T);
+  pl.o_orig = take(4 * p->T);
+  pl.o_rowcnt = take(4 * p->T);
+  pl.o_rowptr = take(4 * (p->T + 1));
+  pl.o_ids = take(4 * TK);
+  pl.o_pair_t = take(4 * TK);
+  pl.o_pair_v = take(4 * TK);
+  pl.o_grp_t = take(4 * TK);
+  pl.o_grp_v = take(4 * TK);
+  pl.o_hc = take(pl.elem * static_cast<size_t>(pl.Tpad) * pl.DP);
+  pl.o_lpart = take(8 * kNumEpiWarps * pl.n_vitems);
+  pl.o_cpart = take(8 * pl.n_gather_blocks);
+  pl.o_cursor = take(4 * static_cast<size_t>(kMaxCtas) * pl.ngroups_max);
+  pl.o_dhpart = take(4 * static_cast<size_t>(pl.S) * pl.Tpad * pl.DP);
+  pl.total = o;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// ---------------------------------------------------------------- device facts (cached)
+struct DeviceFacts {
+  int sms = 0, major = 0, minor = 0;
+};
+DeviceFacts g_dev[64];
+std::mutex g_dev_mu;
+
+cutbce_status device_facts(DeviceFacts& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CUTBCE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_dev[dev].sms == 0) {
+    DeviceFacts f;
+    if (cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&f.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&f.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return CUTBCE_ERR_CUDA;
+    g_dev[dev] = f;
+  }
+  out = g_dev[dev];
+  return CUTBCE_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// A row-major bf16 matrix [rows, cols] with row stride `stride_elems`, read in
+// boxes of 64 columns (128 bytes, 128-byte swizzle) by `box_rows` rows.
+// Columns >= cols and rows >= rows read as zero.
+bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t stride_elems, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_elems * 2)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- tile-engine dispatch
+template <int DP, bool kLoss, bool kGrad, bool kDH>
+cudaError_t launch_tile(int grid, const CUtensorMap& s, const CUtensorMap& x, const TileParams& tp,
+                        cudaStream_t st) {
+  auto kern = k_tile<DP, kLoss, kGrad, kDH>;
+  constexpr uint32_t smem = TileCfg<DP>::SMEM_BYTES;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  kern<<<grid, kTileThreads, smem, st>>>(s, x, tp);
+  return cudaGetLastError();
+}
+
+template <bool kLoss, bool kGrad, bool kDH>
+cudaError_t launch_tile_dp(int DP, int grid, const CUtensorMap& s, const CUtensorMap& x, const TileParams& tp,
+                           cudaStream_t st) {
+  switch (DP) {
+    case 64: return launch_tile<64, kLoss, kGrad, kDH>(grid, s, x, tp, st);
+    case 128: return launch_tile<128, kLoss, kGrad, kDH>(grid, s, x, tp, st);
+    case 192: return launch_tile<192, kLoss, kGrad, kDH>(grid, s, x, tp, st);
+    case 256: return launch_tile<256, kLoss, kGrad, kDH>(grid, s, x, tp, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+struct Want {
+  bool loss, dE, dH;
+};
+
+int count_launches(const Plan& pl, Want w) {
+  const bool bf16 = pl.dtype == CUTBCE_BF16;
+  int n = 3;                                        // rows, scan, gather
+  if (bf16 && (w.dE || w.dH)) n += 1;               // group sort
+  if (w.loss || w.dE) n += 1;                       // item-owned pass
+  if (w.dH) n += 1;                                 // position-owned pass
+  if (w.loss || w.dH) n += 1;                       // finish
+  return n;
+}
+
+cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss, float* dH, float* dE, Want w,
+                  void* ws, size_t ws_bytes, cudaStream_t st) {
+  cutbce_status s = check_problem(p, true);
+  if (s != CUTBCE_OK) return s;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return CUTBCE_ERR_INVALID_ARG;
+  if (w.loss && loss == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  Plan pl;
+  make_plan(p, pl);
+  if (ws_bytes < pl.total) return CUTBCE_ERR_WORKSPACE;
+  DeviceFacts dev;
+  if ((s = device_facts(dev)) != CUTBCE_OK) return s;
+  const bool bf16 = p->dtype == CUTBCE_BF16;
+  if (bf16 && !(dev.major == 10 && dev.minor == 0)) return CUTBCE_ERR_UNSUPPORTED;
+
+  const int T = static_cast<int>(p->T), V = static_cast<int>(p->V), D = static_cast<int>(p->D),
+            K = static_cast<int>(p->K);
+  WsHeader* hdr = at<WsHeader>(ws, pl.o_hdr);
+  int* cidx = at<int>(ws, pl.o_cidx);
+  int* orig = at<int>(ws, pl.o_orig);
+  int* rowcnt = at<int>(ws, pl.o_rowcnt);
+  int* rowptr = at<int>(ws, pl.o_rowptr);
+  int* ids = at<int>(ws, pl.o_ids);
+  int* pair_t = at<int>(ws, pl.o_pair_t);
+  int* pair_v = at<int>(ws, pl.o_pair_v);
+  int* grp_t = at<int>(ws, pl.o_grp_t);
+  int* grp_v = at<int>(ws, pl.o_grp_v);
+  double* lpart = at<double>(ws, pl.o_lpart);
+  double* cpart = at<double>(ws, pl.o_cpart);
+  int* cursors = at<int>(ws, pl.o_cursor);
+  float* dhpart = at<float>(ws, pl.o_dhpart);
+
+#define CUTBCE_CK(x)                           \
+  do {                                         \
+    if ((x) != cudaSuccess) return CUTBCE_ERR_CUDA; \
+  } while (0)
+
+  CUTBCE_CK(cudaMemsetAsync(hdr, 0, 256, st));
+  k_prep_rows<<<static_cast<unsigned>(ceil_div(T, 128)), 128, 0, st>>>(p->targets, p->mask, T, K, V, ids, rowcnt,
+                                                                        hdr);
+  CUTBCE_CK(cudaGetLastError());
+  k_prep_scan<<<1, kScanThreads, 0, st>>>(p->mask, rowcnt, T, V, p->reduction, grad_loss, cidx, orig, rowptr, hdr);
+  CUTBCE_CK(cudaGetLastError());
+  if (bf16) {
+    k_prep_gather<__nv_bfloat16><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(p->H), static_cast<const __nv_bfloat16*>(p->E), D, pl.DP, K, pl.Tpad,
+        orig, ids, rowcnt, rowptr, hdr, at<__nv_bfloat16>(ws, pl.o_hc), pair_t, pair_v, cpart);
+  } else {
+    k_prep_gather<float><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
+        static_cast<const float*>(p->H), static_cast<const float*>(p->E), D, pl.DP, K, pl.Tpad, orig, ids, rowcnt,
+        rowptr, hdr, at<float>(ws, pl.o_hc), pair_t, pair_v, cpart);
+  }
+  CUTBCE_CK(cudaGetLastError());
+
+  const bool item_pass = w.loss || w.dE;
+  if (bf16) {
+    if (w.dE || w.dH) {
+      int npow = 1;
+      while (npow < kGroupRows * K) npow <<= 1;
+      const size_t smem = static_cast<size_t>(npow) * 8;
+      static bool sort_cfg = false;
+      if (!sort_cfg) {
+        CUTBCE_CK(cudaFuncSetAttribute(k_group_sort, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kGroupRows * kMaxK * 8)));
+        sort_cfg = true;
+      }
+      k_group_sort<<<static_cast<unsigned>(pl.ngroups_max), 256, smem, st>>>(rowptr, pair_t, pair_v, hdr, grp_t,
+                                                                             grp_v);
+      CUTBCE_CK(cudaGetLastError());
+    }
+    TileParams tp{};
+    tp.V = V;
+    tp.D = D;
+    tp.Tpad = pl.Tpad;
+    tp.hdr = hdr;
+    tp.row_ptr = rowptr;
+    tp.grp_v = grp_v;
+    tp.grp_t = grp_t;
+    tp.cursors = cursors;
+    tp.ngroups_max = static_cast<int>(pl.ngroups_max);
+    tp.dE = dE;
+    tp.loss_part = lpart;
+    tp.dh_part = dhpart;
+    tp.nsplit = pl.S;
+    tp.tiles_per_split = pl.tps;
+    tp.n_item_tiles_bn = pl.n_vtiles_bn;
+    tp.timeout_ns = kDefaultTimeoutNs;
+    const __nv_bfloat16* hc = at<__nv_bfloat16>(ws, pl.o_hc);
+    if (item_pass) {
+      CUtensorMap ms, mx;
+      if (!make_map(&ms, p->E, D, V, D, kTileM) || !make_map(&mx, hc, pl.DP, pl.Tpad, pl.DP, pl.BN))
+        return CUTBCE_ERR_CUDA;
+      const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(dev.sms), pl.n_vitems,
+                                                           static_cast<int64_t>(kMaxCtas)}));
+      cudaError_t e;
+      if (w.loss && w.dE) e = launch_tile_dp<true, true, false>(pl.DP, grid, ms, mx, tp, st);
+      else if (w.loss) e = launch_tile_dp<true, false, false>(pl.DP, grid, ms, mx, tp, st);
+      else e = launch_tile_dp<false, true, false>(pl.DP, grid, ms, mx, tp, st);
+      CUTBCE_CK(e);
+    }
+    if (w.dH) {
+      CUtensorMap ms, mx;
+      if (!make_map(&ms, hc, pl.DP, pl.Tpad, pl.DP, kTileM) || !make_map(&mx, p->E, D, V, D, pl.BN))
+        return CUTBCE_ERR_CUDA;
+      const int64_t items_max = static_cast<int64_t>(pl.S) * ceil_div(T, kTileM);
+      const int grid = static_cast<int>(
+          std::min<int64_t>({static_cast<int64_t>(dev.sms), items_max, static_cast<int64_t>(kMaxCtas)}));
+      CUTBCE_CK((launch_tile_dp<false, true, true>(pl.DP, grid, ms, mx, tp, st)));
+    }
+  } else {
+    const float* hc = at<float>(ws, pl.o_hc);
+    if (item_pass) {
+      k_simt_items<<<static_cast<unsigned>(pl.n_vitems), 128, 0, st>>>(
+          hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, w.dE ? dE : nullptr,
+          w.loss ? lpart : nullptr);
+      CUTBCE_CK(cudaGetLastError());
+    }
+    if (w.dH) {
+      k_simt_rows<<<static_cast<unsigned>(ceil_div(pl.Tpad, 128)), 128, 0, st>>>(
+          hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, dhpart);
+      CUTBCE_CK(cudaGetLastError());
+    }
+  }
+  if (w.loss || w.dH) {
+    const int64_t n = w.dH ? static_cast<int64_t>(T) * D : 1;
+    const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n, kFinishThreads)));
+    k_finish<<<grid, kFinishThreads, 0, st>>>(T, D, pl.DP, pl.Tpad, pl.S, cidx, dhpart, w.dH ? dH : nullptr, lpart,
+                                             static_cast<int>(pl.n_vitems * kNumEpiWarps), cpart,
+                                             static_cast<int>(pl.n_gather_blocks), w.loss ? loss : nullptr, hdr);
+    CUTBCE_CK(cudaGetLastError());
+  }
+#undef CUTBCE_CK
+  return CUTBCE_OK;
+}
+
+// Host-buffer entry: layout of the caller's device buffer.
+struct HostLayout {
+  size_t o_H, o_E, o_tg, o_mask, o_loss, o_grad, o_dH, o_dE, o_ws, total;
+};
+
+void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t a = o;
+    o = align256(o + bytes);
+    return a;
+  };
+  hl.o_H = take(pl.elem * p->T * p->D);
+  hl.o_E = take(pl.elem * p->V * p->D);
+  hl.o_tg = take(4 * p->T * p->K);
+  hl.o_mask = take(p->T);
+  hl.o_loss = take(8);
+  hl.o_grad = take(4);
+  hl.o_dH = take(4 * p->T * p->D);
+  hl.o_dE = take(4 * p->V * p->D);
+  hl.o_ws = take(pl.total);
+  hl.total = o;
+}
+
+}  // namespace
+
+extern "C" {
+
+cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes) {
+  if (bytes == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  const cutbce_status s = check_problem(prob, false);
+  if (s != CUTBCE_OK) return s;
+  Plan pl;
+  make_plan(prob, pl);
+  *bytes = pl.total;
+  return CUTBCE_OK;
+}
+
+cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_bytes, double* loss,
+                             cutbce_stream_t stream) {
+  if (loss == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false}, ws, ws_bytes,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+cutbce_status cutbce_backward(const cutbce_problem* prob, const float* grad_loss, float* dH, float* dE, void* ws,
+                              size_t ws_bytes, cutbce_stream_t stream) {
+  if (dH == nullptr && dE == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  return run(prob, grad_loss, nullptr, dH, dE, Want{false, dE != nullptr, dH != nullptr}, ws, ws_bytes,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+cutbce_status cutbce_forward_backward(const cutbce_problem* prob, const float* grad_loss, double* loss, float* dH,
+                                      float* dE, void* ws, size_t ws_bytes, cutbce_stream_t stream) {
+  if (loss == nullptr && dH == nullptr && dE == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  return run(prob, grad_loss, loss, dH, dE, Want{loss != nullptr, dE != nullptr, dH != nullptr}, ws, ws_bytes,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes) {
+  if (bytes == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  const cutbce_status s = check_problem(prob, false);
+  if (s != CUTBCE_OK) return s;
+  Plan pl;
+  make_plan(prob, pl);
+  HostLayout hl;
+  host_layout(prob, pl, hl);
+  *bytes = hl.total;
+  return CUTBCE_OK;
+}
+
+cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float grad_loss, double* loss, float* dH,
+                                           float* dE, void* dev_buf, size_t dev_bytes, cutbce_stream_t stream) {
+  cutbce_status s = check_problem(prob, true);
+  if (s != CUTBCE_OK) return s;
+  if (loss == nullptr || dev_buf == nullptr || (reinterpret_cast<uintptr_t>(dev_buf) & 255) != 0)
+    return CUTBCE_ERR_INVALID_ARG;
+  Plan pl;
+  make_plan(prob, pl);
+  HostLayout hl;
+  host_layout(prob, pl, hl);
+  if (dev_bytes < hl.total) return CUTBCE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* b = static_cast<uint8_t*>(dev_buf);
+  const size_t szH = pl.elem * prob->T * prob->D, szE = pl.elem * prob->V * prob->D;
+  if (cudaMemcpyAsync(b + hl.o_H, prob->H, szH, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(b + hl.o_E, prob->E, szE, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(b + hl.o_tg, prob->targets, 4 * prob->T * prob->K, cudaMemcpyHostToDevice, st) !=
+          cudaSuccess ||
+      (prob->mask != nullptr &&
+       cudaMemcpyAsync(b + hl.o_mask, prob->mask, prob->T, cudaMemcpyHostToDevice, st) != cudaSuccess) ||
+      cudaMemcpyAsync(b + hl.o_grad, &grad_loss, 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return CUTBCE_ERR_CUDA;
+  cutbce_problem dp = *prob;
+  dp.H = b + hl.o_H;
+  dp.E = b + hl.o_E;
+  dp.targets = reinterpret_cast<const int32_t*>(b + hl.o_tg);
+  dp.mask = prob->mask != nullptr ? reinterpret_cast<const uint8_t*>(b + hl.o_mask) : nullptr;
+  float* ddH = dH ? reinterpret_cast<float*>(b + hl.o_dH) : nullptr;
+  float* ddE = dE ? reinterpret_cast<float*>(b + hl.o_dE) : nullptr;
+  s = run(&dp, reinterpret_cast<const float*>(b + hl.o_grad), reinterpret_cast<double*>(b + hl.o_loss), ddH, ddE,
+          Want{true, dE != nullptr, dH != nullptr}, b + hl.o_ws, pl.total, st);
+  if (s != CUTBCE_OK) return s;
+  int dev_status = 0;
+  if (cudaMemcpyAsync(loss, b + hl.o_loss, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      (dH && cudaMemcpyAsync(dH, ddH, 4 * prob->T * prob->D, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
+      (dE && cudaMemcpyAsync(dE, ddE, 4 * prob->V * prob->D, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
+      cudaMemcpyAsync(&dev_status, b + hl.o_ws + pl.o_hdr, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return CUTBCE_ERR_CUDA;
+  return static_cast<cutbce_status>(dev_status);
+}
+
+cutbce_status cutbce_read_status(const void* ws, cutbce_stream_t stream) {
+  if (ws == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  int v = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return CUTBCE_ERR_CUDA;
+  return static_cast<cutbce_status>(v);
+}
+
+cutbce_status cutbce_read_counts(const cutbce_problem* prob, const void* ws, int64_t* n_valid, int64_t* n_pairs,
+                                 int32_t* row_counts, cutbce_stream_t stream) {
+  const cutbce_status s = check_problem(prob, false);
+  if (s != CUTBCE_OK) return s;
+  if (ws == nullptr || n_valid == nullptr || n_pairs == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  Plan pl;
+  make_plan(prob, pl);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader h;
+  const uint8_t* b = static_cast<const uint8_t*>(ws);
+  if (cudaMemcpyAsync(&h, b + pl.o_hdr, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return CUTBCE_ERR_CUDA;
+  if (row_counts != nullptr &&
+      cudaMemcpyAsync(row_counts, b + pl.o_rowcnt, 4 * prob->T, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return CUTBCE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return CUTBCE_ERR_CUDA;
+  *n_valid = h.n_valid;
+  *n_pairs = h.n_pairs;
+  return CUTBCE_OK;
+}
+
+int cutbce_kernel_launches(const cutbce_problem* prob, int entry) {
+  if (check_problem(prob, false) != CUTBCE_OK || entry < 0 || entry > 2) return -1;
+  Plan pl;
+  make_plan(prob, pl);
+  const Want w = entry == 0 ? Want{true, false, false} : entry == 1 ? Want{false, true, true} : Want{true, true, true};
+  return count_launches(pl, w);
+}
+
+const char* cutbce_status_string(cutbce_status s) {
+  switch (s) {
+    case CUTBCE_OK: return "ok";
+    case CUTBCE_ERR_INVALID_ARG: return "invalid argument";
+    case CUTBCE_ERR_UNSUPPORTED: return "unsupported problem or device";
+    case CUTBCE_ERR_WORKSPACE: return "workspace too small";
+    case CUTBCE_ERR_TARGET_RANGE: return "target id out of range";
+    case CUTBCE_ERR_TIMEOUT: return "bounded wait in a kernel ran out";
+    case CUTBCE_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+cutbce_status cutbce_selftest_wait_timeout(int64_t limit_ns, int32_t* status_dev, cutbce_stream_t stream) {
+  if (status_dev == nullptr || limit_ns <= 0 || limit_ns > 10000000000LL) return CUTBCE_ERR_INVALID_ARG;
+  k_selftest_wait<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, status_dev);
+  return cudaGetLastError() == cudaSuccess ? CUTBCE_OK : CUTBCE_ERR_CUDA;
+}
+
+}  // extern "C"

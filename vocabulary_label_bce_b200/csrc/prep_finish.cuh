@@ -1,0 +1,386 @@
+// CUDA-core kernels around the tensor-core engine:
+//   prep   -- apply the mask and the id rules, compact the valid rows, build the
+//             (position, item) pair lists, sum the sparse target correction;
+//   finish -- reduce the dH partials in a fixed order, scale, form the loss;
+//   simt   -- a plain fp32 path for fp32 inputs (small correctness cases).
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "common.cuh"
+
+namespace cutbce {
+
+__device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(status, 0, code); }
+
+// ------------------------------------------------------------------ prep: rows
+// One thread per position t.  A valid row's ids become its positive set P_t
+// (section III-B: sparse [B,N,L] ids, no multi-hot tensor): -1 slots dropped,
+// repeats collapsed (y is 0/1), sorted ascending.  Ids of masked rows are ignored.
+__global__ void k_prep_rows(const int32_t* __restrict__ targets, const uint8_t* __restrict__ mask, int T,
+                            int K, int V, int* __restrict__ ids_out, int* __restrict__ row_cnt,
+                            WsHeader* hdr) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const bool valid = mask == nullptr || mask[t] != 0;
+  if (!valid) {
+    row_cnt[t] = 0;
+    return;
+  }
+  int buf[kMaxK];
+  int n = 0;
+  bool bad = false;
+  const int32_t* row = targets + static_cast<int64_t>(t) * K;
+  for (int k = 0; k < K; ++k) {
+    const int id = row[k];
+    if (id == -1) continue;
+    if (id < -1 || id >= V) {
+      bad = true;
+      continue;
+    }
+    int pos = n;
+    while (pos > 0 && buf[pos - 1] > id) --pos;
+    if (pos > 0 && buf[pos - 1] == id) continue;
+    for (int j = n; j > pos; --j) buf[j] = buf[j - 1];
+    buf[pos] = id;
+    ++n;
+  }
+  if (bad) set_status(&hdr->status, kErrTargetRange);
+  int* dst = ids_out + static_cast<int64_t>(t) * K;
+  for (int j = 0; j < n; ++j) dst[j] = buf[j];
+  row_cnt[t] = n;
+}
+
+// ------------------------------------------------------------------ prep: scan
+// One block.  Exclusive scans over t of valid[t] (compacted row index c) and of
+// |P_t| (pair offsets), then the normalisation s and the gradient scale g*s.
+constexpr int kScanThreads = 1024;
+constexpr int kScanItems = 8;
+
+__global__ void __launch_bounds__(kScanThreads) k_prep_scan(const uint8_t* __restrict__ mask,
+                                                            const int* __restrict__ row_cnt, int T, int V,
+                                                            int reduction, const float* __restrict__ grad_loss,
+                                                            int* __restrict__ cidx, int* __restrict__ orig,
+                                                            int* __restrict__ row_ptr, WsHeader* hdr) {
+  __shared__ int warp_v[32], warp_c[32];
+  __shared__ int carry_v, carry_c;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) {
+    carry_v = 0;
+    carry_c = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < T; base += kScanThreads * kScanItems) {
+    int vloc[kScanItems], cloc[kScanItems];
+    int vs = 0, cs = 0;
+#pragma unroll
+    for (int i = 0; i < kScanItems; ++i) {
+      const int t = base + tid * kScanItems + i;
+      const int v = (t < T && (mask == nullptr || mask[t] != 0)) ? 1 : 0;
+      const int c = (t < T) ? row_cnt[t] : 0;
+      vloc[i] = v;
+      cloc[i] = c;
+      vs += v;
+      cs += c;
+    }
+    int vi = vs, ci = cs;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int nv = __shfl_up_sync(0xffffffffu, vi, off);
+      const int nc = __shfl_up_sync(0xffffffffu, ci, off);
+      if (lane >= off) {
+        vi += nv;
+        ci += nc;
+      }
+    }
+    if (lane == 31) {
+      warp_v[wid] = vi;
+      warp_c[wid] = ci;
+    }
+    __syncthreads();
+    if (wid == 0) {
+      int a = warp_v[lane], b = warp_c[lane];
+      int ai = a, bi = b;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int na = __shfl_up_sync(0xffffffffu, ai, off);
+        const int nb = __shfl_up_sync(0xffffffffu, bi, off);
+        if (lane >= off) {
+          ai += na;
+          bi += nb;
+        }
+      }
+      warp_v[lane] = ai - a;
+      warp_c[lane] = bi - b;
+    }
+    __syncthreads();
+    int vex = carry_v + warp_v[wid] + vi - vs;
+    int cex = carry_c + warp_c[wid] + ci - cs;
+    __syncthreads();  // everyone has read carry_*
+#pragma unroll
+    for (int i = 0; i < kScanItems; ++i) {
+      const int t = base + tid * kScanItems + i;
+      if (t < T) {
+        if (vloc[i]) {
+          cidx[t] = vex;
+          orig[vex] = t;
+          row_ptr[vex] = cex;
+          ++vex;
+        } else {
+          cidx[t] = -1;
+        }
+        cex += cloc[i];
+      }
+    }
+    if (tid == kScanThreads - 1) {
+      carry_v = vex;
+      carry_c = cex;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const int nv = carry_v;
+    row_ptr[nv] = carry_c;
+    hdr->n_valid = nv;
+    hdr->n_pairs = carry_c;
+    double s = 0.0;
+    if (nv > 0) {
+      if (reduction == kMeanValidPositions) s = 1.0 / nv;
+      else if (reduction == kSum) s = 1.0;
+      else s = 1.0 / (static_cast<double>(nv) * static_cast<double>(V));
+    }
+    const double g = grad_loss ? static_cast<double>(*grad_loss) : 1.0;
+    hdr->loss_scale = s;
+    hdr->grad_scale = static_cast<float>(g * s);
+  }
+}
+
+// ------------------------------------------------------------------ prep: gather
+// One warp per compacted row c in [0, Tpad).  Copies h_t into the compacted,
+// zero-padded H_c (rows >= n_valid are zero so padded tiles contribute exactly
+// nothing to any gradient), writes the pair lists, and sums the sparse target
+// correction sum_{v in P_t} h_t . e_v of Eq. (2) in fp32 per pair, in a fixed
+// order, into one double per block.
+template <typename TIn>
+__global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, const TIn* __restrict__ E,
+                                                     int D, int DP, int K, int64_t Tpad,
+                                                     const int* __restrict__ orig, const int* __restrict__ ids,
+                                                     const int* __restrict__ row_cnt,
+                                                     const int* __restrict__ row_ptr, const WsHeader* hdr,
+                                                     TIn* __restrict__ Hc, int* __restrict__ pair_t,
+                                                     int* __restrict__ pair_v, double* __restrict__ corr_part) {
+  __shared__ double wsum[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  const int nv = hdr->n_valid;
+  double acc = 0.0;
+  if (c < Tpad) {
+    TIn* dst = Hc + c * DP;
+    if (c < nv) {
+      const int t = orig[c];
+      const TIn* src = H + static_cast<int64_t>(t) * D;
+      for (int d = lane; d < DP; d += 32) dst[d] = d < D ? src[d] : TIn(0.0f);
+      const int p0 = row_ptr[c];
+      const int n = row_cnt[t];
+      for (int k = 0; k < n; ++k) {
+        const int v = ids[static_cast<int64_t>(t) * K + k];
+        if (lane == 0) {
+          pair_t[p0 + k] = static_cast<int>(c);
+          pair_v[p0 + k] = v;
+        }
+        const TIn* e = E + static_cast<int64_t>(v) * D;
+        float z = 0.f;
+        for (int d = lane; d < D; d += 32) z = fmaf(static_cast<float>(src[d]), static_cast<float>(e[d]), z);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+        acc += static_cast<double>(z);
+      }
+    } else {
+      for (int d = lane; d < DP; d += 32) dst[d] = TIn(0.0f);
+    }
+  }
+  if (lane == 0) wsum[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int w = 0; w < 8; ++w) s += wsum[w];
+    corr_part[blockIdx.x] = s;
+  }
+}
+
+// ------------------------------------------------------------------ prep: group sort
+// One block per group of 64 compacted rows: sorts the group's pairs by
+// (item, position) so that the tile engine can walk, for any range of items,
+// the positives that fall inside a tile with a forward-only cursor.
+__global__ void __launch_bounds__(256) k_group_sort(const int* __restrict__ row_ptr,
+                                                    const int* __restrict__ pair_t,
+                                                    const int* __restrict__ pair_v, const WsHeader* hdr,
+                                                    int* __restrict__ grp_t, int* __restrict__ grp_v) {
+  extern __shared__ unsigned long long keys[];
+  const int nv = hdr->n_valid;
+  const int r0 = blockIdx.x * kGroupRows;
+  if (r0 >= nv) return;
+  const int r1 = min(r0 + kGroupRows, nv);
+  const int p0 = row_ptr[r0], p1 = row_ptr[r1];
+  const int n = p1 - p0;
+  if (n == 0) return;
+  int npow = 1;
+  while (npow < n) npow <<= 1;
+  for (int i = threadIdx.x; i < npow; i += blockDim.x)
+    keys[i] = i < n ? ((static_cast<unsigned long long>(pair_v[p0 + i]) << 32) |
+                       static_cast<unsigned int>(pair_t[p0 + i]))
+                    : ~0ull;
+  __syncthreads();
+  for (int k = 2; k <= npow; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < npow; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const bool up = (i & k) == 0;
+          const unsigned long long a = keys[i], b = keys[ixj];
+          if ((a > b) == up) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    grp_v[p0 + i] = static_cast<int>(keys[i] >> 32);
+    grp_t[p0 + i] = static_cast<int>(keys[i] & 0xffffffffu);
+  }
+}
+
+// ------------------------------------------------------------------ finish
+// dH[t, d] = g*s * sum_{split} partial[split][c(t)][d] in split order (0 for
+// masked rows); the last block also forms loss = s * (dense - correction),
+// both sums taken in a fixed order.
+constexpr int kFinishThreads = 256;
+
+__device__ double block_sum_fixed(double v, double* red) {
+  // deterministic: contiguous per-thread values, then a fixed tree
+  red[threadIdx.x] = v;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  const double r = red[0];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kFinishThreads) k_finish(
+    int T, int D, int DP, int64_t Tpad, int S, const int* __restrict__ cidx,
+    const float* __restrict__ dh_part, float* __restrict__ dH, const double* __restrict__ loss_part,
+    int n_loss_part, const double* __restrict__ corr_part, int n_corr_part, double* __restrict__ loss,
+    const WsHeader* hdr) {
+  __shared__ double red[kFinishThreads];
+  const float gs = hdr->grad_scale;
+  if (dH != nullptr) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx < static_cast<int64_t>(T) * D) {
+      const int t = static_cast<int>(idx / D);
+      const int d = static_cast<int>(idx - static_cast<int64_t>(t) * D);
+      const int c = cidx[t];
+      float out = 0.f;
+      if (c >= 0) {
+        float acc = 0.f;
+        for (int s = 0; s < S; ++s) acc += dh_part[(static_cast<int64_t>(s) * Tpad + c) * DP + d];
+        out = acc * gs;
+      }
+      dH[idx] = out;
+    }
+  }
+  if (loss != nullptr && blockIdx.x == gridDim.x - 1) {
+    double a = 0.0, b = 0.0;
+    const int per_a = (n_loss_part + blockDim.x - 1) / blockDim.x;
+    for (int i = threadIdx.x * per_a; i < min(n_loss_part, (threadIdx.x + 1) * per_a); ++i) a += loss_part[i];
+    const int per_b = (n_corr_part + blockDim.x - 1) / blockDim.x;
+    for (int i = threadIdx.x * per_b; i < min(n_corr_part, (threadIdx.x + 1) * per_b); ++i) b += corr_part[i];
+    const double dense = block_sum_fixed(a, red);
+    const double corr = block_sum_fixed(b, red);
+    if (threadIdx.x == 0) *loss = hdr->n_valid > 0 ? hdr->loss_scale * (dense - corr) : 0.0;
+  }
+}
+
+// ------------------------------------------------------------------ fp32 CUDA-core path
+__device__ __forceinline__ float sigmoid_f32(float z) {
+  if (z >= 0.f) return 1.f / (1.f + expf(-z));
+  const float e = expf(z);
+  return e / (1.f + e);
+}
+
+// One thread per item v (blocks of 128 items, matching the tensor-core path's
+// item tiles): the dense loss sum over valid positions and dE_v = g s sum_t (s(x)-y) h_t.
+__global__ void __launch_bounds__(128) k_simt_items(const float* __restrict__ Hc, const float* __restrict__ E,
+                                                    int V, int D, const int* __restrict__ row_ptr,
+                                                    const int* __restrict__ pair_v, const WsHeader* hdr,
+                                                    float* __restrict__ dE, double* __restrict__ loss_part) {
+  __shared__ double red[128];
+  const int v = blockIdx.x * 128 + threadIdx.x;
+  const int nv = hdr->n_valid;
+  const float gs = hdr->grad_scale;
+  double lsum = 0.0;
+  float acc[kMaxDim];
+  if (v < V) {
+    for (int d = 0; d < D; ++d) acc[d] = 0.f;
+    const float* e = E + static_cast<int64_t>(v) * D;
+    for (int c = 0; c < nv; ++c) {
+      const float* h = Hc + static_cast<int64_t>(c) * D;
+      float z = 0.f;
+      for (int d = 0; d < D; ++d) z = fmaf(h[d], e[d], z);
+      float y = 0.f;
+      for (int p = row_ptr[c]; p < row_ptr[c + 1]; ++p) y = pair_v[p] == v ? 1.f : y;
+      lsum += static_cast<double>(fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))));
+      if (dE != nullptr) {
+        const float g = sigmoid_f32(z) - y;
+        for (int d = 0; d < D; ++d) acc[d] = fmaf(g, h[d], acc[d]);
+      }
+    }
+    if (dE != nullptr)
+      for (int d = 0; d < D; ++d) dE[static_cast<int64_t>(v) * D + d] = acc[d] * gs;
+  }
+  if (loss_part != nullptr) {
+    // same layout as the tensor-core path: kNumEpiWarps partials per 128-item tile
+    const double s = block_sum_fixed(v < V ? lsum : 0.0, red);
+    if (threadIdx.x < kNumEpiWarps) loss_part[static_cast<int64_t>(blockIdx.x) * kNumEpiWarps + threadIdx.x] = threadIdx.x == 0 ? s : 0.0;
+  }
+}
+
+// One thread per compacted row c: dH partial sum_v (s(x)-y) e_v over all items.
+__global__ void __launch_bounds__(128) k_simt_rows(const float* __restrict__ Hc, const float* __restrict__ E,
+                                                   int V, int D, const int* __restrict__ row_ptr,
+                                                   const int* __restrict__ pair_v, const WsHeader* hdr,
+                                                   float* __restrict__ dh_part) {
+  const int c = blockIdx.x * 128 + threadIdx.x;
+  if (c >= hdr->n_valid) return;
+  float acc[kMaxDim];
+  for (int d = 0; d < D; ++d) acc[d] = 0.f;
+  const float* h = Hc + static_cast<int64_t>(c) * D;
+  int p = row_ptr[c];
+  const int pend = row_ptr[c + 1];
+  for (int v = 0; v < V; ++v) {
+    const float* e = E + static_cast<int64_t>(v) * D;
+    float z = 0.f;
+    for (int d = 0; d < D; ++d) z = fmaf(h[d], e[d], z);
+    float y = 0.f;
+    if (p < pend && pair_v[p] == v) {
+      y = 1.f;
+      ++p;
+    }
+    const float g = sigmoid_f32(z) - y;
+    for (int d = 0; d < D; ++d) acc[d] = fmaf(g, e[d], acc[d]);
+  }
+  for (int d = 0; d < D; ++d) dh_part[static_cast<int64_t>(c) * D + d] = acc[d];
+}
+
+// Zero a float buffer (used for dE when no position is valid).
+__global__ void k_zero_f32(float* __restrict__ p, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = 0.f;
+}
+
+}  // namespace cutbce

@@ -1,0 +1,585 @@
+// The tensor-core engine: one persistent, warp-specialised sm_100a kernel
+// template that forms logit tiles on tcgen05 (accumulators in tensor memory),
+// applies the BCE element math to them in registers and, for the gradient,
+// feeds the bf16 tile of G = sigmoid(X) - Y straight back into a second
+// tcgen05 contraction.  No logit or gradient tile ever leaves the SM.
+//
+// Two instantiations cover the hot path of "Cut Binary Cross Entropy"
+// (section III-A Eqs. (2)-(3); section III-B Eq. (4)):
+//
+//   item-owned pass (kDH = false): a CTA owns a tile of 128 items v (rows of E,
+//     the stationary operand) and streams every tile of the compacted H.
+//     Z^T = E_v H_t^T  -> softplus sum (loss) and sigmoid -> G^T (bf16, smem)
+//     dE_v += G^T H_t  (accumulated in TMEM across all t, written once, no atomics)
+//
+//   position-owned pass (kDH = true): a CTA owns a tile of 128 valid positions
+//     (rows of H) and streams the item tiles of one vocabulary split.
+//     Z = H_t E_v^T    -> sigmoid -> G (bf16, smem)
+//     dH_t += G E_v    (partial per split, reduced later in a fixed order)
+//
+// The sparse targets enter in-tile: after the epilogue warps write sigmoid(z)
+// for a tile, a fix-up warp subtracts 1 at the (at most a few) positions of the
+// tile where y = 1, walking lists of pairs pre-sorted by item.  The dense loss
+// term uses no Y at all (Eq. (2): l(x,y) = l(x,0) - y x); the -y x part is the
+// separate sparse correction summed in the prep kernel.
+//
+// Warp roles (384 threads, one CTA per SM):
+//   warp 0      TMA producer (stationary tile, ring of streamed tiles)
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 2      fix-up warp (Y in-tile)
+//   warp 3      idle
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4).. and one half of
+//               the tile's columns
+//
+// Every wait is bounded (global timer); on expiry the CTA records
+// CUTBCE_ERR_TIMEOUT in the status word, the other roles leave their loops, the
+// producer and the MMA issuer wait (bounded) for their own copies and MMAs in
+// flight, and the CTA frees its tensor memory and returns.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace cutbce {
+
+struct TileParams {
+  int V;                       // items
+  int D;                       // real feature width (<= DP)
+  int64_t Tpad;                // rows of H_c (multiple of 128)
+  WsHeader* hdr;               // n_valid, grad scale, status
+  const int* row_ptr;          // [n_valid + 1] pair offsets of compacted rows
+  const int* grp_v;            // pairs sorted by (item, position) inside 64-row groups
+  const int* grp_t;
+  int* cursors;                // item-owned pass: [gridDim.x * ngroups_max] fix-up cursors
+  int ngroups_max;
+  float* dE;                   // item-owned pass output [V, D] (may be null when no gradient)
+  double* loss_part;           // item-owned pass: one double per (item tile, epilogue warp)
+  float* dh_part;              // position-owned pass output [S, Tpad, DP]
+  int nsplit;                  // position-owned pass: vocabulary splits S
+  int tiles_per_split;         // streamed item tiles per split
+  int n_item_tiles_bn;         // ceil(V / BN)
+  long long timeout_ns;
+};
+
+struct WaitCtx {
+  volatile int* abort_flag;
+  int* status;
+  long long limit;
+};
+
+// Bounded wait for phase `parity` of `bar`.  Returns false if the CTA aborted
+// or the limit ran out (then it records the timeout and raises the abort flag).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*w.abort_flag) return false;
+    if (static_cast<long long>(global_timer_ns() - t0) > w.limit) {
+      *w.abort_flag = 1;
+      atomicCAS(w.status, 0, kErrTimeout);
+      return false;
+    }
+  }
+}
+// Bounded wait that ignores the abort flag (used to drain in-flight copies/MMAs).
+__device__ __forceinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity, long long limit) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (static_cast<long long>(global_timer_ns() - t0) > limit) return false;
+  }
+  return true;
+}
+// Whole-warp wait with a warp-uniform result.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const bool ok = wait_bar(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+struct ItemInfo {
+  int s_row0;     // first stationary row
+  int x_tile0;    // first streamed tile (in units of BN rows)
+  int n_x;        // streamed tiles
+  int split;      // position-owned pass: vocabulary split
+};
+
+template <int DP, bool kDH>
+__device__ __forceinline__ ItemInfo item_info(int i, int n_valid, const TileParams& p) {
+  using Cfg = TileCfg<DP>;
+  ItemInfo it;
+  if (!kDH) {
+    it.s_row0 = i * kTileM;
+    it.x_tile0 = 0;
+    it.n_x = static_cast<int>(ceil_div(n_valid, Cfg::BN));
+    it.split = 0;
+  } else {
+    const int nT = static_cast<int>(ceil_div(n_valid, kTileM));
+    const int s = i / nT, m = i - s * nT;
+    it.s_row0 = m * kTileM;
+    it.x_tile0 = s * p.tiles_per_split;
+    it.n_x = min(p.tiles_per_split, p.n_item_tiles_bn - it.x_tile0);
+    it.split = s;
+  }
+  return it;
+}
+
+// Walk the v-sorted pairs of one 64-row group from cursor `cur` (warp-uniform):
+// first skip items < lo, then apply every pair with item in [lo, hi) to the G
+// tile by subtracting 1 (y = 1) from the stored bf16 value.
+template <bool kDH>
+__device__ __forceinline__ int fixup_walk(int cur, int end, int lo, int hi, int x0, int s0, uint8_t* G,
+                                          const int* __restrict__ grp_v, const int* __restrict__ grp_t,
+                                          int lane) {
+  while (true) {
+    const int idx = cur + lane;
+    const int v = idx < end ? __ldg(grp_v + idx) : 0x7fffffff;
+    const unsigned m = __ballot_sync(0xffffffffu, v < lo);
+    cur += __popc(m);
+    if (m != 0xffffffffu) break;
+  }
+  while (true) {
+    const int idx = cur + lane;
+    const int v = idx < end ? __ldg(grp_v + idx) : 0x7fffffff;
+    const bool in = v < hi;
+    if (in) {
+      const int t = __ldg(grp_t + idx);
+      // item-owned: rows are items, columns are positions; position-owned: the reverse
+      const int row = kDH ? (t - s0) : (v - s0);
+      const int col = kDH ? (v - x0) : (t - x0);
+      const uint32_t off = static_cast<uint32_t>(col >> 6) * 16384u + static_cast<uint32_t>(row) * 128u +
+                           ((((static_cast<uint32_t>(col) & 63u) >> 3) ^ (static_cast<uint32_t>(row) & 7u)) << 4) +
+                           ((static_cast<uint32_t>(col) & 7u) << 1);
+      __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(G + off);
+      *e = __float2bfloat16_rn(__bfloat162float(*e) - 1.0f);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, in);
+    cur += __popc(m);
+    if (m != 0xffffffffu) break;
+  }
+  return cur;
+}
+
+template <int DP, bool kLoss, bool kGrad, bool kDH>
+__global__ void __launch_bounds__(kTileThreads, 1)
+    k_tile(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmX, TileParams p) {
+  using Cfg = TileCfg<DP>;
+  constexpr int BN = Cfg::BN;
+  constexpr int NKB = Cfg::NKB;
+  constexpr int NX = Cfg::NX;
+  constexpr uint32_t S_BYTES = Cfg::S_BYTES, X_BYTES = Cfg::X_BYTES, G_BYTES = Cfg::G_BYTES;
+  constexpr int ACC_COL = Cfg::ACC_COL;
+  static_assert(!kDH || (kGrad && !kLoss), "the position-owned pass computes dH only");
+  static_assert(kLoss || kGrad, "nothing to do");
+  constexpr float kLog2e = 1.4426950408889634f;
+  constexpr float kLn2 = 0.6931471805599453f;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sS = smem;
+  uint8_t* sX = sS + S_BYTES;
+  uint8_t* sG = sX + NX * X_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + 2 * G_BYTES);
+  uint64_t* bar_sfull = bars + 0;
+  uint64_t* bar_sempty = bars + 1;
+  uint64_t* bar_xfull = bars + 2;
+  uint64_t* bar_xempty = bars + 2 + NX;
+  uint64_t* bar_zfull = bars + 2 + 2 * NX;
+  uint64_t* bar_zempty = bar_zfull + 2;
+  uint64_t* bar_gwritten = bar_zfull + 4;
+  uint64_t* bar_gfull = bar_zfull + 6;
+  uint64_t* bar_gempty = bar_zfull + 8;
+  uint64_t* bar_accfull = bar_zfull + 10;
+  uint64_t* bar_accempty = bar_zfull + 11;
+  uint64_t* bar_drain = bar_zfull + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  WsHeader* hdr = p.hdr;
+  // read the header once so every thread takes the same early-exit decision
+  __shared__ int s_status, s_nvalid;
+  if (threadIdx.x == 0) {
+    s_status = *reinterpret_cast<volatile int*>(&hdr->status);
+    s_nvalid = hdr->n_valid;
+  }
+  __syncthreads();
+  if (s_status != 0) return;  // an earlier step failed
+  const int n_valid = s_nvalid;
+  const int n_items = kDH ? p.nsplit * static_cast<int>(ceil_div(n_valid, kTileM))
+                          : static_cast<int>(ceil_div(p.V, kTileM));
+
+  if (!kDH && n_valid == 0) {
+    // no valid position: dE = 0 and every item's loss is 0
+    for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
+      if (kLoss && threadIdx.x < kNumEpiWarps) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + threadIdx.x] = 0.0;
+      if (kGrad && p.dE != nullptr) {
+        const int64_t r0 = static_cast<int64_t>(i) * kTileM;
+        const int64_t r1 = min(static_cast<int64_t>(p.V), r0 + kTileM);
+        for (int64_t k = r0 * p.D + threadIdx.x; k < r1 * p.D; k += blockDim.x) p.dE[k] = 0.f;
+      }
+    }
+    return;
+  }
+  if (static_cast<int>(blockIdx.x) >= n_items) return;
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_sempty, 1);
+    for (int s = 0; s < NX; ++s) {
+      mbar_init(bar_xfull + s, 1);
+      mbar_init(bar_xempty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_zfull + b, 1);
+      mbar_init(bar_zempty + b, kNumEpiWarps);
+      mbar_init(bar_gwritten + b, kNumEpiWarps);
+      mbar_init(bar_gfull + b, 1);
+      mbar_init(bar_gempty + b, 1);
+    }
+    mbar_init(bar_accfull, 1);
+    mbar_init(bar_accempty, kNumEpiWarps);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmS);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtx wc{abort_flag, &hdr->status, p.timeout_ns};
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      uint32_t ic = 0, xc = 0;
+      for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++ic) {
+        const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
+        if (!wait_bar(bar_sempty, (ic & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(bar_sfull, S_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < NKB; ++kb)
+          tma_load_2d(sS + kb * (kTileM * 128), &tmS, kb * 64, it.s_row0, bar_sfull);
+        bool ok = true;
+        for (int j = 0; j < it.n_x; ++j, ++xc) {
+          const uint32_t st = xc % NX;
+          if (!wait_bar(bar_xempty + st, ((xc / NX) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_xfull + st, X_BYTES);
+          const int row0 = (it.x_tile0 + j) * BN;
+#pragma unroll
+          for (int kb = 0; kb < NKB; ++kb)
+            tma_load_2d(sX + st * X_BYTES + kb * (BN * 128), &tmX, kb * 64, row0, bar_xfull + st);
+        }
+        if (!ok) {
+          ++ic;
+          break;
+        }
+      }
+      // wait (bounded) for every copy this thread issued to land
+      const long long lim = p.timeout_ns;
+      if (ic > 0) wait_bar_drain(bar_sfull, (ic - 1) & 1, lim);
+      for (uint32_t st = 0; st < NX; ++st) {
+        const uint32_t issued = xc > st ? (xc - st + NX - 1) / NX : 0;
+        if (issued > 0) wait_bar_drain(bar_xfull + st, (issued - 1) & 1, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_z = idesc_bf16_f32(kTileM, BN, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(kTileM, DP, false, true);
+      const uint32_t sS_a = smem_u32(sS), sX_a = smem_u32(sX), sG_a = smem_u32(sG);
+      uint32_t ic = 0, cnt = 0;
+      bool ok = true;
+      // Z[b] = S * X[st]^T : both operands K-major, 128-byte swizzle
+      auto issue_z = [&](uint32_t c) -> bool {
+        const uint32_t st = c % NX, b = c & 1;
+        if (!wait_bar(bar_xfull + st, (c / NX) & 1, wc)) return false;
+        if (!wait_bar(bar_zempty + b, ((c >> 1) & 1) ^ 1, wc)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DP / 16; ++ks) {
+          const uint64_t a = smem_desc_sw128(sS_a + (ks >> 2) * (kTileM * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sX_a + st * X_BYTES + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
+          umma_bf16(tmem_base + b * BN, a, bd, idesc_z, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_zfull + b);
+        if (!kGrad) umma_commit(bar_xempty + st);
+        return true;
+      };
+      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ic) {
+        const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
+        const int n = it.n_x;
+        if (!wait_bar(bar_sfull, ic & 1, wc)) break;
+        tc_fence_after();
+        if (!issue_z(cnt)) break;
+        for (int j = 0; j < n; ++j) {
+          const uint32_t c = cnt + j;
+          if (j + 1 < n) {
+            if (!issue_z(c + 1)) {
+              ok = false;
+              break;
+            }
+          } else {
+            umma_commit(bar_sempty);
+          }
+          if (kGrad) {
+            const uint32_t b = c & 1, st = c % NX;
+            if (!wait_bar(bar_gfull + b, (c >> 1) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (j == 0) {
+              if (!wait_bar(bar_accempty, (ic & 1) ^ 1, wc)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            // ACC += G[b] * X[st] : G K-major, X read MN-major (its rows are the K index)
+#pragma unroll
+            for (int ks = 0; ks < BN / 16; ++ks) {
+              const uint64_t a = smem_desc_sw128(sG_a + b * G_BYTES + (ks >> 2) * (kTileM * 128) + (ks & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(sX_a + st * X_BYTES + ks * 2048, BN * 128, 1024);
+              umma_bf16(tmem_base + ACC_COL, a, bd, idesc_acc, (j > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(bar_gempty + b);
+            umma_commit(bar_xempty + st);
+          }
+        }
+        if (!ok) break;
+        if (kGrad) umma_commit(bar_accfull);
+        cnt += n;
+      }
+      // every MMA this thread issued has completed once the drain barrier flips
+      umma_commit(bar_drain);
+      wait_bar_drain(bar_drain, 0, p.timeout_ns);
+    }
+  } else if (warp == 2) {
+    // ============================================================ Y fix-up warp
+    if (kGrad) {
+      int* curs = p.cursors + static_cast<int64_t>(blockIdx.x) * p.ngroups_max;
+      const int n_groups = static_cast<int>(ceil_div(n_valid, kGroupRows));
+      if (!kDH) {
+        for (int g = lane; g < n_groups; g += 32) curs[g] = p.row_ptr[g * kGroupRows];
+        __syncwarp();
+      }
+      uint32_t cnt = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x) {
+        const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
+        // position-owned pass: the two groups of the stationary 128 positions, cursors in registers
+        int c0 = 0, e0 = 0, c1 = 0, e1 = 0;
+        if (kDH) {
+          const int g0 = it.s_row0 / kGroupRows;
+          c0 = p.row_ptr[g0 * kGroupRows];
+          e0 = p.row_ptr[min(g0 * kGroupRows + kGroupRows, n_valid)];
+          c1 = e0;
+          e1 = p.row_ptr[min(g0 * kGroupRows + 2 * kGroupRows, n_valid)];
+        }
+        for (int j = 0; j < it.n_x; ++j) {
+          const uint32_t c = cnt + j, b = c & 1;
+          if (!wait_bar_warp(bar_gwritten + b, (c >> 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          uint8_t* G = sG + b * G_BYTES;
+          if (!kDH) {
+            const int t0 = j * BN;
+            const int v0 = it.s_row0;
+            for (int g = t0 / kGroupRows; g < (t0 + BN) / kGroupRows && g < n_groups; ++g) {
+              const int end = p.row_ptr[min(g * kGroupRows + kGroupRows, n_valid)];
+              const int cur = fixup_walk<false>(curs[g], end, v0, v0 + kTileM, t0, v0, G, p.grp_v, p.grp_t, lane);
+              __syncwarp();
+              if (lane == 0) curs[g] = cur;
+              __syncwarp();
+            }
+          } else {
+            const int v0 = (it.x_tile0 + j) * BN;
+            const int t0 = it.s_row0;
+            c0 = fixup_walk<true>(c0, e0, v0, v0 + BN, v0, t0, G, p.grp_v, p.grp_t, lane);
+            c1 = fixup_walk<true>(c1, e1, v0, v0 + BN, v0, t0, G, p.grp_v, p.grp_t, lane);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_gfull + b);
+        }
+        cnt += it.n_x;
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ============================================================ epilogue
+    const int q = warp & 3;                       // TMEM lane quarter
+    const int hh = (warp - kEpiWarp0) >> 2;       // column half
+    const int row = q * 32 + lane;                // stationary row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t sG_a = smem_u32(sG);
+    const float gs = hdr->grad_scale;
+    uint32_t cnt = 0, ic = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ic) {
+      const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
+      const int n = it.n_x;
+      double item_acc = 0.0;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t c = cnt + j, b = c & 1;
+        if (!wait_bar_warp(bar_zfull + b, (c >> 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (kGrad) {
+          if (!wait_bar_warp(bar_gempty + b, ((c >> 1) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+        }
+        const uint32_t zaddr = tmem_base + lane_base + b * BN + hh * (BN / 2);
+        const uint32_t grow = sG_a + b * G_BYTES + row * 128;
+        float tile_mx = 0.f, tile_l2 = 0.f;
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 64; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(zaddr + ch * 32, r);
+          tmem_ld_wait();
+          if (ch == BN / 64 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_zempty + b);
+          }
+          uint32_t pk[16];
+          float prod = 1.f;
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float gpair[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const float z = __uint_as_float(r[e + k]);
+              if (kLoss) {
+                const float u = ex2_approx(-fabsf(z) * kLog2e);   // e^{-|z|}
+                const float pz = 1.f + u;
+                prod *= pz;                                        // log1p batched: one lg2 per 32
+                tile_mx += fmaxf(z, 0.f);
+                if (kGrad) {
+                  const float rp = rcp_approx(pz);                 // 1 / (1 + e^{-|z|})
+                  gpair[k] = z >= 0.f ? rp : u * rp;               // sigmoid(z)
+                }
+              } else {
+                gpair[k] = fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);  // sigmoid(z)
+              }
+            }
+            if (kGrad) pk[e >> 1] = pack_bf16x2(gpair[0], gpair[1]);
+          }
+          if (kLoss) tile_l2 += lg2_approx(prod);
+          if (kGrad) {
+            const int col0 = hh * (BN / 2) + ch * 32;
+            const uint32_t base = grow + (col0 >> 6) * (kTileM * 128);
+            const uint32_t j0 = (col0 & 63) >> 3;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              st_shared_v4(base + (((j0 + k) ^ (row & 7)) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
+                           pk[4 * k + 3]);
+          }
+        }
+        if (kGrad) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_gwritten + b);
+        }
+        if (kLoss) {
+          if (j == n - 1) {
+            // zero rows of H_c past n_valid give z = 0 exactly: each adds log2(2) = 1 to tile_l2
+            const int t0 = j * BN;
+            const int lo = hh * (BN / 2), hi = lo + BN / 2;
+            const int pad = hi - max(min(n_valid - t0, hi), lo);
+            tile_l2 -= static_cast<float>(pad);
+          }
+          item_acc += static_cast<double>(tile_mx + tile_l2 * kLn2);
+        }
+      }
+      if (!ok) break;
+      if (kLoss) {
+        // one partial per (item tile, epilogue warp): no cross-warp barrier, fixed summation order
+        double val = (it.s_row0 + row < p.V) ? item_acc : 0.0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
+        if (lane == 0) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + (warp - kEpiWarp0)] = val;
+      }
+      if (kGrad) {
+        if (!wait_bar_warp(bar_accfull, ic & 1, wc)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int ch = 0; ch < DP / 64; ++ch) {
+          uint32_t r[32];
+          const int col0 = hh * (DP / 2) + ch * 32;
+          tmem_ld32(tmem_base + lane_base + ACC_COL + col0, r);
+          tmem_ld_wait();
+          if (!kDH) {
+            const int v = it.s_row0 + row;
+            if (v < p.V && p.dE != nullptr) {
+              float* dst = p.dE + static_cast<int64_t>(v) * p.D + col0;
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                if (col0 + e < p.D)
+                  *reinterpret_cast<float4*>(dst + e) =
+                      make_float4(__uint_as_float(r[e]) * gs, __uint_as_float(r[e + 1]) * gs,
+                                  __uint_as_float(r[e + 2]) * gs, __uint_as_float(r[e + 3]) * gs);
+            }
+          } else {
+            float* dst = p.dh_part + (static_cast<int64_t>(it.split) * p.Tpad + it.s_row0 + row) * DP + col0;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                                                __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_accempty);
+      }
+      cnt += n;
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// A deliberately unsignalled barrier: the bounded wait must give up, record the
+// timeout and return.  Used only by cutbce_selftest_wait_timeout.
+__global__ void k_selftest_wait(long long limit_ns, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *status = 0;
+    const WaitCtx wc{&abort_flag, status, limit_ns};
+    if (!wait_bar(&bar, 0, wc)) {
+      if (*status == 0) *status = kErrTimeout;
+    }
+  }
+}
+
+}  // namespace cutbce
