@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of the fused large-vocabulary BCE loss + gradient on B200.
+
+One step = one call of cutbce_forward_backward (loss, dH, dE) over one batch
+of synthetic input shaped like the multi-label SASRec head of "Cut Binary
+Cross Entropy" (B=64, N=200, D=64, V=876,000 items, Poisson(3) positives per
+position drawn Zipf(1.05), 20% trailing padding).  Inputs are resident in HBM
+when the timed region starts; L2 is flushed (a 256 MiB write) before every
+timed step, outside the step's event pair.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line.  Under torchrun every rank runs its own independent batch
+(replicas, weak scaling, no collective on the data path); the step time is the
+max over ranks.  --impl reference times the float64 CPU oracle on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "fused BCE fwd+bwd tokens/s at V=876k,D=64 on 1 B200; % of roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+TILE_SOURCES = ["tile_engine.cuh", "common.cuh", "ptx_sm100.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="sasrec_876k")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-items", type=int, default=16384)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def tile_source_sha():
+    h = hashlib.sha256()
+    for name in TILE_SOURCES:
+        with open(os.path.join(ROOT, "vocabulary_label_bce_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entries = json.load(f)
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_sha") == tile_source_sha():
+            return e.get("dram_bytes_per_launch")
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def sample_problem(p, n_items):
+    """The first n_items items (columns) of a drawn problem: ids outside become empty slots."""
+    E = p.E[:n_items]
+    tg = np.where(p.targets < n_items, p.targets, -1).astype(np.int32)
+    return E, tg
+
+
+def time_oracle_sample(p, n_items):
+    from oracle import cutbce_oracle as O
+    E, tg = sample_problem(p, n_items)
+    t0 = time.perf_counter()
+    O.forward_backward(p.H, E, tg, p.mask, reduction=O.MEAN_VALID_POSITIONS)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def workload_config(p, n_valid, world, l2_note):
+    return {"workload": p.name, "B": p.B, "N": p.N, "T": p.T, "n_valid": n_valid, "V": p.V, "D": p.D, "K": p.K,
+            "inputs": "bf16 H, E; int32 targets; uint8 mask", "seed": 0, "l2": l2_note,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def roofline_times(n_valid, V, D, peaks, clock_mhz):
+    f = (clock_mhz or peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    flops = 8.0 * n_valid * V * D
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    r_mufu, r_fma = 16 * 148 * f, 128 * 148 * f
+    t_alu = n_valid * V / (r_mufu + r_fma / 8)
+    return flops, t_tensor, t_alu
+
+
+# ---------------------------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    from vocabulary_label_bce_b200 import workloads as W
+    p = W.draw_config(args.workload)
+    # size each step's sample from a measured rate so that the whole run takes about two minutes
+    probe = 1024
+    rate = probe / time_oracle_sample(p, probe)
+    n_items = int(rate * 120.0 / max(1, args.steps + args.warmup))
+    n_items = max(512, min(p.V, n_items // 512 * 512))
+    for _ in range(args.warmup):
+        time_oracle_sample(p, n_items)
+    ts = [time_oracle_sample(p, n_items) for _ in range(args.steps)]
+    step = statistics.mean(ts) * p.V / n_items
+    value = p.B * p.N / step
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(p, int(p.mask.sum()), 1, "n/a (CPU)"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"float64 numpy oracle on the first {n_items} of {p.V} items, all "
+                                   f"{p.T} positions, per step; time scaled by V/{n_items}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from vocabulary_label_bce_b200 import binding as B
+    from vocabulary_label_bce_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peaks_src = load_peaks()
+    p = W.draw_config(args.workload, seed=0)
+    H = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    E = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    tg = torch.from_numpy(p.targets).to(dev)
+    m = torch.from_numpy(p.mask).to(dev)
+    prob = B.make_problem(H, E, tg, m, "mean")
+    ws = torch.empty(B.cutbce_workspace_size(prob), dtype=torch.uint8, device=dev)
+    loss = torch.empty((), dtype=torch.float64, device=dev)
+    dH = torch.empty((p.T, p.D), dtype=torch.float32, device=dev)
+    dE = torch.empty((p.V, p.D), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        B.cutbce_forward_backward(prob, None, loss, dH, dE, ws, stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    status = B.cutbce_read_status(ws, stream)
+    if status != 0:
+        raise SystemExit(f"device status {B.cutbce_status_string(status)}")
+    n_valid, n_pairs = B.cutbce_read_counts(prob, ws, None, stream)
+
+    B.cutbce_profile_read(reset=True)
+    B.cutbce_profile_enable(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for s, e in ev:
+        flush.zero_()
+        s.record(stream)
+        step()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    B.cutbce_profile_enable(False)
+    prof = B.cutbce_profile_read(reset=True)
+    status = B.cutbce_read_status(ws, stream)
+    if status != 0:
+        raise SystemExit(f"device status {B.cutbce_status_string(status)}")
+    step_ms_local = statistics.mean(s.elapsed_time(e) for s, e in ev)
+    step_ms = max_over_ranks(step_ms_local)
+    tokens = p.B * p.N
+    value = world * tokens / (step_ms * 1e-3)
+
+    # per-kernel durations (events inside the library, same stream)
+    avg = {k: (ms / n if n else 0.0) for k, (ms, n) in prof.items()}
+    dominant = max(("item_pass", "position_pass"), key=lambda k: avg[k])
+    kern_ms = max_over_ranks(avg[dominant])
+    flops_path, t_tensor, t_alu = roofline_times(n_valid, p.V, p.D, peaks, None)
+    kernel_flops = 4.0 * n_valid * p.V * p.D
+    achieved = kernel_flops / (kern_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    traffic = committed_traffic(dominant, p.name)
+    t_roof = max(t_tensor, t_alu)
+
+    # end to end through the host-buffer entry (pinned host memory, copies inside the timed call)
+    e2e = None
+    if not args.no_e2e:
+        Hh = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Eh = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        th = torch.from_numpy(p.targets).pin_memory()
+        mh = torch.from_numpy(p.mask).pin_memory()
+        hprob = B.make_problem(Hh, Eh, th, mh, "mean")
+        buf = torch.empty(B.cutbce_host_buffer_size(hprob), dtype=torch.uint8, device=dev)
+        lh = torch.empty((), dtype=torch.float64).pin_memory()
+        dHh = torch.empty((p.T, p.D), dtype=torch.float32).pin_memory()
+        dEh = torch.empty((p.V, p.D), dtype=torch.float32).pin_memory()
+        for _ in range(2):
+            B.cutbce_forward_backward_host(hprob, 1.0, lh, dHh, dEh, buf, stream)
+        n_e2e = max(3, min(args.steps, 10))
+        barrier()
+        ts = []
+        for _ in range(n_e2e):
+            flush.zero_()
+            torch.cuda.synchronize(dev)
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            B.cutbce_forward_backward_host(hprob, 1.0, lh, dHh, dEh, buf, stream)
+            e.record(stream)
+            e.synchronize()
+            ts.append(s.elapsed_time(e))
+        barrier()
+        e2e_ms = max_over_ranks(statistics.mean(ts))
+        bi = Hh.numel() * 2 + Eh.numel() * 2 + th.numel() * 4 + mh.numel() + 4
+        bo = 8 + dHh.numel() * 4 + dEh.numel() * 4
+        e2e = {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms,
+               "entry": "cutbce_forward_backward_host (pinned host H, E, targets, mask in; loss, dH, dE out)"}
+        del buf
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_items = min(p.V, args.cpu_sample_items)
+        t = time_oracle_sample(p, n_items)
+        cpu_step = t * p.V / n_items
+        cpu = {"value": tokens / cpu_step, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 numpy oracle on the first {n_items} of {p.V} items, all {p.T} positions "
+                         f"({t:.1f} s), time scaled by V/{n_items}"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(p, n_valid, world, "flushed before each timed step (256 MiB write)"),
+            "valid_tokens_per_s": world * n_valid / (step_ms * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
+                         "kernel_ms": kern_ms, "algorithmic_flops_per_launch": kernel_flops,
+                         "peak_source": f"{peaks_src} bf16_tflops (burst)",
+                         "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak)},
+            "path_roofline": {"flops": flops_path, "t_tensor_ms": t_tensor * 1e3, "t_alu_ms": t_alu * 1e3,
+                              "t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / step_ms},
+            "kernels_ms": {k: round(v, 4) for k, v in avg.items()},
+            "n_pairs": n_pairs,
+            "gpu_launches": args.steps * B.cutbce_kernel_launches(prob, 2),
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -152,6 +152,29 @@ cutbce_status cutbce_read_counts(const cutbce_problem* prob, const void* ws,
  * 2 forward_backward) launches for this problem (for launch accounting). */
 int cutbce_kernel_launches(const cutbce_problem* prob, int entry);
 
+/* Kernel kinds reported by the profiling calls, in launch order. */
+enum {
+  CUTBCE_KERNEL_PREP_ROWS = 0,      /* mask and id rules per position */
+  CUTBCE_KERNEL_PREP_SCAN = 1,      /* row compaction, pair offsets, scales */
+  CUTBCE_KERNEL_PREP_GATHER = 2,    /* compacted H, pair lists, sparse correction */
+  CUTBCE_KERNEL_GROUP_SORT = 3,     /* pairs sorted by item within 64-row groups */
+  CUTBCE_KERNEL_ITEM_PASS = 4,      /* tensor-core pass owning item tiles: loss and dE */
+  CUTBCE_KERNEL_POSITION_PASS = 5,  /* tensor-core pass owning position tiles: dH partials */
+  CUTBCE_KERNEL_FINISH = 6,         /* fixed-order dH reduction and the loss */
+  CUTBCE_NUM_KERNEL_KINDS = 7
+};
+
+/* Per-kernel device timing for benchmarks.  While enabled (process-wide),
+ * every compute call records a CUDA event on its stream before and after each
+ * kernel it launches (the events are created by the library, once, and reused).
+ * Always returns CUTBCE_OK; disabling keeps what was already recorded. */
+cutbce_status cutbce_profile_enable(int enable);
+
+/* Waits for the recorded events, adds their elapsed times to per-kind totals
+ * and writes the totals (milliseconds) to ms[CUTBCE_NUM_KERNEL_KINDS] and the
+ * launch counts to launches[CUTBCE_NUM_KERNEL_KINDS]; clears them if reset != 0. */
+cutbce_status cutbce_profile_read(double* ms, int64_t* launches, int reset);
+
 /* Human-readable name of a status code (static storage). */
 const char* cutbce_status_string(cutbce_status status);
 

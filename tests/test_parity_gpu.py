@@ -84,7 +84,9 @@ def test_all_masked():
 
 
 def test_single_position_single_item():
-    p = W.draw(T=1, V=1, D=64, K=2, dtype="bf16", seed=6, mask="none")
+    p = W.draw(T=1, V=1, D=64, K=1, dtype="bf16", seed=6, mask="none")
+    p.targets = np.array([[0, -1]], dtype=np.int32)
+    p.K = 2
     got = run_gpu(p, "sum")
     check_against_oracle(p, got, "sum")
 

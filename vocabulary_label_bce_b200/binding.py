@@ -20,7 +20,8 @@ __all__ = [
     "cutbce_workspace_size", "cutbce_forward", "cutbce_backward", "cutbce_forward_backward",
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
-    "cutbce_selftest_wait_timeout", "REDUCTIONS",
+    "cutbce_selftest_wait_timeout", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
+    "KERNEL_KINDS",
 ]
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TARGET_RANGE, ERR_TIMEOUT, ERR_CUDA = range(7)
@@ -65,7 +66,10 @@ _SIGS = {
     "cutbce_kernel_launches": (ctypes.c_int, [_P, ctypes.c_int]),
     "cutbce_status_string": (ctypes.c_char_p, [_i32]),
     "cutbce_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
+    "cutbce_profile_enable": (_i32, [ctypes.c_int]),
+    "cutbce_profile_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64), ctypes.c_int]),
 }
+KERNEL_KINDS = ["prep_rows", "prep_scan", "prep_gather", "group_sort", "item_pass", "position_pass", "finish"]
 
 
 def load_library() -> ctypes.CDLL:
@@ -192,3 +196,16 @@ def cutbce_status_string(status: int) -> str:
 def cutbce_selftest_wait_timeout(limit_ns: int, status_dev: torch.Tensor, stream=None) -> None:
     _check(load_library().cutbce_selftest_wait_timeout(int(limit_ns), status_dev.data_ptr(), _stream(stream)),
            "cutbce_selftest_wait_timeout")
+
+
+def cutbce_profile_enable(enable: bool) -> None:
+    _check(load_library().cutbce_profile_enable(1 if enable else 0), "cutbce_profile_enable")
+
+
+def cutbce_profile_read(reset: bool = True) -> dict:
+    """{kernel kind: (total ms, launches)} accumulated since the last reset."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (_i64 * n)()
+    _check(load_library().cutbce_profile_read(ms, cnt, 1 if reset else 0), "cutbce_profile_read")
+    return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "cutbce.h"
 #include "common.cuh"
@@ -167,6 +168,64 @@ bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ---------------------------------------------------------------- launch profiling (benchmarks)
+struct ProfRecord {
+  int kind;
+  cudaEvent_t start, end;
+};
+struct Profiler {
+  std::mutex mu;
+  bool enabled = false;
+  std::vector<cudaEvent_t> pool;
+  std::vector<ProfRecord> pending;
+  double ms[CUTBCE_NUM_KERNEL_KINDS] = {};
+  int64_t launches[CUTBCE_NUM_KERNEL_KINDS] = {};
+
+  cudaEvent_t take() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    return cudaEventCreate(&e) == cudaSuccess ? e : nullptr;
+  }
+  void drain() {  // caller holds mu
+    for (const ProfRecord& r : pending) {
+      float t = 0.f;
+      if (cudaEventSynchronize(r.end) == cudaSuccess && cudaEventElapsedTime(&t, r.start, r.end) == cudaSuccess) {
+        ms[r.kind] += t;
+        launches[r.kind] += 1;
+      }
+      pool.push_back(r.start);
+      pool.push_back(r.end);
+    }
+    pending.clear();
+  }
+};
+Profiler g_prof;
+
+// Brackets one kernel launch with events when profiling is on.
+struct LaunchScope {
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  LaunchScope(int k, cudaStream_t s) : kind(k), st(s) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (!g_prof.enabled) return;
+    if (g_prof.pending.size() > 4096) g_prof.drain();
+    a = g_prof.take();
+    b = g_prof.take();
+    if (a && b) cudaEventRecord(a, st);
+  }
+  ~LaunchScope() {
+    if (!(a && b)) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    g_prof.pending.push_back(ProfRecord{kind, a, b});
+  }
+};
+
 // ---------------------------------------------------------------- tile-engine dispatch
 template <int DP, bool kLoss, bool kGrad, bool kDH>
 cudaError_t launch_tile(int grid, const CUtensorMap& s, const CUtensorMap& x, const TileParams& tp,
@@ -246,11 +305,19 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   } while (0)
 
   CUTBCE_CK(cudaMemsetAsync(hdr, 0, 256, st));
+  {
+  LaunchScope ls(CUTBCE_KERNEL_PREP_ROWS, st);
   k_prep_rows<<<static_cast<unsigned>(ceil_div(T, 128)), 128, 0, st>>>(p->targets, p->mask, T, K, V, ids, rowcnt,
                                                                         hdr);
   CUTBCE_CK(cudaGetLastError());
+  }
+  {
+  LaunchScope ls(CUTBCE_KERNEL_PREP_SCAN, st);
   k_prep_scan<<<1, kScanThreads, 0, st>>>(p->mask, rowcnt, T, V, p->reduction, grad_loss, cidx, orig, rowptr, hdr);
   CUTBCE_CK(cudaGetLastError());
+  }
+  {
+  LaunchScope ls(CUTBCE_KERNEL_PREP_GATHER, st);
   if (bf16) {
     k_prep_gather<__nv_bfloat16><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(p->H), static_cast<const __nv_bfloat16*>(p->E), D, pl.DP, K, pl.Tpad,
@@ -261,6 +328,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
         rowptr, hdr, at<float>(ws, pl.o_hc), pair_t, pair_v, cpart);
   }
   CUTBCE_CK(cudaGetLastError());
+  }
 
   const bool item_pass = w.loss || w.dE;
   if (bf16) {
@@ -274,6 +342,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
                                        static_cast<int>(kGroupRows * kMaxK * 8)));
         sort_cfg = true;
       }
+      LaunchScope ls(CUTBCE_KERNEL_GROUP_SORT, st);
       k_group_sort<<<static_cast<unsigned>(pl.ngroups_max), 256, smem, st>>>(rowptr, pair_t, pair_v, hdr, grp_t,
                                                                              grp_v);
       CUTBCE_CK(cudaGetLastError());
@@ -303,6 +372,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
       const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(dev.sms), pl.n_vitems,
                                                            static_cast<int64_t>(kMaxCtas)}));
       cudaError_t e;
+      LaunchScope ls(CUTBCE_KERNEL_ITEM_PASS, st);
       if (w.loss && w.dE) e = launch_tile_dp<true, true, false>(pl.DP, grid, ms, mx, tp, st);
       else if (w.loss) e = launch_tile_dp<true, false, false>(pl.DP, grid, ms, mx, tp, st);
       else e = launch_tile_dp<false, true, false>(pl.DP, grid, ms, mx, tp, st);
@@ -315,17 +385,20 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
       const int64_t items_max = static_cast<int64_t>(pl.S) * ceil_div(T, kTileM);
       const int grid = static_cast<int>(
           std::min<int64_t>({static_cast<int64_t>(dev.sms), items_max, static_cast<int64_t>(kMaxCtas)}));
+      LaunchScope ls(CUTBCE_KERNEL_POSITION_PASS, st);
       CUTBCE_CK((launch_tile_dp<false, true, true>(pl.DP, grid, ms, mx, tp, st)));
     }
   } else {
     const float* hc = at<float>(ws, pl.o_hc);
     if (item_pass) {
+      LaunchScope ls(CUTBCE_KERNEL_ITEM_PASS, st);
       k_simt_items<<<static_cast<unsigned>(pl.n_vitems), 128, 0, st>>>(
           hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, w.dE ? dE : nullptr,
           w.loss ? lpart : nullptr);
       CUTBCE_CK(cudaGetLastError());
     }
     if (w.dH) {
+      LaunchScope ls(CUTBCE_KERNEL_POSITION_PASS, st);
       k_simt_rows<<<static_cast<unsigned>(ceil_div(pl.Tpad, 128)), 128, 0, st>>>(
           hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, dhpart);
       CUTBCE_CK(cudaGetLastError());
@@ -334,6 +407,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   if (w.loss || w.dH) {
     const int64_t n = w.dH ? static_cast<int64_t>(T) * D : 1;
     const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n, kFinishThreads)));
+    LaunchScope ls(CUTBCE_KERNEL_FINISH, st);
     k_finish<<<grid, kFinishThreads, 0, st>>>(T, D, pl.DP, pl.Tpad, pl.S, cidx, dhpart, w.dH ? dH : nullptr, lpart,
                                              static_cast<int>(pl.n_vitems * kNumEpiWarps), cpart,
                                              static_cast<int>(pl.n_gather_blocks), w.loss ? loss : nullptr, hdr);
@@ -491,6 +565,26 @@ int cutbce_kernel_launches(const cutbce_problem* prob, int entry) {
   make_plan(prob, pl);
   const Want w = entry == 0 ? Want{true, false, false} : entry == 1 ? Want{false, true, true} : Want{true, true, true};
   return count_launches(pl, w);
+}
+
+cutbce_status cutbce_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.enabled = enable != 0;
+  return CUTBCE_OK;
+}
+
+cutbce_status cutbce_profile_read(double* ms, int64_t* launches, int reset) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.drain();
+  for (int k = 0; k < CUTBCE_NUM_KERNEL_KINDS; ++k) {
+    if (ms) ms[k] = g_prof.ms[k];
+    if (launches) launches[k] = g_prof.launches[k];
+    if (reset) {
+      g_prof.ms[k] = 0.0;
+      g_prof.launches[k] = 0;
+    }
+  }
+  return CUTBCE_OK;
 }
 
 const char* cutbce_status_string(cutbce_status s) {
