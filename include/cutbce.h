@@ -157,11 +157,12 @@ enum {
   CUTBCE_KERNEL_PREP_ROWS = 0,      /* mask and id rules per position */
   CUTBCE_KERNEL_PREP_SCAN = 1,      /* row compaction, pair offsets, scales */
   CUTBCE_KERNEL_PREP_GATHER = 2,    /* compacted H, pair lists, sparse correction */
-  CUTBCE_KERNEL_GROUP_SORT = 3,     /* pairs sorted by item within 64-row groups */
+  CUTBCE_KERNEL_GROUP_SORT = 3,     /* pairs sorted by item within 128-row groups */
   CUTBCE_KERNEL_ITEM_PASS = 4,      /* tensor-core pass owning item tiles: loss and dE */
   CUTBCE_KERNEL_POSITION_PASS = 5,  /* tensor-core pass owning position tiles: dH partials */
   CUTBCE_KERNEL_FINISH = 6,         /* fixed-order dH reduction and the loss */
-  CUTBCE_NUM_KERNEL_KINDS = 7
+  CUTBCE_KERNEL_PAIR_SORT = 7,      /* pairs sorted by (item tile, position): all radix passes */
+  CUTBCE_NUM_KERNEL_KINDS = 8
 };
 
 /* Per-kernel device timing for benchmarks.  While enabled (process-wide),

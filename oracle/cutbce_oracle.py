@@ -212,26 +212,29 @@ def dE_rows(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np
 
 def dH_rows(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np.ndarray],
             positions: Sequence[int], reduction: int = MEAN_VALID_POSITIONS,
-            grad_loss: float = 1.0, chunk: int = 1 << 20) -> np.ndarray:
-    """Selected rows of grad_A = grad_H (Eq. (4)), each from its own logit row X[t, :]."""
+            grad_loss: float = 1.0, chunk: int = 1 << 18) -> np.ndarray:
+    """Selected rows of grad_A = grad_H (Eq. (4)), each from its own logit row X[t, :].
+
+    The vocabulary is walked chunk by chunk; within a chunk every selected row's
+    logits, sigmoid minus targets and contribution are formed densely."""
     V = E.shape[0]
     tg = positive_sets(targets, mask, V)
     s = scale_factor(reduction, tg.n_valid, V)
+    pos = [t for t in positions if tg.valid[t]]
+    Hs = np.asarray(H, dtype=np.float64)[pos]
+    acc = np.zeros((len(pos), H.shape[1]), dtype=np.float64)
+    for c0 in range(0, V, chunk):
+        c1 = min(V, c0 + chunk)
+        Ec = np.asarray(E[c0:c1], dtype=np.float64)
+        Z = Hs @ Ec.T
+        Y = _multi_hot([tg.sets[t] for t in pos], c0, c1)
+        acc += (sigmoid(Z) - Y) @ Ec
     out = np.zeros((len(positions), H.shape[1]), dtype=np.float64)
+    k = 0
     for i, t in enumerate(positions):
-        if not tg.valid[t]:
-            continue
-        h = np.asarray(H[t], dtype=np.float64)
-        acc = np.zeros(H.shape[1], dtype=np.float64)
-        for c0 in range(0, V, chunk):
-            c1 = min(V, c0 + chunk)
-            Ec = np.asarray(E[c0:c1], dtype=np.float64)
-            z = Ec @ h
-            y = np.zeros(c1 - c0)
-            ids = tg.sets[t]
-            y[ids[(ids >= c0) & (ids < c1)] - c0] = 1.0
-            acc += (sigmoid(z) - y) @ Ec
-        out[i] = grad_loss * s * acc
+        if tg.valid[t]:
+            out[i] = grad_loss * s * acc[k]
+            k += 1
     return out
 
 

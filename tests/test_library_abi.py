@@ -34,8 +34,8 @@ def test_status_strings():
 def test_workspace_has_no_T_times_V_term():
     base = B.cutbce_workspace_size(_prob(V=100_000))
     big = B.cutbce_workspace_size(_prob(V=10_000_000))
-    # growth in V is only the per-item-tile loss partials (8 doubles per 128 items)
-    assert big - base <= 8 * 8 * (10_000_000 // 128 + 2) + 4096
+    # growth in V is only per item tile (128 items): 8 double loss partials and one int range start
+    assert big - base <= (8 * 8 + 4) * (10_000_000 // 128 + 2) + 8192
     # and it is far below one [T, V] fp32 logit tensor
     assert big < 12800 * 10_000_000 * 4 / 100
 
@@ -78,8 +78,9 @@ def test_compute_calls_reject_before_launch():
 
 def test_launch_accounting():
     p = _prob()
-    assert B.cutbce_kernel_launches(p, 2) == 7          # rows, scan, gather, sort, item pass, dH pass, finish
-    assert B.cutbce_kernel_launches(p, 0) == 5
+    # rows, scan, gather, group sort, 2 radix passes x 3 + item ranges, item pass, dH pass, finish
+    assert B.cutbce_kernel_launches(p, 2) == 14
+    assert B.cutbce_kernel_launches(p, 0) == 5          # rows, scan, gather, item pass, finish
     assert B.cutbce_kernel_launches(p, 3) == -1
 
 

@@ -69,7 +69,8 @@ _SIGS = {
     "cutbce_profile_enable": (_i32, [ctypes.c_int]),
     "cutbce_profile_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64), ctypes.c_int]),
 }
-KERNEL_KINDS = ["prep_rows", "prep_scan", "prep_gather", "group_sort", "item_pass", "position_pass", "finish"]
+KERNEL_KINDS = ["prep_rows", "prep_scan", "prep_gather", "group_sort", "item_pass", "position_pass", "finish",
+                "pair_sort"]
 
 
 def load_library() -> ctypes.CDLL:

@@ -20,7 +20,7 @@ enum : int { kMeanValidPositions = 0, kSum = 1, kMeanElements = 2 };
 constexpr int kMaxK = 128;            // target slots per position
 constexpr int kMaxDim = 256;          // feature width
 constexpr int kTileM = 128;           // stationary rows per tile = TMEM lanes
-constexpr int kGroupRows = 64;        // rows per group of v-sorted pairs
+constexpr int kGroupRows = 128;       // rows per group of item-sorted pairs (= one position tile)
 constexpr int kMaxCtas = 256;         // upper bound of a persistent grid
 constexpr int kMaxSplits = 64;        // dH partial splits over the vocabulary
 constexpr int kTileThreads = 384;     // 12 warps: TMA, MMA, fix-up, idle, 8 epilogue

@@ -16,6 +16,7 @@
 #include "cutbce.h"
 #include "common.cuh"
 #include "prep_finish.cuh"
+#include "pair_sort.cuh"
 #include "tile_engine.cuh"
 
 namespace {
@@ -32,9 +33,10 @@ struct Plan {
   int DP, BN;
   int64_t Tpad, ngroups_max, n_vitems, n_gather_blocks;
   int S, tps, n_vtiles_bn;
+  int radix_passes, radix_blocks;
   size_t elem;
-  size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_grp_t, o_grp_v, o_hc, o_lpart,
-      o_cpart, o_cursor, o_dhpart, total;
+  size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_grp_t, o_grp_v, o_srt[4], o_ghist,
+      o_istart, o_hc, o_lpart, o_cpart, o_dhpart, total;
 };
 
 cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
@@ -70,6 +72,12 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.ngroups_max = ceil_div(p->T, kGroupRows);
   pl.n_vitems = ceil_div(p->V, kTileM);
   pl.n_gather_blocks = ceil_div(pl.Tpad, 8);
+  {
+    int bits = 0;
+    while ((int64_t(1) << bits) < pl.n_vitems) ++bits;
+    pl.radix_passes = (bits + 7) / 8;     // 8-bit digits of the item-tile index
+    pl.radix_blocks = static_cast<int>(std::max<int64_t>(1, ceil_div(p->T * p->K, kRadixTile)));
+  }
   if (bf16) {
     pl.n_vtiles_bn = static_cast<int>(ceil_div(p->V, pl.BN));
     const int64_t nTmax = ceil_div(p->T, kTileM);
@@ -99,10 +107,12 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.o_pair_v = take(4 * TK);
   pl.o_grp_t = take(4 * TK);
   pl.o_grp_v = take(4 * TK);
+  for (int k = 0; k < 4; ++k) pl.o_srt[k] = take(4 * TK);
+  pl.o_ghist = take(4 * 256 * static_cast<size_t>(pl.radix_blocks));
+  pl.o_istart = take(4 * static_cast<size_t>(pl.n_vitems + 1));
   pl.o_hc = take(pl.elem * static_cast<size_t>(pl.Tpad) * pl.DP);
   pl.o_lpart = take(8 * kNumEpiWarps * pl.n_vitems);
   pl.o_cpart = take(8 * pl.n_gather_blocks);
-  pl.o_cursor = take(4 * static_cast<size_t>(kMaxCtas) * pl.ngroups_max);
   pl.o_dhpart = take(4 * static_cast<size_t>(pl.S) * pl.Tpad * pl.DP);
   pl.total = o;
 }
@@ -260,11 +270,12 @@ struct Want {
 
 int count_launches(const Plan& pl, Want w) {
   const bool bf16 = pl.dtype == CUTBCE_BF16;
-  int n = 3;                                        // rows, scan, gather
-  if (bf16 && (w.dE || w.dH)) n += 1;               // group sort
-  if (w.loss || w.dE) n += 1;                       // item-owned pass
-  if (w.dH) n += 1;                                 // position-owned pass
-  if (w.loss || w.dH) n += 1;                       // finish
+  int n = 3;                                            // rows, scan, gather
+  if (bf16 && w.dH) n += 1;                             // group sort
+  if (bf16 && w.dE) n += 3 * pl.radix_passes + 1;       // radix passes and item ranges
+  if (w.loss || w.dE) n += 1;                           // item-owned pass
+  if (w.dH) n += 1;                                     // position-owned pass
+  if (w.loss || w.dH) n += 1;                           // finish
   return n;
 }
 
@@ -296,7 +307,8 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   int* grp_v = at<int>(ws, pl.o_grp_v);
   double* lpart = at<double>(ws, pl.o_lpart);
   double* cpart = at<double>(ws, pl.o_cpart);
-  int* cursors = at<int>(ws, pl.o_cursor);
+  int* istart = at<int>(ws, pl.o_istart);
+  int* ghist = at<int>(ws, pl.o_ghist);
   float* dhpart = at<float>(ws, pl.o_dhpart);
 
 #define CUTBCE_CK(x)                           \
@@ -332,7 +344,8 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
 
   const bool item_pass = w.loss || w.dE;
   if (bf16) {
-    if (w.dE || w.dH) {
+    if (w.dH) {
+      // pairs of each 128-row group ordered by (item, position) for the position-owned pass
       int npow = 1;
       while (npow < kGroupRows * K) npow <<= 1;
       const size_t smem = static_cast<size_t>(npow) * 8;
@@ -347,6 +360,25 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
                                                                              grp_v);
       CUTBCE_CK(cudaGetLastError());
     }
+    const int* srt_v = pair_v;
+    const int* srt_t = pair_t;
+    if (w.dE) {
+      // pairs ordered by (item tile, position): stable LSD radix sort on the item-tile index
+      LaunchScope ls(CUTBCE_KERNEL_PAIR_SORT, st);
+      for (int pass = 0; pass < pl.radix_passes; ++pass) {
+        int* out_v = at<int>(ws, pl.o_srt[2 * (pass & 1)]);
+        int* out_t = at<int>(ws, pl.o_srt[2 * (pass & 1) + 1]);
+        k_radix_hist<<<pl.radix_blocks, kRadixThreads, 0, st>>>(srt_v, hdr, 8 * pass, pl.radix_blocks, ghist);
+        k_exclusive_scan<<<1, 1024, 0, st>>>(ghist, 256 * pl.radix_blocks);
+        k_radix_scatter<<<pl.radix_blocks, kRadixThreads, 0, st>>>(srt_v, srt_t, out_v, out_t, hdr, 8 * pass,
+                                                                   pl.radix_blocks, ghist);
+        srt_v = out_v;
+        srt_t = out_t;
+      }
+      k_item_ranges<<<static_cast<unsigned>(ceil_div(pl.n_vitems + 1, 256)), 256, 0, st>>>(
+          srt_v, hdr, static_cast<int>(pl.n_vitems), istart);
+      CUTBCE_CK(cudaGetLastError());
+    }
     TileParams tp{};
     tp.V = V;
     tp.D = D;
@@ -355,8 +387,9 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     tp.row_ptr = rowptr;
     tp.grp_v = grp_v;
     tp.grp_t = grp_t;
-    tp.cursors = cursors;
-    tp.ngroups_max = static_cast<int>(pl.ngroups_max);
+    tp.srt_t = srt_t;
+    tp.srt_v = srt_v;
+    tp.item_start = istart;
     tp.dE = dE;
     tp.loss_part = lpart;
     tp.dh_part = dhpart;

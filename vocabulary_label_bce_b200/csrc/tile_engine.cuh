@@ -50,10 +50,11 @@ struct TileParams {
   int64_t Tpad;                // rows of H_c (multiple of 128)
   WsHeader* hdr;               // n_valid, grad scale, status
   const int* row_ptr;          // [n_valid + 1] pair offsets of compacted rows
-  const int* grp_v;            // pairs sorted by (item, position) inside 64-row groups
+  const int* grp_v;            // position-owned pass: pairs sorted by (item, position) per 128-row group
   const int* grp_t;
-  int* cursors;                // item-owned pass: [gridDim.x * ngroups_max] fix-up cursors
-  int ngroups_max;
+  const int* srt_t;            // item-owned pass: pairs sorted by (item tile, position, item)
+  const int* srt_v;
+  const int* item_start;       // item-owned pass: [n_item_tiles + 1] ranges into srt_*
   float* dE;                   // item-owned pass output [V, D] (may be null when no gradient)
   double* loss_part;           // item-owned pass: one double per (item tile, epilogue warp)
   float* dh_part;              // position-owned pass output [S, Tpad, DP]
@@ -125,29 +126,28 @@ __device__ __forceinline__ ItemInfo item_info(int i, int n_valid, const TilePara
   return it;
 }
 
-// Walk the v-sorted pairs of one 64-row group from cursor `cur` (warp-uniform):
-// first skip items < lo, then apply every pair with item in [lo, hi) to the G
-// tile by subtracting 1 (y = 1) from the stored bf16 value.
+// Forward-only cursor over one sorted pair range, lane-uniform.  `nxt` holds
+// the key (position for the item-owned pass, item for the position-owned pass)
+// of the next unapplied pair, so a tile without positives costs no memory
+// access.  Every pair with key < hi is applied to the bf16 G tile by
+// subtracting 1 (y = 1 in G = sigmoid(X) - Y).
+struct PairCursor {
+  int cur, end, nxt;
+};
+
 template <bool kDH>
-__device__ __forceinline__ int fixup_walk(int cur, int end, int lo, int hi, int x0, int s0, uint8_t* G,
-                                          const int* __restrict__ grp_v, const int* __restrict__ grp_t,
-                                          int lane) {
-  while (true) {
-    const int idx = cur + lane;
-    const int v = idx < end ? __ldg(grp_v + idx) : 0x7fffffff;
-    const unsigned m = __ballot_sync(0xffffffffu, v < lo);
-    cur += __popc(m);
-    if (m != 0xffffffffu) break;
-  }
-  while (true) {
-    const int idx = cur + lane;
-    const int v = idx < end ? __ldg(grp_v + idx) : 0x7fffffff;
-    const bool in = v < hi;
+__device__ __forceinline__ void fixup_apply(PairCursor& c, int hi, int x0, int s0, uint8_t* G,
+                                            const int* __restrict__ keys, const int* __restrict__ others,
+                                            int lane) {
+  while (c.nxt < hi) {
+    const int idx = c.cur + lane;
+    const int key = idx < c.end ? __ldg(keys + idx) : 0x7fffffff;
+    const bool in = key < hi;
     if (in) {
-      const int t = __ldg(grp_t + idx);
+      const int other = __ldg(others + idx);
       // item-owned: rows are items, columns are positions; position-owned: the reverse
-      const int row = kDH ? (t - s0) : (v - s0);
-      const int col = kDH ? (v - x0) : (t - x0);
+      const int row = other - s0;
+      const int col = key - x0;
       const uint32_t off = static_cast<uint32_t>(col >> 6) * 16384u + static_cast<uint32_t>(row) * 128u +
                            ((((static_cast<uint32_t>(col) & 63u) >> 3) ^ (static_cast<uint32_t>(row) & 7u)) << 4) +
                            ((static_cast<uint32_t>(col) & 7u) << 1);
@@ -155,10 +155,24 @@ __device__ __forceinline__ int fixup_walk(int cur, int end, int lo, int hi, int 
       *e = __float2bfloat16_rn(__bfloat162float(*e) - 1.0f);
     }
     const unsigned m = __ballot_sync(0xffffffffu, in);
-    cur += __popc(m);
-    if (m != 0xffffffffu) break;
+    const int n = __popc(m);
+    c.cur += n;
+    if (n < 32) {
+      c.nxt = __shfl_sync(0xffffffffu, key, n);
+    } else {
+      c.nxt = c.cur < c.end ? __ldg(keys + c.cur) : 0x7fffffff;
+    }
   }
-  return cur;
+}
+
+// First index in [lo, hi) of an ascending int array whose value is >= target.
+__device__ __forceinline__ int lower_bound_idx(const int* __restrict__ a, int lo, int hi, int target) {
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a + mid) < target) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
 }
 
 template <int DP, bool kLoss, bool kGrad, bool kDH>
@@ -370,24 +384,24 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   } else if (warp == 2) {
     // ============================================================ Y fix-up warp
     if (kGrad) {
-      int* curs = p.cursors + static_cast<int64_t>(blockIdx.x) * p.ngroups_max;
-      const int n_groups = static_cast<int>(ceil_div(n_valid, kGroupRows));
-      if (!kDH) {
-        for (int g = lane; g < n_groups; g += 32) curs[g] = p.row_ptr[g * kGroupRows];
-        __syncwarp();
-      }
       uint32_t cnt = 0;
       bool ok = true;
       for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x) {
         const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
-        // position-owned pass: the two groups of the stationary 128 positions, cursors in registers
-        int c0 = 0, e0 = 0, c1 = 0, e1 = 0;
-        if (kDH) {
-          const int g0 = it.s_row0 / kGroupRows;
-          c0 = p.row_ptr[g0 * kGroupRows];
-          e0 = p.row_ptr[min(g0 * kGroupRows + kGroupRows, n_valid)];
-          c1 = e0;
-          e1 = p.row_ptr[min(g0 * kGroupRows + 2 * kGroupRows, n_valid)];
+        PairCursor pc;
+        if (!kDH) {
+          // the item tile's pairs, ordered by position
+          pc.cur = __ldg(p.item_start + i);
+          pc.end = __ldg(p.item_start + i + 1);
+          pc.nxt = pc.cur < pc.end ? __ldg(p.srt_t + pc.cur) : 0x7fffffff;
+        } else {
+          // the 128 stationary positions' pairs, ordered by item, from the split's first item on
+          const int g0 = it.s_row0;
+          const int gs = __ldg(p.row_ptr + g0);
+          const int ge = __ldg(p.row_ptr + min(g0 + kGroupRows, n_valid));
+          pc.cur = lower_bound_idx(p.grp_v, gs, ge, it.x_tile0 * BN);
+          pc.end = ge;
+          pc.nxt = pc.cur < pc.end ? __ldg(p.grp_v + pc.cur) : 0x7fffffff;
         }
         for (int j = 0; j < it.n_x; ++j) {
           const uint32_t c = cnt + j, b = c & 1;
@@ -398,19 +412,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           uint8_t* G = sG + b * G_BYTES;
           if (!kDH) {
             const int t0 = j * BN;
-            const int v0 = it.s_row0;
-            for (int g = t0 / kGroupRows; g < (t0 + BN) / kGroupRows && g < n_groups; ++g) {
-              const int end = p.row_ptr[min(g * kGroupRows + kGroupRows, n_valid)];
-              const int cur = fixup_walk<false>(curs[g], end, v0, v0 + kTileM, t0, v0, G, p.grp_v, p.grp_t, lane);
-              __syncwarp();
-              if (lane == 0) curs[g] = cur;
-              __syncwarp();
-            }
+            fixup_apply<false>(pc, t0 + BN, t0, it.s_row0, G, p.srt_t, p.srt_v, lane);
           } else {
             const int v0 = (it.x_tile0 + j) * BN;
-            const int t0 = it.s_row0;
-            c0 = fixup_walk<true>(c0, e0, v0, v0 + BN, v0, t0, G, p.grp_v, p.grp_t, lane);
-            c1 = fixup_walk<true>(c1, e1, v0, v0 + BN, v0, t0, G, p.grp_v, p.grp_t, lane);
+            fixup_apply<true>(pc, v0 + BN, v0, it.s_row0, G, p.grp_v, p.grp_t, lane);
           }
           fence_proxy_async_smem();
           __syncwarp();
