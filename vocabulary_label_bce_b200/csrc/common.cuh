@@ -23,19 +23,19 @@ constexpr int kTileM = 128;           // stationary rows per tile = TMEM lanes
 constexpr int kGroupRows = 128;       // rows per group of item-sorted pairs (= one position tile)
 constexpr int kMaxCtas = 256;         // upper bound of a persistent grid
 constexpr int kMaxSplits = 64;        // dH partial splits over the vocabulary
-constexpr int kTileThreads = 384;     // 12 warps: TMA, MMA, fix-up, idle, 8 epilogue
+constexpr int kTileThreads = 640;     // 20 warps: TMA, MMA, fix-up, idle, 16 epilogue
 constexpr int kEpiWarp0 = 4;
-constexpr int kNumEpiWarps = 8;
+constexpr int kNumEpiWarps = 16;      // 4 per TMEM lane quarter (one per SM sub-partition each)
 
 // First 256 bytes of the workspace.
 struct WsHeader {
   int status;          // first device-detected error, 0 = none
   int n_valid;         // valid positions
   int n_pairs;         // distinct (position, positive item) pairs
-  int pad0;
+  int wait_tag;        // where the first bounded wait gave up: role<<28 | barrier<<20 | counter
   double loss_scale;   // s
   float grad_scale;    // g * s
-  float pad1;
+  int wait_block;      // CTA of that wait
 };
 
 // Geometry of the tcgen05 tile engine for one padded feature width DP.
@@ -45,14 +45,16 @@ struct TileCfg {
   static constexpr int BN = DP <= 128 ? 128 : 64;          // streamed rows per tile (Z columns)
   static constexpr int NKB = DP / 64;                        // 128-byte column blocks per row
   static constexpr int NX = DP == 64 ? 4 : 3;                // stages of the streamed-operand ring
+  static constexpr int NZ = 3;                               // logit tiles in tensor memory
+  static constexpr int NG = DP == 128 ? 2 : 3;               // bf16 sigmoid tiles in shared memory
   static constexpr uint32_t S_BYTES = kTileM * DP * 2;       // stationary tile
   static constexpr uint32_t X_BYTES = BN * DP * 2;           // streamed tile
   static constexpr uint32_t G_BYTES = kTileM * BN * 2;       // bf16 sigmoid tile
-  static constexpr int ACC_COL = 2 * BN;                     // TMEM column of the gradient accumulator
+  static constexpr int ACC_COL = NZ * BN;                    // TMEM column of the gradient accumulator
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NUM_BARS = 2 + 2 * NX + 2 * 5 + 3;    // see the kernel for the list
+  static constexpr int NUM_BARS = 2 + 2 * NX + 2 * NZ + 3 * NG + 3;  // see the kernel for the list
   static constexpr uint32_t SMEM_BYTES =
-      1024 + S_BYTES + NX * X_BYTES + 2 * G_BYTES + NUM_BARS * 8 + 16 + 64;
+      1024 + S_BYTES + NX * X_BYTES + NG * G_BYTES + NUM_BARS * 8 + 16 + 64;
   static_assert(ACC_COL + DP <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(SMEM_BYTES > 232448 / 2, "one CTA per SM keeps the TMEM allocation uncontended");

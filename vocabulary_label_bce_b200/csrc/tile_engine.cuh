@@ -23,13 +23,13 @@
 // term uses no Y at all (Eq. (2): l(x,y) = l(x,0) - y x); the -y x part is the
 // separate sparse correction summed in the prep kernel.
 //
-// Warp roles (384 threads, one CTA per SM):
+// Warp roles (640 threads, one CTA per SM):
 //   warp 0      TMA producer (stationary tile, ring of streamed tiles)
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warp 2      fix-up warp (Y in-tile)
 //   warp 3      idle
-//   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4).. and one half of
-//               the tile's columns
+//   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. and one quarter
+//               of the tile's columns
 //
 // Every wait is bounded (global timer); on expiry the CTA records
 // CUTBCE_ERR_TIMEOUT in the status word, the other roles leave their loops, the
@@ -66,21 +66,35 @@ struct TileParams {
 
 struct WaitCtx {
   volatile int* abort_flag;
-  int* status;
+  WsHeader* hdr;
   long long limit;
 };
 
+// Where a wait happens, recorded if it gives up: role (1 producer, 2 MMA,
+// 3 fix-up, 4 epilogue), barrier id, and the role's tile or item counter.
+__device__ __forceinline__ int wait_tag(int role, int barrier, uint32_t counter) {
+  return (role << 28) | (barrier << 20) | static_cast<int>(counter & 0xFFFFFu);
+}
+
 // Bounded wait for phase `parity` of `bar`.  Returns false if the CTA aborted
-// or the limit ran out (then it records the timeout and raises the abort flag).
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+// or the limit ran out (then it records the timeout, where it happened, and
+// raises the abort flag).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitCtx& w, int tag = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*w.abort_flag) return false;
+    if (*w.abort_flag) {
+      // record where each role stood when the CTA gave up (first record per role wins)
+      if (tag != 0) atomicCAS(reinterpret_cast<int*>(w.hdr) + 8 + ((tag >> 28) & 7), 0, tag);
+      return false;
+    }
     if (static_cast<long long>(global_timer_ns() - t0) > w.limit) {
       *w.abort_flag = 1;
-      atomicCAS(w.status, 0, kErrTimeout);
+      if (atomicCAS(&w.hdr->status, 0, kErrTimeout) == 0) {
+        w.hdr->wait_tag = tag;
+        w.hdr->wait_block = static_cast<int>(blockIdx.x);
+      }
       return false;
     }
   }
@@ -94,8 +108,8 @@ __device__ __forceinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity, l
   return true;
 }
 // Whole-warp wait with a warp-uniform result.
-__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  const bool ok = wait_bar(bar, parity, w);
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w, int tag = 0) {
+  const bool ok = wait_bar(bar, parity, w, tag);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -182,6 +196,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   constexpr int BN = Cfg::BN;
   constexpr int NKB = Cfg::NKB;
   constexpr int NX = Cfg::NX;
+  constexpr int NZ = Cfg::NZ;
+  constexpr int NG = Cfg::NG;
   constexpr uint32_t S_BYTES = Cfg::S_BYTES, X_BYTES = Cfg::X_BYTES, G_BYTES = Cfg::G_BYTES;
   constexpr int ACC_COL = Cfg::ACC_COL;
   static_assert(!kDH || (kGrad && !kLoss), "the position-owned pass computes dH only");
@@ -194,19 +210,19 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   uint8_t* sS = smem;
   uint8_t* sX = sS + S_BYTES;
   uint8_t* sG = sX + NX * X_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + 2 * G_BYTES);
-  uint64_t* bar_sfull = bars + 0;
-  uint64_t* bar_sempty = bars + 1;
-  uint64_t* bar_xfull = bars + 2;
-  uint64_t* bar_xempty = bars + 2 + NX;
-  uint64_t* bar_zfull = bars + 2 + 2 * NX;
-  uint64_t* bar_zempty = bar_zfull + 2;
-  uint64_t* bar_gwritten = bar_zfull + 4;
-  uint64_t* bar_gfull = bar_zfull + 6;
-  uint64_t* bar_gempty = bar_zfull + 8;
-  uint64_t* bar_accfull = bar_zfull + 10;
-  uint64_t* bar_accempty = bar_zfull + 11;
-  uint64_t* bar_drain = bar_zfull + 12;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + NG * G_BYTES);
+  uint64_t* bar_sfull = bars + 0;                 // stationary tile landed (TMA)
+  uint64_t* bar_sempty = bars + 1;                // stationary tile free (MMA commit)
+  uint64_t* bar_xfull = bars + 2;                 // [NX] streamed tile landed
+  uint64_t* bar_xempty = bar_xfull + NX;          // [NX] streamed tile free
+  uint64_t* bar_zfull = bar_xempty + NX;          // [NZ] logit tile ready in TMEM
+  uint64_t* bar_zempty = bar_zfull + NZ;          // [NZ] logit tile read by the epilogue
+  uint64_t* bar_gwritten = bar_zempty + NZ;       // [NG] sigmoid tile written by the epilogue
+  uint64_t* bar_fixdone = bar_gwritten + NG;      // [NG] target fix-ups of the tile applied
+  uint64_t* bar_gempty = bar_fixdone + NG;        // [NG] sigmoid tile consumed by the MMA
+  uint64_t* bar_accfull = bar_gempty + NG;        // gradient accumulator complete
+  uint64_t* bar_accempty = bar_accfull + 1;       // gradient accumulator read out
+  uint64_t* bar_drain = bar_accempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -247,11 +263,13 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       mbar_init(bar_xfull + s, 1);
       mbar_init(bar_xempty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NZ; ++b) {
       mbar_init(bar_zfull + b, 1);
       mbar_init(bar_zempty + b, kNumEpiWarps);
+    }
+    for (int b = 0; b < NG; ++b) {
       mbar_init(bar_gwritten + b, kNumEpiWarps);
-      mbar_init(bar_gfull + b, 1);
+      mbar_init(bar_fixdone + b, 1);
       mbar_init(bar_gempty + b, 1);
     }
     mbar_init(bar_accfull, 1);
@@ -269,7 +287,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const WaitCtx wc{abort_flag, &hdr->status, p.timeout_ns};
+  const WaitCtx wc{abort_flag, hdr, p.timeout_ns};
 
   if (warp == 0) {
     // ============================================================ TMA producer
@@ -277,7 +295,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       uint32_t ic = 0, xc = 0;
       for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++ic) {
         const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
-        if (!wait_bar(bar_sempty, (ic & 1) ^ 1, wc)) break;
+        if (!wait_bar(bar_sempty, (ic & 1) ^ 1, wc, wait_tag(1, 1, ic))) break;
         mbar_arrive_expect_tx(bar_sfull, S_BYTES);
 #pragma unroll
         for (int kb = 0; kb < NKB; ++kb)
@@ -285,7 +303,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         bool ok = true;
         for (int j = 0; j < it.n_x; ++j, ++xc) {
           const uint32_t st = xc % NX;
-          if (!wait_bar(bar_xempty + st, ((xc / NX) & 1) ^ 1, wc)) {
+          if (!wait_bar(bar_xempty + st, ((xc / NX) & 1) ^ 1, wc, wait_tag(1, 3, xc))) {
             ok = false;
             break;
           }
@@ -310,17 +328,25 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
+    // One thread.  Logit tiles (Z) run up to NZ tiles ahead of the gradient
+    // MMAs, so the epilogue always finds its next tile computed.
     if (lane == 0) {
       constexpr uint32_t idesc_z = idesc_bf16_f32(kTileM, BN, false, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kTileM, DP, false, true);
       const uint32_t sS_a = smem_u32(sS), sX_a = smem_u32(sX), sG_a = smem_u32(sG);
-      uint32_t ic = 0, cnt = 0;
-      bool ok = true;
-      // Z[b] = S * X[st]^T : both operands K-major, 128-byte swizzle
-      auto issue_z = [&](uint32_t c) -> bool {
-        const uint32_t st = c % NX, b = c & 1;
-        if (!wait_bar(bar_xfull + st, (c / NX) & 1, wc)) return false;
-        if (!wait_bar(bar_zempty + b, ((c >> 1) & 1) ^ 1, wc)) return false;
+      int zi = blockIdx.x, zj = 0, gi = blockIdx.x, gj = 0;
+      uint32_t zic = 0, cz = 0, gic = 0, cg = 0;
+      ItemInfo zit{}, git{};
+      if (zi < n_items) zit = git = item_info<DP, kDH>(zi, n_valid, p);
+      // Z[cz % NZ] = S * X^T : both operands K-major, 128-byte swizzle
+      auto issue_next_z = [&]() -> bool {
+        if (zj == 0) {
+          if (!wait_bar(bar_sfull, zic & 1, wc, wait_tag(2, 0, zic))) return false;
+          tc_fence_after();
+        }
+        const uint32_t st = cz % NX, b = cz % NZ;
+        if (!wait_bar(bar_xfull + st, (cz / NX) & 1, wc, wait_tag(2, 2, cz))) return false;
+        if (!wait_bar(bar_zempty + b, ((cz / NZ) & 1) ^ 1, wc, wait_tag(2, 5, cz))) return false;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DP / 16; ++ks) {
@@ -330,52 +356,50 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         }
         umma_commit(bar_zfull + b);
         if (!kGrad) umma_commit(bar_xempty + st);
+        ++cz;
+        if (++zj == zit.n_x) {
+          umma_commit(bar_sempty);                 // the stationary tile is no longer read
+          zj = 0;
+          ++zic;
+          zi += gridDim.x;
+          if (zi < n_items) zit = item_info<DP, kDH>(zi, n_valid, p);
+        }
         return true;
       };
-      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ic) {
-        const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
-        const int n = it.n_x;
-        if (!wait_bar(bar_sfull, ic & 1, wc)) break;
-        tc_fence_after();
-        if (!issue_z(cnt)) break;
-        for (int j = 0; j < n; ++j) {
-          const uint32_t c = cnt + j;
-          if (j + 1 < n) {
-            if (!issue_z(c + 1)) {
-              ok = false;
-              break;
-            }
-          } else {
-            umma_commit(bar_sempty);
-          }
-          if (kGrad) {
-            const uint32_t b = c & 1, st = c % NX;
-            if (!wait_bar(bar_gfull + b, (c >> 1) & 1, wc)) {
-              ok = false;
-              break;
-            }
+      bool ok = true;
+      if (!kGrad) {
+        while (ok && zi < n_items) ok = issue_next_z();
+      } else {
+        while (ok && gi < n_items) {
+          while (ok && zi < n_items && cz < cg + NZ) ok = issue_next_z();
+          if (!ok) break;
+          const uint32_t b = cg % NG, st = cg % NX;
+          if (!wait_bar(bar_gwritten + b, (cg / NG) & 1, wc, wait_tag(2, 6, cg)) ||
+              !wait_bar(bar_fixdone + b, (cg / NG) & 1, wc, wait_tag(2, 7, cg)))
+            break;
+          tc_fence_after();
+          if (gj == 0) {
+            if (!wait_bar(bar_accempty, (gic & 1) ^ 1, wc, wait_tag(2, 10, gic))) break;
             tc_fence_after();
-            if (j == 0) {
-              if (!wait_bar(bar_accempty, (ic & 1) ^ 1, wc)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            // ACC += G[b] * X[st] : G K-major, X read MN-major (its rows are the K index)
+          }
+          // ACC += G[b] * X[st] : G K-major, X read MN-major (its rows are the K index)
 #pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks) {
-              const uint64_t a = smem_desc_sw128(sG_a + b * G_BYTES + (ks >> 2) * (kTileM * 128) + (ks & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(sX_a + st * X_BYTES + ks * 2048, BN * 128, 1024);
-              umma_bf16(tmem_base + ACC_COL, a, bd, idesc_acc, (j > 0 || ks > 0) ? 1u : 0u);
-            }
-            umma_commit(bar_gempty + b);
-            umma_commit(bar_xempty + st);
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t a = smem_desc_sw128(sG_a + b * G_BYTES + (ks >> 2) * (kTileM * 128) + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sX_a + st * X_BYTES + ks * 2048, BN * 128, 1024);
+            umma_bf16(tmem_base + ACC_COL, a, bd, idesc_acc, (gj > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(bar_gempty + b);
+          umma_commit(bar_xempty + st);
+          ++cg;
+          if (++gj == git.n_x) {
+            umma_commit(bar_accfull);
+            gj = 0;
+            ++gic;
+            gi += gridDim.x;
+            if (gi < n_items) git = item_info<DP, kDH>(gi, n_valid, p);
           }
         }
-        if (!ok) break;
-        if (kGrad) umma_commit(bar_accfull);
-        cnt += n;
       }
       // every MMA this thread issued has completed once the drain barrier flips
       umma_commit(bar_drain);
@@ -404,30 +428,42 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           pc.nxt = pc.cur < pc.end ? __ldg(p.grp_v + pc.cur) : 0x7fffffff;
         }
         for (int j = 0; j < it.n_x; ++j) {
-          const uint32_t c = cnt + j, b = c & 1;
-          if (!wait_bar_warp(bar_gwritten + b, (c >> 1) & 1, wc)) {
+          const uint32_t c = cnt + j, b = c % NG;
+          const int x0 = kDH ? (it.x_tile0 + j) * BN : j * BN;   // first streamed row of the tile
+          // The previous use of this buffer (tile c - NG) must be consumed by the MMA first:
+          // that keeps this warp at most one phase ahead on gwritten[b] and fixdone[b], so a
+          // parity wait can never match a phase two uses ahead.
+          if (!wait_bar_warp(bar_gempty + b, ((c / NG) & 1) ^ 1, wc, wait_tag(3, 8, c))) {
             ok = false;
             break;
           }
-          uint8_t* G = sG + b * G_BYTES;
-          if (!kDH) {
-            const int t0 = j * BN;
-            fixup_apply<false>(pc, t0 + BN, t0, it.s_row0, G, p.srt_t, p.srt_v, lane);
-          } else {
-            const int v0 = (it.x_tile0 + j) * BN;
-            fixup_apply<true>(pc, v0 + BN, v0, it.s_row0, G, p.grp_v, p.grp_t, lane);
+          if (pc.nxt < x0 + BN) {
+            // positives fall in this tile: wait for the epilogue's sigmoid tile, then subtract 1
+            if (!wait_bar_warp(bar_gwritten + b, (c / NG) & 1, wc, wait_tag(3, 6, c))) {
+              ok = false;
+              break;
+            }
+            uint8_t* G = sG + b * G_BYTES;
+            if (!kDH) fixup_apply<false>(pc, x0 + BN, x0, it.s_row0, G, p.srt_t, p.srt_v, lane);
+            else fixup_apply<true>(pc, x0 + BN, x0, it.s_row0, G, p.grp_v, p.grp_t, lane);
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_gfull + b);
+          if (lane == 0) mbar_arrive(bar_fixdone + b);
         }
         cnt += it.n_x;
       }
     }
   } else if (warp >= kEpiWarp0) {
     // ============================================================ epilogue
+    // Warp w reads TMEM lanes 32*(w%4).. (its sub-partition's quarter) and one
+    // column slab of each tile: 4 warps per quarter keep the sub-partition's
+    // MUFU/FMA pipes fed while others wait on tensor-memory loads.
+    constexpr int kSlabs = kNumEpiWarps / 4;
+    constexpr int ZC = BN / kSlabs;               // Z columns per warp per tile (32 or 16)
+    constexpr int AC = DP / kSlabs;               // accumulator columns per warp (16 .. 64)
     const int q = warp & 3;                       // TMEM lane quarter
-    const int hh = (warp - kEpiWarp0) >> 2;       // column half
+    const int slab = (warp - kEpiWarp0) >> 2;     // column slab
     const int row = q * 32 + lane;                // stationary row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t sG_a = smem_u32(sG);
@@ -439,75 +475,63 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       const int n = it.n_x;
       double item_acc = 0.0;
       for (int j = 0; j < n; ++j) {
-        const uint32_t c = cnt + j, b = c & 1;
-        if (!wait_bar_warp(bar_zfull + b, (c >> 1) & 1, wc)) {
+        const uint32_t c = cnt + j, bz = c % NZ, bg = c % NG;
+        if (!wait_bar_warp(bar_zfull + bz, (c / NZ) & 1, wc, wait_tag(4, 4, c))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        uint32_t r[ZC];
+        tmem_ld<ZC>(tmem_base + lane_base + bz * BN + slab * ZC, r);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_zempty + bz);   // this warp's part of Z[bz] is in registers
+        uint32_t pk[ZC / 2];
+        float prod = 1.f, tile_mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < ZC; e += 2) {
+          float gpair[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const float z = __uint_as_float(r[e + k]);
+            if (kLoss) {
+              const float u = ex2_approx(-fabsf(z) * kLog2e);   // e^{-|z|}
+              const float pz = 1.f + u;
+              prod *= pz;                                        // log1p batched: one lg2 per slab
+              tile_mx += fmaxf(z, 0.f);
+              if (kGrad) {
+                const float rp = rcp_approx(pz);                 // 1 / (1 + e^{-|z|})
+                gpair[k] = z >= 0.f ? rp : u * rp;               // sigmoid(z)
+              }
+            } else {
+              gpair[k] = fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);  // sigmoid(z)
+            }
+          }
+          if (kGrad) pk[e >> 1] = pack_bf16x2(gpair[0], gpair[1]);
+        }
         if (kGrad) {
-          if (!wait_bar_warp(bar_gempty + b, ((c >> 1) & 1) ^ 1, wc)) {
+          if (!wait_bar_warp(bar_gempty + bg, ((c / NG) & 1) ^ 1, wc, wait_tag(4, 8, c))) {
             ok = false;
             break;
           }
-        }
-        const uint32_t zaddr = tmem_base + lane_base + b * BN + hh * (BN / 2);
-        const uint32_t grow = sG_a + b * G_BYTES + row * 128;
-        float tile_mx = 0.f, tile_l2 = 0.f;
-#pragma unroll 1
-        for (int ch = 0; ch < BN / 64; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(zaddr + ch * 32, r);
-          tmem_ld_wait();
-          if (ch == BN / 64 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_zempty + b);
-          }
-          uint32_t pk[16];
-          float prod = 1.f;
+          const int col0 = slab * ZC;
+          const uint32_t base = sG_a + bg * G_BYTES + (col0 >> 6) * (kTileM * 128) + row * 128;
+          const uint32_t j0 = (col0 & 63) >> 3;
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float gpair[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const float z = __uint_as_float(r[e + k]);
-              if (kLoss) {
-                const float u = ex2_approx(-fabsf(z) * kLog2e);   // e^{-|z|}
-                const float pz = 1.f + u;
-                prod *= pz;                                        // log1p batched: one lg2 per 32
-                tile_mx += fmaxf(z, 0.f);
-                if (kGrad) {
-                  const float rp = rcp_approx(pz);                 // 1 / (1 + e^{-|z|})
-                  gpair[k] = z >= 0.f ? rp : u * rp;               // sigmoid(z)
-                }
-              } else {
-                gpair[k] = fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);  // sigmoid(z)
-              }
-            }
-            if (kGrad) pk[e >> 1] = pack_bf16x2(gpair[0], gpair[1]);
-          }
-          if (kLoss) tile_l2 += lg2_approx(prod);
-          if (kGrad) {
-            const int col0 = hh * (BN / 2) + ch * 32;
-            const uint32_t base = grow + (col0 >> 6) * (kTileM * 128);
-            const uint32_t j0 = (col0 & 63) >> 3;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              st_shared_v4(base + (((j0 + k) ^ (row & 7)) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
-                           pk[4 * k + 3]);
-          }
-        }
-        if (kGrad) {
+          for (int k = 0; k < ZC / 8; ++k)
+            st_shared_v4(base + (((j0 + k) ^ (row & 7)) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
+                         pk[4 * k + 3]);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_gwritten + b);
+          if (lane == 0) mbar_arrive(bar_gwritten + bg);
         }
         if (kLoss) {
+          float tile_l2 = lg2_approx(prod);
           if (j == n - 1) {
             // zero rows of H_c past n_valid give z = 0 exactly: each adds log2(2) = 1 to tile_l2
             const int t0 = j * BN;
-            const int lo = hh * (BN / 2), hi = lo + BN / 2;
+            const int lo = slab * ZC, hi = lo + ZC;
             const int pad = hi - max(min(n_valid - t0, hi), lo);
             tile_l2 -= static_cast<float>(pad);
           }
@@ -523,20 +547,20 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         if (lane == 0) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + (warp - kEpiWarp0)] = val;
       }
       if (kGrad) {
-        if (!wait_bar_warp(bar_accfull, ic & 1, wc)) break;
+        if (!wait_bar_warp(bar_accfull, ic & 1, wc, wait_tag(4, 9, ic))) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int ch = 0; ch < DP / 64; ++ch) {
-          uint32_t r[32];
-          const int col0 = hh * (DP / 2) + ch * 32;
-          tmem_ld32(tmem_base + lane_base + ACC_COL + col0, r);
+        for (int ch = 0; ch < AC / 16; ++ch) {
+          uint32_t r[16];
+          const int col0 = slab * AC + ch * 16;
+          tmem_ld<16>(tmem_base + lane_base + ACC_COL + col0, r);
           tmem_ld_wait();
           if (!kDH) {
             const int v = it.s_row0 + row;
             if (v < p.V && p.dE != nullptr) {
               float* dst = p.dE + static_cast<int64_t>(v) * p.D + col0;
 #pragma unroll
-              for (int e = 0; e < 32; e += 4)
+              for (int e = 0; e < 16; e += 4)
                 if (col0 + e < p.D)
                   *reinterpret_cast<float4*>(dst + e) =
                       make_float4(__uint_as_float(r[e]) * gs, __uint_as_float(r[e + 1]) * gs,
@@ -545,7 +569,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           } else {
             float* dst = p.dh_part + (static_cast<int64_t>(it.split) * p.Tpad + it.s_row0 + row) * DP + col0;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
+            for (int e = 0; e < 16; e += 4)
               *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
                                                                 __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
           }
@@ -571,19 +595,14 @@ __global__ void __launch_bounds__(kTileThreads, 1)
 // timeout and return.  Used only by cutbce_selftest_wait_timeout.
 __global__ void k_selftest_wait(long long limit_ns, int* status) {
   __shared__ uint64_t bar;
-  __shared__ int abort_flag;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
-    abort_flag = 0;
     fence_mbarrier_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     *status = 0;
-    const WaitCtx wc{&abort_flag, status, limit_ns};
-    if (!wait_bar(&bar, 0, wc)) {
-      if (*status == 0) *status = kErrTimeout;
-    }
+    if (!wait_bar_drain(&bar, 0, limit_ns)) *status = kErrTimeout;
   }
 }
 
