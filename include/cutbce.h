@@ -96,7 +96,7 @@ typedef struct {
 } cutbce_problem;
 
 /* Bytes of device workspace that a compute call on this problem needs.  The
- * size has no T*V term: it is O(T*K + S*T*D + V/128) for a split count S <= 64
+ * size has no T*V term: it is O(T*K + S*T*D + V) for a split count S <= 64
  * chosen from T.  Host-only; launches nothing.  Returns INVALID_ARG or
  * UNSUPPORTED for a problem the compute calls would reject. */
 cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes);
@@ -157,11 +157,11 @@ enum {
   CUTBCE_KERNEL_PREP_ROWS = 0,      /* mask and id rules per position */
   CUTBCE_KERNEL_PREP_SCAN = 1,      /* row compaction, pair offsets, scales */
   CUTBCE_KERNEL_PREP_GATHER = 2,    /* compacted H, pair lists, sparse correction */
-  CUTBCE_KERNEL_GROUP_SORT = 3,     /* pairs sorted by item within 128-row groups */
+  CUTBCE_KERNEL_CSC_OFFSETS = 3,    /* first pair of every item in the item-sorted pairs */
   CUTBCE_KERNEL_ITEM_PASS = 4,      /* tensor-core pass owning item tiles: loss and dE */
   CUTBCE_KERNEL_POSITION_PASS = 5,  /* tensor-core pass owning position tiles: dH partials */
   CUTBCE_KERNEL_FINISH = 6,         /* fixed-order dH reduction and the loss */
-  CUTBCE_KERNEL_PAIR_SORT = 7,      /* pairs sorted by (item tile, position): all radix passes */
+  CUTBCE_KERNEL_PAIR_SORT = 7,      /* pairs sorted by (item, position): all radix passes */
   CUTBCE_NUM_KERNEL_KINDS = 8
 };
 
@@ -175,6 +175,43 @@ cutbce_status cutbce_profile_enable(int enable);
  * and writes the totals (milliseconds) to ms[CUTBCE_NUM_KERNEL_KINDS] and the
  * launch counts to launches[CUTBCE_NUM_KERNEL_KINDS]; clears them if reset != 0. */
 cutbce_status cutbce_profile_read(double* ms, int64_t* launches, int reset);
+
+/* Operation kinds measured by cutbce_probe_pipe_rate. */
+enum {
+  CUTBCE_PROBE_FFMA = 0,    /* fma.rn.f32 */
+  CUTBCE_PROBE_FFMA2 = 1,   /* fma.rn.f32x2, counted as two operations */
+  CUTBCE_PROBE_EX2 = 2,     /* ex2.approx.ftz.f32 */
+  CUTBCE_PROBE_RCP = 3,     /* rcp.approx.ftz.f32 */
+  CUTBCE_PROBE_TANH = 4,    /* tanh.approx.f32 */
+  CUTBCE_PROBE_LG2 = 5,     /* lg2.approx.ftz.f32 */
+  CUTBCE_PROBE_CVT_BF16X2 = 6, /* cvt.rn.bf16x2.f32, counted as one instruction */
+  CUTBCE_PROBE_FMAX = 7,    /* max.f32 */
+  CUTBCE_PROBE_ADD2 = 8,    /* add.rn.f32x2, counted as two operations */
+  CUTBCE_PROBE_IADD = 9,    /* add.s32 */
+  CUTBCE_PROBE_PRMT = 10,   /* prmt.b32 */
+  CUTBCE_NUM_PROBES = 11
+};
+
+/* Bytes of device scratch cutbce_probe_pipe_rate needs. */
+size_t cutbce_probe_scratch_bytes(void);
+
+/* Measures how many operations of one kind an SM retires per clock: one CTA
+ * of 1024 threads per SM runs independent dependency chains of the operation
+ * and times them with the SM clock.  These rates set the arithmetic roofline
+ * of the loss's element math (one exp, a reciprocal and a share of a log per
+ * logit).  scratch: caller-owned device memory (cutbce_probe_scratch_bytes).
+ * Synchronises `stream`.  Writes the median over SMs to *ops_per_clock_per_sm. */
+cutbce_status cutbce_probe_pipe_rate(int op, void* scratch, size_t scratch_bytes, double* ops_per_clock_per_sm,
+                                     cutbce_stream_t stream);
+
+/* Tensor-core probe: on every SM one thread issues `iters` bf16 tcgen05.mma
+ * instructions of shape 128 x n x 16 (n = 64, 128 or 256; fp32 accumulator in
+ * tensor memory; A from shared memory, or from tensor memory if bit 0 of
+ * a_in_tmem is set; B K-major, or MN-major if bit 1 is set) and waits for them.  Writes the median over SMs of the cycles per instruction
+ * spent issuing and until completion (the dense ideal on B200 is n/2 cycles).
+ * Synchronises `stream`. */
+cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratch, size_t scratch_bytes,
+                               double* issue_cycles_per_mma, double* cycles_per_mma, cutbce_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* cutbce_status_string(cutbce_status status);

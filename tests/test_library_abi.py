@@ -34,8 +34,9 @@ def test_status_strings():
 def test_workspace_has_no_T_times_V_term():
     base = B.cutbce_workspace_size(_prob(V=100_000))
     big = B.cutbce_workspace_size(_prob(V=10_000_000))
-    # growth in V is only per item tile (128 items): 16 double loss partials and one int range start
-    assert big - base <= (16 * 8 + 4) * (10_000_000 // 128 + 2) + 8192
+    # growth in V is per item: one int offset into the item-sorted pairs, and per tile of
+    # 128 items 16 double loss partials
+    assert big - base <= (16 * 8 + 4 * 128) * (10_000_000 // 128 + 2) + 8192
     # and it is far below one [T, V] fp32 logit tensor
     assert big < 12800 * 10_000_000 * 4 / 100
 
@@ -78,8 +79,8 @@ def test_compute_calls_reject_before_launch():
 
 def test_launch_accounting():
     p = _prob()
-    # rows, scan, gather, group sort, 2 radix passes x 3 + item ranges, item pass, dH pass, finish
-    assert B.cutbce_kernel_launches(p, 2) == 14
+    # rows, scan, gather, 3 radix passes x 3 + item offsets, item pass, dH pass, finish
+    assert B.cutbce_kernel_launches(p, 2) == 16
     assert B.cutbce_kernel_launches(p, 0) == 5          # rows, scan, gather, item pass, finish
     assert B.cutbce_kernel_launches(p, 3) == -1
 

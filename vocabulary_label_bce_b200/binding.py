@@ -21,7 +21,7 @@ __all__ = [
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
     "cutbce_selftest_wait_timeout", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
-    "KERNEL_KINDS",
+    "KERNEL_KINDS", "cutbce_probe_scratch_bytes", "cutbce_probe_pipe_rate", "PROBES", "cutbce_probe_mma",
 ]
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TARGET_RANGE, ERR_TIMEOUT, ERR_CUDA = range(7)
@@ -68,8 +68,13 @@ _SIGS = {
     "cutbce_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
     "cutbce_profile_enable": (_i32, [ctypes.c_int]),
     "cutbce_profile_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64), ctypes.c_int]),
+    "cutbce_probe_scratch_bytes": (_sz, []),
+    "cutbce_probe_pipe_rate": (_i32, [ctypes.c_int, _vp, _sz, ctypes.POINTER(ctypes.c_double), _vp]),
+    "cutbce_probe_mma": (_i32, [ctypes.c_int, ctypes.c_int, _i64, _vp, _sz, ctypes.POINTER(ctypes.c_double),
+                                ctypes.POINTER(ctypes.c_double), _vp]),
 }
-KERNEL_KINDS = ["prep_rows", "prep_scan", "prep_gather", "group_sort", "item_pass", "position_pass", "finish",
+PROBES = ["ffma", "ffma2", "ex2", "rcp", "tanh", "lg2", "cvt_bf16x2", "fmax", "add2", "iadd", "prmt"]
+KERNEL_KINDS = ["prep_rows", "prep_scan", "prep_gather", "csc_offsets", "item_pass", "position_pass", "finish",
                 "pair_sort"]
 
 
@@ -210,3 +215,31 @@ def cutbce_profile_read(reset: bool = True) -> dict:
     cnt = (_i64 * n)()
     _check(load_library().cutbce_profile_read(ms, cnt, 1 if reset else 0), "cutbce_profile_read")
     return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def cutbce_probe_scratch_bytes() -> int:
+    return int(load_library().cutbce_probe_scratch_bytes())
+
+
+def cutbce_probe_pipe_rate(op: str | int, scratch: Optional[torch.Tensor] = None, stream=None) -> float:
+    """Operations of one kind an SM retires per clock (median over SMs)."""
+    k = PROBES.index(op) if isinstance(op, str) else int(op)
+    if scratch is None:
+        scratch = torch.empty(cutbce_probe_scratch_bytes(), dtype=torch.uint8, device="cuda")
+    r = ctypes.c_double(0.0)
+    _check(load_library().cutbce_probe_pipe_rate(k, scratch.data_ptr(), scratch.numel(), ctypes.byref(r),
+                                                 _stream(stream)), "cutbce_probe_pipe_rate")
+    return float(r.value)
+
+
+def cutbce_probe_mma(n: int, a_in_tmem: bool, iters: int = 4096, scratch: Optional[torch.Tensor] = None,
+                     stream=None, b_mn_major: bool = False) -> tuple[float, float]:
+    """(issue cycles, total cycles) per 128 x n x 16 bf16 tcgen05.mma, median over SMs."""
+    if scratch is None:
+        scratch = torch.empty(cutbce_probe_scratch_bytes(), dtype=torch.uint8, device="cuda")
+    a, b = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    flags = (1 if a_in_tmem else 0) | (2 if b_mn_major else 0)
+    _check(load_library().cutbce_probe_mma(int(n), flags, int(iters), scratch.data_ptr(),
+                                           scratch.numel(), ctypes.byref(a), ctypes.byref(b), _stream(stream)),
+           "cutbce_probe_mma")
+    return float(a.value), float(b.value)

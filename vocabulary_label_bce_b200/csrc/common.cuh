@@ -20,12 +20,12 @@ enum : int { kMeanValidPositions = 0, kSum = 1, kMeanElements = 2 };
 constexpr int kMaxK = 128;            // target slots per position
 constexpr int kMaxDim = 256;          // feature width
 constexpr int kTileM = 128;           // stationary rows per tile = TMEM lanes
-constexpr int kGroupRows = 128;       // rows per group of item-sorted pairs (= one position tile)
 constexpr int kMaxCtas = 256;         // upper bound of a persistent grid
 constexpr int kMaxSplits = 64;        // dH partial splits over the vocabulary
 constexpr int kTileThreads = 640;     // 20 warps: TMA, MMA, fix-up, idle, 16 epilogue
 constexpr int kEpiWarp0 = 4;
-constexpr int kNumEpiWarps = 16;      // 4 per TMEM lane quarter (one per SM sub-partition each)
+constexpr int kNumEpiWarps = 16;      // 2 groups x (4 TMEM lane quarters x 2 column slabs)
+constexpr int kEpiGroupWarps = 8;     // warps that take one tile
 
 // First 256 bytes of the workspace.
 struct WsHeader {
@@ -44,17 +44,24 @@ struct TileCfg {
   static_assert(DP % 64 == 0 && DP >= 64 && DP <= 256, "DP must be 64, 128, 192 or 256");
   static constexpr int BN = DP <= 128 ? 128 : 64;          // streamed rows per tile (Z columns)
   static constexpr int NKB = DP / 64;                        // 128-byte column blocks per row
-  static constexpr int NX = DP == 64 ? 4 : 3;                // stages of the streamed-operand ring
-  static constexpr int NZ = 3;                               // logit tiles in tensor memory
-  static constexpr int NG = DP == 128 ? 2 : 3;               // bf16 sigmoid tiles in shared memory
+  // stages of the streamed-operand ring: a streamed tile is held from its logit MMA
+  // (issued up to NZ-1 tiles early) until its gradient MMA completes, and the ring
+  // must still cover the L2 -> shared memory latency of the next loads
+  static constexpr int NX = DP == 64 ? 12 : DP == 128 ? 6 : DP == 192 ? 7 : 5;
+  static constexpr int NZ = 2;                               // fp32 logit tiles in tensor memory
+  static constexpr int NG = 2;                               // bf16 sigmoid tiles in tensor memory
   static constexpr uint32_t S_BYTES = kTileM * DP * 2;       // stationary tile
   static constexpr uint32_t X_BYTES = BN * DP * 2;           // streamed tile
-  static constexpr uint32_t G_BYTES = kTileM * BN * 2;       // bf16 sigmoid tile
-  static constexpr int ACC_COL = NZ * BN;                    // TMEM column of the gradient accumulator
+  static constexpr int G_COL = NZ * BN;                      // TMEM column of the first G buffer
+  static constexpr int G_COLS = BN / 2;                      // a G tile: BN bf16 per lane, two per column
+  static constexpr int ACC_COL = G_COL + NG * G_COLS;        // TMEM column of the gradient accumulator
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NUM_BARS = 2 + 2 * NX + 2 * NZ + 3 * NG + 3;  // see the kernel for the list
-  static constexpr uint32_t SMEM_BYTES =
-      1024 + S_BYTES + NX * X_BYTES + NG * G_BYTES + NUM_BARS * 8 + 16 + 64;
+  // The stationary tile is copied into tensor memory (bf16 pairs, DP/2 columns)
+  // when it fits, so the logit MMA reads only its B operand from shared memory.
+  static constexpr int S_COL = ACC_COL + DP;
+  static constexpr bool S_IN_TMEM = S_COL + DP / 2 <= TMEM_COLS;
+  static constexpr int NUM_BARS = 2 + 2 * NX + 2 * NZ + 2 * NG + 3;  // see the kernel for the list
+  static constexpr uint32_t SMEM_BYTES = 1024 + S_BYTES + NX * X_BYTES + NUM_BARS * 8 + 16 + 64;
   static_assert(ACC_COL + DP <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(SMEM_BYTES > 232448 / 2, "one CTA per SM keeps the TMEM allocation uncontended");

@@ -18,6 +18,7 @@
 #include "prep_finish.cuh"
 #include "pair_sort.cuh"
 #include "tile_engine.cuh"
+#include "probes.cuh"
 
 namespace {
 using namespace cutbce;
@@ -31,12 +32,12 @@ struct Plan {
   int64_t T, V, D, K;
   int dtype, reduction;
   int DP, BN;
-  int64_t Tpad, ngroups_max, n_vitems, n_gather_blocks;
+  int64_t Tpad, n_vitems, n_gather_blocks;
   int S, tps, n_vtiles_bn;
   int radix_passes, radix_blocks;
   size_t elem;
-  size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_grp_t, o_grp_v, o_srt[4], o_ghist,
-      o_istart, o_hc, o_lpart, o_cpart, o_dhpart, total;
+  size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_srt[4], o_ghist, o_cscoff, o_hc,
+      o_lpart, o_cpart, o_dhpart, total;
 };
 
 cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
@@ -69,13 +70,12 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.BN = (bf16 && pl.DP > 128) ? 64 : 128;
   pl.elem = bf16 ? 2 : 4;
   pl.Tpad = round_up(p->T, kTileM);
-  pl.ngroups_max = ceil_div(p->T, kGroupRows);
   pl.n_vitems = ceil_div(p->V, kTileM);
   pl.n_gather_blocks = ceil_div(pl.Tpad, 8);
   {
     int bits = 0;
-    while ((int64_t(1) << bits) < pl.n_vitems) ++bits;
-    pl.radix_passes = (bits + 7) / 8;     // 8-bit digits of the item-tile index
+    while ((int64_t(1) << bits) < p->V) ++bits;
+    pl.radix_passes = (bits + 7) / 8;     // 8-bit digits of the item id
     pl.radix_blocks = static_cast<int>(std::max<int64_t>(1, ceil_div(p->T * p->K, kRadixTile)));
   }
   if (bf16) {
@@ -105,11 +105,9 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.o_ids = take(4 * TK);
   pl.o_pair_t = take(4 * TK);
   pl.o_pair_v = take(4 * TK);
-  pl.o_grp_t = take(4 * TK);
-  pl.o_grp_v = take(4 * TK);
   for (int k = 0; k < 4; ++k) pl.o_srt[k] = take(4 * TK);
   pl.o_ghist = take(4 * 256 * static_cast<size_t>(pl.radix_blocks));
-  pl.o_istart = take(4 * static_cast<size_t>(pl.n_vitems + 1));
+  pl.o_cscoff = take(4 * static_cast<size_t>(p->V + 1));
   pl.o_hc = take(pl.elem * static_cast<size_t>(pl.Tpad) * pl.DP);
   pl.o_lpart = take(8 * kNumEpiWarps * pl.n_vitems);
   pl.o_cpart = take(8 * pl.n_gather_blocks);
@@ -271,8 +269,7 @@ struct Want {
 int count_launches(const Plan& pl, Want w) {
   const bool bf16 = pl.dtype == CUTBCE_BF16;
   int n = 3;                                            // rows, scan, gather
-  if (bf16 && w.dH) n += 1;                             // group sort
-  if (bf16 && w.dE) n += 3 * pl.radix_passes + 1;       // radix passes and item ranges
+  if (bf16 && w.dE) n += 3 * pl.radix_passes + 1;       // radix passes and item offsets
   if (w.loss || w.dE) n += 1;                           // item-owned pass
   if (w.dH) n += 1;                                     // position-owned pass
   if (w.loss || w.dH) n += 1;                           // finish
@@ -303,11 +300,9 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   int* ids = at<int>(ws, pl.o_ids);
   int* pair_t = at<int>(ws, pl.o_pair_t);
   int* pair_v = at<int>(ws, pl.o_pair_v);
-  int* grp_t = at<int>(ws, pl.o_grp_t);
-  int* grp_v = at<int>(ws, pl.o_grp_v);
   double* lpart = at<double>(ws, pl.o_lpart);
   double* cpart = at<double>(ws, pl.o_cpart);
-  int* istart = at<int>(ws, pl.o_istart);
+  int* cscoff = at<int>(ws, pl.o_cscoff);
   int* ghist = at<int>(ws, pl.o_ghist);
   float* dhpart = at<float>(ws, pl.o_dhpart);
 
@@ -344,39 +339,26 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
 
   const bool item_pass = w.loss || w.dE;
   if (bf16) {
-    if (w.dH) {
-      // pairs of each 128-row group ordered by (item, position) for the position-owned pass
-      int npow = 1;
-      while (npow < kGroupRows * K) npow <<= 1;
-      const size_t smem = static_cast<size_t>(npow) * 8;
-      static bool sort_cfg = false;
-      if (!sort_cfg) {
-        CUTBCE_CK(cudaFuncSetAttribute(k_group_sort, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kGroupRows * kMaxK * 8)));
-        sort_cfg = true;
-      }
-      LaunchScope ls(CUTBCE_KERNEL_GROUP_SORT, st);
-      k_group_sort<<<static_cast<unsigned>(pl.ngroups_max), 256, smem, st>>>(rowptr, pair_t, pair_v, hdr, grp_t,
-                                                                             grp_v);
-      CUTBCE_CK(cudaGetLastError());
-    }
-    const int* srt_v = pair_v;
-    const int* srt_t = pair_t;
+    const int* csc_v = pair_v;
+    const int* csc_t = pair_t;
     if (w.dE) {
-      // pairs ordered by (item tile, position): stable LSD radix sort on the item-tile index
+      // pairs ordered by (item, position): stable LSD radix sort on the item id, then offsets
       LaunchScope ls(CUTBCE_KERNEL_PAIR_SORT, st);
       for (int pass = 0; pass < pl.radix_passes; ++pass) {
         int* out_v = at<int>(ws, pl.o_srt[2 * (pass & 1)]);
         int* out_t = at<int>(ws, pl.o_srt[2 * (pass & 1) + 1]);
-        k_radix_hist<<<pl.radix_blocks, kRadixThreads, 0, st>>>(srt_v, hdr, 8 * pass, pl.radix_blocks, ghist);
+        k_radix_hist<<<pl.radix_blocks, kRadixThreads, 0, st>>>(csc_v, hdr, 8 * pass, pl.radix_blocks, ghist);
         k_exclusive_scan<<<1, 1024, 0, st>>>(ghist, 256 * pl.radix_blocks);
-        k_radix_scatter<<<pl.radix_blocks, kRadixThreads, 0, st>>>(srt_v, srt_t, out_v, out_t, hdr, 8 * pass,
+        k_radix_scatter<<<pl.radix_blocks, kRadixThreads, 0, st>>>(csc_v, csc_t, out_v, out_t, hdr, 8 * pass,
                                                                    pl.radix_blocks, ghist);
-        srt_v = out_v;
-        srt_t = out_t;
+        csc_v = out_v;
+        csc_t = out_t;
       }
-      k_item_ranges<<<static_cast<unsigned>(ceil_div(pl.n_vitems + 1, 256)), 256, 0, st>>>(
-          srt_v, hdr, static_cast<int>(pl.n_vitems), istart);
+      CUTBCE_CK(cudaGetLastError());
+    }
+    if (w.dE) {
+      LaunchScope ls(CUTBCE_KERNEL_CSC_OFFSETS, st);
+      k_csc_offsets<<<static_cast<unsigned>(ceil_div(V + 1, 256)), 256, 0, st>>>(csc_v, hdr, V, cscoff);
       CUTBCE_CK(cudaGetLastError());
     }
     TileParams tp{};
@@ -385,11 +367,9 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     tp.Tpad = pl.Tpad;
     tp.hdr = hdr;
     tp.row_ptr = rowptr;
-    tp.grp_v = grp_v;
-    tp.grp_t = grp_t;
-    tp.srt_t = srt_t;
-    tp.srt_v = srt_v;
-    tp.item_start = istart;
+    tp.pair_v = pair_v;
+    tp.csc_off = cscoff;
+    tp.csc_t = csc_t;
     tp.dE = dE;
     tp.loss_part = lpart;
     tp.dh_part = dhpart;
@@ -617,6 +597,105 @@ cutbce_status cutbce_profile_read(double* ms, int64_t* launches, int reset) {
       g_prof.launches[k] = 0;
     }
   }
+  return CUTBCE_OK;
+}
+
+size_t cutbce_probe_scratch_bytes(void) { return 16 * kMaxCtas + 4 * kProbeThreads; }
+
+cutbce_status cutbce_probe_pipe_rate(int op, void* scratch, size_t scratch_bytes, double* ops_per_clock_per_sm,
+                                     cutbce_stream_t stream) {
+  if (op < 0 || op >= kProbeCount || scratch == nullptr || ops_per_clock_per_sm == nullptr ||
+      scratch_bytes < cutbce_probe_scratch_bytes())
+    return CUTBCE_ERR_INVALID_ARG;
+  DeviceFacts dev;
+  cutbce_status s = device_facts(dev);
+  if (s != CUTBCE_OK) return s;
+  const int grid = std::min(dev.sms, kMaxCtas);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* cycles = static_cast<unsigned long long*>(scratch);
+  float* sink = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + 16 * kMaxCtas);
+  constexpr int kIters = 2048;
+  constexpr int kSmem = 120 * 1024;   // more than half of an SM's shared memory: one CTA per SM
+  cudaError_t e = cudaSuccess;
+  auto launch = [&](auto kern) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e == cudaSuccess) {
+      kern<<<grid, kProbeThreads, kSmem, st>>>(kIters, cycles, sink);
+      e = cudaGetLastError();
+    }
+  };
+  switch (op) {
+    case kProbeFfma: launch(k_probe<kProbeFfma>); break;
+    case kProbeFfma2: launch(k_probe<kProbeFfma2>); break;
+    case kProbeEx2: launch(k_probe<kProbeEx2>); break;
+    case kProbeRcp: launch(k_probe<kProbeRcp>); break;
+    case kProbeTanh: launch(k_probe<kProbeTanh>); break;
+    case kProbeLg2: launch(k_probe<kProbeLg2>); break;
+    case kProbeCvtBf16x2: launch(k_probe<kProbeCvtBf16x2>); break;
+    case kProbeFmax: launch(k_probe<kProbeFmax>); break;
+    case kProbeAdd2: launch(k_probe<kProbeAdd2>); break;
+    case kProbeIadd: launch(k_probe<kProbeIadd>); break;
+    default: launch(k_probe<kProbePrmt>); break;
+  }
+  if (e != cudaSuccess) return CUTBCE_ERR_CUDA;
+  std::vector<unsigned long long> h(grid);
+  if (cudaMemcpyAsync(h.data(), cycles, 8 * grid, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return CUTBCE_ERR_CUDA;
+  std::sort(h.begin(), h.end());
+  const double ops = static_cast<double>(kProbeThreads) * kIters * kProbeChains * ((op == kProbeFfma2 || op == kProbeAdd2) ? 2 : 1);
+  *ops_per_clock_per_sm = h[grid / 2] > 0 ? ops / static_cast<double>(h[grid / 2]) : 0.0;
+  return CUTBCE_OK;
+}
+
+cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratch, size_t scratch_bytes,
+                               double* issue_cycles_per_mma, double* cycles_per_mma, cutbce_stream_t stream) {
+  if ((n != 64 && n != 128 && n != 256) || iters <= 0 || iters > (1 << 24) || scratch == nullptr ||
+      scratch_bytes < cutbce_probe_scratch_bytes() || issue_cycles_per_mma == nullptr || cycles_per_mma == nullptr)
+    return CUTBCE_ERR_INVALID_ARG;
+  DeviceFacts dev;
+  cutbce_status s = device_facts(dev);
+  if (s != CUTBCE_OK) return s;
+  if (!(dev.major == 10 && dev.minor == 0)) return CUTBCE_ERR_UNSUPPORTED;
+  const int grid = std::min(dev.sms, kMaxCtas);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* out = static_cast<unsigned long long*>(scratch);
+  const int smem = 1024 + 16384 + n * 128 + 16 * 2048;
+  const int smem_req = std::max(smem, 120 * 1024);   // one CTA per SM: TMEM allocation uncontended
+  cudaError_t e = cudaSuccess;
+  auto launch = [&](auto kern) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_req);
+    if (e == cudaSuccess) {
+      kern<<<grid, 128, smem_req, st>>>(static_cast<int>(iters), out);
+      e = cudaGetLastError();
+    }
+  };
+  const bool bmn = (a_in_tmem & 2) != 0;
+  const bool at = (a_in_tmem & 1) != 0;
+  if (n == 64) {
+    if (bmn) at ? launch(k_probe_mma<64, true, true>) : launch(k_probe_mma<64, false, true>);
+    else at ? launch(k_probe_mma<64, true, false>) : launch(k_probe_mma<64, false, false>);
+  } else if (n == 128) {
+    if (bmn) at ? launch(k_probe_mma<128, true, true>) : launch(k_probe_mma<128, false, true>);
+    else at ? launch(k_probe_mma<128, true, false>) : launch(k_probe_mma<128, false, false>);
+  } else {
+    if (bmn) at ? launch(k_probe_mma<256, true, true>) : launch(k_probe_mma<256, false, true>);
+    else at ? launch(k_probe_mma<256, true, false>) : launch(k_probe_mma<256, false, false>);
+  }
+  if (e != cudaSuccess) return CUTBCE_ERR_CUDA;
+  std::vector<unsigned long long> h(2 * grid);
+  if (cudaMemcpyAsync(h.data(), out, 16 * grid, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return CUTBCE_ERR_CUDA;
+  std::vector<unsigned long long> issue(grid), total(grid);
+  for (int b = 0; b < grid; ++b) {
+    issue[b] = h[2 * b];
+    total[b] = h[2 * b + 1];
+  }
+  std::sort(issue.begin(), issue.end());
+  std::sort(total.begin(), total.end());
+  *issue_cycles_per_mma = static_cast<double>(issue[grid / 2]) / static_cast<double>(iters);
+  *cycles_per_mma = static_cast<double>(total[grid / 2]) / static_cast<double>(iters);
   return CUTBCE_OK;
 }
 

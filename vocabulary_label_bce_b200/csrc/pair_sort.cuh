@@ -1,15 +1,11 @@
-// Ordering of the (position, item) pairs for the two tensor-core passes.
+// Item-major order of the (position, item) pairs (a CSC of the sparse target
+// matrix Y) for the item-owned tensor-core pass: every item's positives as an
+// ascending list of compacted positions, so that the epilogue thread owning an
+// item row walks them with a forward-only cursor as position tiles stream by.
 //
-//  * item-owned pass: pairs ordered by item tile (v / 128), then by position t
-//    (then by v).  A stable LSD radix sort on the item-tile index does this,
-//    because the pairs are produced in (t, v) order.  Each item tile then owns
-//    one contiguous, position-sorted range: its fix-up cursor only moves forward
-//    as the position tiles stream by.
-//  * position-owned pass: pairs of each group of 128 compacted rows ordered by
-//    (v, t) (a bitonic sort per group in shared memory), so the cursor of a
-//    position tile moves forward as the item tiles stream by.
-//
-// Every result is unique (pairs are distinct), so the order is deterministic.
+// The pairs are produced in (position, item) order; a stable LSD radix sort on
+// the item id therefore yields (item, position) order.  Every result is unique
+// (pairs are distinct), so the order is deterministic.
 #pragma once
 #include <cstdint>
 #include "common.cuh"
@@ -20,7 +16,7 @@ constexpr int kRadixThreads = 256;
 constexpr int kRadixTile = 4096;                 // pairs per block
 constexpr int kRadixRounds = kRadixTile / kRadixThreads;
 
-__device__ __forceinline__ int item_tile_digit(int v, int shift) { return ((v >> 7) >> shift) & 255; }
+__device__ __forceinline__ int item_digit(int v, int shift) { return (v >> shift) & 255; }
 
 // Per-block digit histogram, stored digit-major: ghist[d * nblk + blk].
 __global__ void __launch_bounds__(kRadixThreads) k_radix_hist(const int* __restrict__ keys, const WsHeader* hdr,
@@ -32,7 +28,7 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_hist(const int* __restr
   const int base = blockIdx.x * kRadixTile;
   for (int i = threadIdx.x; i < kRadixTile; i += kRadixThreads) {
     const int idx = base + i;
-    if (idx < n) atomicAdd(&h[item_tile_digit(keys[idx], shift)], 1);
+    if (idx < n) atomicAdd(&h[item_digit(keys[idx], shift)], 1);
   }
   __syncthreads();
   ghist[threadIdx.x * nblk + blockIdx.x] = h[threadIdx.x];
@@ -112,7 +108,7 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(const int* __re
     const bool valid = idx < n;
     const int key = valid ? keys_in[idx] : 0;
     const int val = valid ? vals_in[idx] : 0;
-    const int d = valid ? item_tile_digit(key, shift) : 256;
+    const int d = valid ? item_digit(key, shift) : 256;
     const unsigned peers = __match_any_sync(0xffffffffu, d);
     const int rank = __popc(peers & lt_mask);
     if (valid && rank == 0) wcnt[warp][d] = __popc(peers);
@@ -141,21 +137,19 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(const int* __re
   }
 }
 
-// item_start[i] = first index of the item-tile-sorted pairs whose item is >= 128*i,
-// for i in [0, n_items]; item tile i owns [item_start[i], item_start[i+1]).
-__global__ void k_item_ranges(const int* __restrict__ sorted_v, const WsHeader* hdr, int n_items,
-                              int* __restrict__ item_start) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i > n_items) return;
-  const int n = hdr->n_pairs;
-  const int target = i * kTileM;
-  int lo = 0, hi = n;
+// csc_off[v] = first index of the item-sorted pairs whose item is >= v, for v in
+// [0, V]; item v owns [csc_off[v], csc_off[v+1]).
+__global__ void k_csc_offsets(const int* __restrict__ sorted_v, const WsHeader* hdr, int V,
+                              int* __restrict__ csc_off) {
+  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  if (v > V) return;
+  int lo = 0, hi = hdr->n_pairs;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    if (sorted_v[mid] < target) lo = mid + 1;
+    if (sorted_v[mid] < v) lo = mid + 1;
     else hi = mid;
   }
-  item_start[i] = lo;
+  csc_off[v] = lo;
 }
 
 }  // namespace cutbce

@@ -207,51 +207,6 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
   }
 }
 
-// ------------------------------------------------------------------ prep: group sort
-// One block per group of 64 compacted rows: sorts the group's pairs by
-// (item, position) so that the tile engine can walk, for any range of items,
-// the positives that fall inside a tile with a forward-only cursor.
-__global__ void __launch_bounds__(256) k_group_sort(const int* __restrict__ row_ptr,
-                                                    const int* __restrict__ pair_t,
-                                                    const int* __restrict__ pair_v, const WsHeader* hdr,
-                                                    int* __restrict__ grp_t, int* __restrict__ grp_v) {
-  extern __shared__ unsigned long long keys[];
-  const int nv = hdr->n_valid;
-  const int r0 = blockIdx.x * kGroupRows;
-  if (r0 >= nv) return;
-  const int r1 = min(r0 + kGroupRows, nv);
-  const int p0 = row_ptr[r0], p1 = row_ptr[r1];
-  const int n = p1 - p0;
-  if (n == 0) return;
-  int npow = 1;
-  while (npow < n) npow <<= 1;
-  for (int i = threadIdx.x; i < npow; i += blockDim.x)
-    keys[i] = i < n ? ((static_cast<unsigned long long>(pair_v[p0 + i]) << 32) |
-                       static_cast<unsigned int>(pair_t[p0 + i]))
-                    : ~0ull;
-  __syncthreads();
-  for (int k = 2; k <= npow; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < npow; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const bool up = (i & k) == 0;
-          const unsigned long long a = keys[i], b = keys[ixj];
-          if ((a > b) == up) {
-            keys[i] = b;
-            keys[ixj] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    grp_v[p0 + i] = static_cast<int>(keys[i] >> 32);
-    grp_t[p0 + i] = static_cast<int>(keys[i] & 0xffffffffu);
-  }
-}
-
 // ------------------------------------------------------------------ finish
 // dH[t, d] = g*s * sum_{split} partial[split][c(t)][d] in split order (0 for
 // masked rows); the last block also forms loss = s * (dense - correction),

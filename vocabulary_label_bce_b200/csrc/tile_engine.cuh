@@ -1,40 +1,49 @@
 // The tensor-core engine: one persistent, warp-specialised sm_100a kernel
 // template that forms logit tiles on tcgen05 (accumulators in tensor memory),
 // applies the BCE element math to them in registers and, for the gradient,
-// feeds the bf16 tile of G = sigmoid(X) - Y straight back into a second
-// tcgen05 contraction.  No logit or gradient tile ever leaves the SM.
+// writes the bf16 tile of G = sigmoid(X) - Y back into tensor memory, where
+// the second tcgen05 contraction reads it as its A operand.  No logit or
+// gradient tile ever leaves the SM, and G never touches shared memory.
 //
 // Two instantiations cover the hot path of "Cut Binary Cross Entropy"
 // (section III-A Eqs. (2)-(3); section III-B Eq. (4)):
 //
 //   item-owned pass (kDH = false): a CTA owns a tile of 128 items v (rows of E,
 //     the stationary operand) and streams every tile of the compacted H.
-//     Z^T = E_v H_t^T  -> softplus sum (loss) and sigmoid -> G^T (bf16, smem)
+//     Z^T = E_v H_t^T  -> softplus sum (loss) and sigmoid -> G^T (bf16, TMEM)
 //     dE_v += G^T H_t  (accumulated in TMEM across all t, written once, no atomics)
 //
 //   position-owned pass (kDH = true): a CTA owns a tile of 128 valid positions
 //     (rows of H) and streams the item tiles of one vocabulary split.
-//     Z = H_t E_v^T    -> sigmoid -> G (bf16, smem)
+//     Z = H_t E_v^T    -> sigmoid -> G (bf16, TMEM)
 //     dH_t += G E_v    (partial per split, reduced later in a fixed order)
 //
-// The sparse targets enter in-tile: after the epilogue warps write sigmoid(z)
-// for a tile, a fix-up warp subtracts 1 at the (at most a few) positions of the
-// tile where y = 1, walking lists of pairs pre-sorted by item.  The dense loss
-// term uses no Y at all (Eq. (2): l(x,y) = l(x,0) - y x); the -y x part is the
-// separate sparse correction summed in the prep kernel.
+// The sparse targets enter in registers: each epilogue thread owns one row of
+// the tile and walks that row's sorted positives with a forward-only cursor;
+// where a positive falls in the current 32-column chunk it subtracts 1 from
+// sigmoid(z) (y = 1).  The dense loss uses no Y at all (Eq. (2):
+// l(x,y) = l(x,0) - y x); the -y x part is the sparse correction summed in the
+// prep kernel.
 //
 // Warp roles (640 threads, one CTA per SM):
 //   warp 0      TMA producer (stationary tile, ring of streamed tiles)
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warp 2      fix-up warp (Y in-tile)
-//   warp 3      idle
-//   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. and one quarter
-//               of the tile's columns
+//   warps 2-3   idle
+//   warps 4-19  epilogue, two groups of 8 taking alternate tiles; in a group,
+//               warp w reads TMEM lanes 32*(w%4).. and one of two column slabs
+//
+// Tensor memory holds NZ fp32 logit buffers, NG bf16 G buffers, the gradient
+// accumulator and, where it fits, a copy of the stationary tile (the logit
+// MMA's A operand, so that only its B operand is read from shared memory).
+// A logit buffer is free again as soon as the epilogue group has loaded it; a
+// G buffer once the gradient MMA that reads it has completed.  With two groups
+// on alternate tiles, each group's next logit tile is computed while it still
+// works on the current one.
 //
 // Every wait is bounded (global timer); on expiry the CTA records
-// CUTBCE_ERR_TIMEOUT in the status word, the other roles leave their loops, the
-// producer and the MMA issuer wait (bounded) for their own copies and MMAs in
-// flight, and the CTA frees its tensor memory and returns.
+// CUTBCE_ERR_TIMEOUT and where it happened in the workspace header, the other
+// roles leave their loops, the producer and the MMA issuer wait (bounded) for
+// their own copies and MMAs in flight, and the CTA frees its tensor memory.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -49,12 +58,10 @@ struct TileParams {
   int D;                       // real feature width (<= DP)
   int64_t Tpad;                // rows of H_c (multiple of 128)
   WsHeader* hdr;               // n_valid, grad scale, status
-  const int* row_ptr;          // [n_valid + 1] pair offsets of compacted rows
-  const int* grp_v;            // position-owned pass: pairs sorted by (item, position) per 128-row group
-  const int* grp_t;
-  const int* srt_t;            // item-owned pass: pairs sorted by (item tile, position, item)
-  const int* srt_v;
-  const int* item_start;       // item-owned pass: [n_item_tiles + 1] ranges into srt_*
+  const int* row_ptr;          // [n_valid + 1] pair offsets of compacted rows (CSR by position)
+  const int* pair_v;           // CSR by position: items of each row, ascending
+  const int* csc_off;          // [V + 1] offsets into csc_t (CSC by item)
+  const int* csc_t;            // CSC by item: positions of each item, ascending
   float* dE;                   // item-owned pass output [V, D] (may be null when no gradient)
   double* loss_part;           // item-owned pass: one double per (item tile, epilogue warp)
   float* dh_part;              // position-owned pass output [S, Tpad, DP]
@@ -71,7 +78,7 @@ struct WaitCtx {
 };
 
 // Where a wait happens, recorded if it gives up: role (1 producer, 2 MMA,
-// 3 fix-up, 4 epilogue), barrier id, and the role's tile or item counter.
+// 4 epilogue), barrier id, and the role's tile or item counter.
 __device__ __forceinline__ int wait_tag(int role, int barrier, uint32_t counter) {
   return (role << 28) | (barrier << 20) | static_cast<int>(counter & 0xFFFFFu);
 }
@@ -83,7 +90,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const W
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*w.abort_flag) {
       // record where each role stood when the CTA gave up (first record per role wins)
       if (tag != 0) atomicCAS(reinterpret_cast<int*>(w.hdr) + 8 + ((tag >> 28) & 7), 0, tag);
@@ -107,10 +114,19 @@ __device__ __forceinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity, l
   }
   return true;
 }
-// Whole-warp wait with a warp-uniform result.
+// Whole-warp wait: lane 0 waits, the warp then synchronises with it (which
+// orders the other lanes after lane 0's acquire of the barrier phase).
 __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w, int tag = 0) {
-  const bool ok = wait_bar(bar, parity, w, tag);
-  return __all_sync(0xffffffffu, ok);
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, w, tag);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Warp-uniform non-blocking test of a barrier phase (lane 0 tests, the warp shares the answer).
+__device__ __forceinline__ bool test_bar_warp(uint64_t* bar, uint32_t parity) {
+  bool ok = false;
+  if ((threadIdx.x & 31) == 0) ok = mbar_test_wait(bar, parity);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 struct ItemInfo {
@@ -140,53 +156,30 @@ __device__ __forceinline__ ItemInfo item_info(int i, int n_valid, const TilePara
   return it;
 }
 
-// Forward-only cursor over one sorted pair range, lane-uniform.  `nxt` holds
-// the key (position for the item-owned pass, item for the position-owned pass)
-// of the next unapplied pair, so a tile without positives costs no memory
-// access.  Every pair with key < hi is applied to the bf16 G tile by
-// subtracting 1 (y = 1 in G = sigmoid(X) - Y).
-struct PairCursor {
+// Forward-only cursor over one row's ascending positive keys (positions for the
+// item-owned pass, items for the position-owned pass).
+struct RowCursor {
   int cur, end, nxt;
 };
 
-template <bool kDH>
-__device__ __forceinline__ void fixup_apply(PairCursor& c, int hi, int x0, int s0, uint8_t* G,
-                                            const int* __restrict__ keys, const int* __restrict__ others,
-                                            int lane) {
-  while (c.nxt < hi) {
-    const int idx = c.cur + lane;
-    const int key = idx < c.end ? __ldg(keys + idx) : 0x7fffffff;
-    const bool in = key < hi;
-    if (in) {
-      const int other = __ldg(others + idx);
-      // item-owned: rows are items, columns are positions; position-owned: the reverse
-      const int row = other - s0;
-      const int col = key - x0;
-      const uint32_t off = static_cast<uint32_t>(col >> 6) * 16384u + static_cast<uint32_t>(row) * 128u +
-                           ((((static_cast<uint32_t>(col) & 63u) >> 3) ^ (static_cast<uint32_t>(row) & 7u)) << 4) +
-                           ((static_cast<uint32_t>(col) & 7u) << 1);
-      __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(G + off);
-      *e = __float2bfloat16_rn(__bfloat162float(*e) - 1.0f);
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, in);
-    const int n = __popc(m);
-    c.cur += n;
-    if (n < 32) {
-      c.nxt = __shfl_sync(0xffffffffu, key, n);
-    } else {
-      c.nxt = c.cur < c.end ? __ldg(keys + c.cur) : 0x7fffffff;
-    }
-  }
+__device__ __forceinline__ void cursor_init(RowCursor& rc, const int* __restrict__ keys, int begin, int end,
+                                            int first_key) {
+  int c = begin;
+  while (c < end && __ldg(keys + c) < first_key) ++c;
+  rc.cur = c;
+  rc.end = end;
+  rc.nxt = c < end ? __ldg(keys + c) : 0x7fffffff;
 }
 
-// First index in [lo, hi) of an ascending int array whose value is >= target.
-__device__ __forceinline__ int lower_bound_idx(const int* __restrict__ a, int lo, int hi, int target) {
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(a + mid) < target) lo = mid + 1;
-    else hi = mid;
+// Bit e set for each positive whose key is lo + e, e in [0, 32); advances the cursor.
+__device__ __forceinline__ uint32_t cursor_take_mask(RowCursor& rc, const int* __restrict__ keys, int lo) {
+  uint32_t mask = 0;
+  while (rc.nxt < lo + 32) {
+    mask |= 1u << (rc.nxt - lo);
+    ++rc.cur;
+    rc.nxt = rc.cur < rc.end ? __ldg(keys + rc.cur) : 0x7fffffff;
   }
-  return lo;
+  return mask;
 }
 
 template <int DP, bool kLoss, bool kGrad, bool kDH>
@@ -198,7 +191,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   constexpr int NX = Cfg::NX;
   constexpr int NZ = Cfg::NZ;
   constexpr int NG = Cfg::NG;
-  constexpr uint32_t S_BYTES = Cfg::S_BYTES, X_BYTES = Cfg::X_BYTES, G_BYTES = Cfg::G_BYTES;
+  constexpr uint32_t S_BYTES = Cfg::S_BYTES, X_BYTES = Cfg::X_BYTES;
   constexpr int ACC_COL = Cfg::ACC_COL;
   static_assert(!kDH || (kGrad && !kLoss), "the position-owned pass computes dH only");
   static_assert(kLoss || kGrad, "nothing to do");
@@ -209,18 +202,16 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sS = smem;
   uint8_t* sX = sS + S_BYTES;
-  uint8_t* sG = sX + NX * X_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + NG * G_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + NX * X_BYTES);
   uint64_t* bar_sfull = bars + 0;                 // stationary tile landed (TMA)
   uint64_t* bar_sempty = bars + 1;                // stationary tile free (MMA commit)
   uint64_t* bar_xfull = bars + 2;                 // [NX] streamed tile landed
   uint64_t* bar_xempty = bar_xfull + NX;          // [NX] streamed tile free
   uint64_t* bar_zfull = bar_xempty + NX;          // [NZ] logit tile ready in TMEM
-  uint64_t* bar_zempty = bar_zfull + NZ;          // [NZ] logit tile read by the epilogue
-  uint64_t* bar_gwritten = bar_zempty + NZ;       // [NG] sigmoid tile written by the epilogue
-  uint64_t* bar_fixdone = bar_gwritten + NG;      // [NG] target fix-ups of the tile applied
-  uint64_t* bar_gempty = bar_fixdone + NG;        // [NG] sigmoid tile consumed by the MMA
-  uint64_t* bar_accfull = bar_gempty + NG;        // gradient accumulator complete
+  uint64_t* bar_zfree = bar_zfull + NZ;           // [NZ] logit tile loaded by the epilogue group
+  uint64_t* bar_gready = bar_zfree + NZ;          // [NG] G tile written by the epilogue group
+  uint64_t* bar_gfree = bar_gready + NG;          // [NG] G tile consumed by the gradient MMA
+  uint64_t* bar_accfull = bar_gfree + NG;         // gradient accumulator complete
   uint64_t* bar_accempty = bar_accfull + 1;       // gradient accumulator read out
   uint64_t* bar_drain = bar_accempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
@@ -265,15 +256,14 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
     for (int b = 0; b < NZ; ++b) {
       mbar_init(bar_zfull + b, 1);
-      mbar_init(bar_zempty + b, kNumEpiWarps);
+      mbar_init(bar_zfree + b, kEpiGroupWarps);
     }
     for (int b = 0; b < NG; ++b) {
-      mbar_init(bar_gwritten + b, kNumEpiWarps);
-      mbar_init(bar_fixdone + b, 1);
-      mbar_init(bar_gempty + b, 1);
+      mbar_init(bar_gready + b, kEpiGroupWarps);
+      mbar_init(bar_gfree + b, 1);
     }
     mbar_init(bar_accfull, 1);
-    mbar_init(bar_accempty, kNumEpiWarps);
+    mbar_init(bar_accempty, kEpiGroupWarps);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -328,206 +318,262 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    // One thread.  Logit tiles (Z) run up to NZ tiles ahead of the gradient
-    // MMAs, so the epilogue always finds its next tile computed.
-    if (lane == 0) {
+    // The whole warp runs this loop; lane 0 tests the barriers and shares the
+    // answer, one elected lane issues each tcgen05 instruction.  It is an event
+    // loop over two in-order streams: logit tiles Z(c) (ready once their
+    // streamed tile has landed and their logit buffer has been loaded by the
+    // epilogue) and gradient MMAs G(c) (ready once the epilogue group has
+    // written the G tile).  Whichever is ready is issued, so a logit tile for
+    // one epilogue group never waits behind the other group's gradient tile.
+    //
+    // Shared-memory descriptors are built once and advanced by adding the byte
+    // offset / 16 to their 14-bit start-address field (it cannot carry out:
+    // shared memory is below 256 KB); ring positions are counters that wrap.
+    {
       constexpr uint32_t idesc_z = idesc_bf16_f32(kTileM, BN, false, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kTileM, DP, false, true);
-      const uint32_t sS_a = smem_u32(sS), sX_a = smem_u32(sX), sG_a = smem_u32(sG);
+      constexpr uint32_t kXStep = X_BYTES >> 4;                       // one ring stage, in descriptor units
+      static_assert(NZ == 2 && NG == 2, "ring positions below use & 1");
+      const uint64_t dS = smem_desc_sw128(smem_u32(sS), 16, 1024);     // stationary tile, K-major
+      const uint64_t dXk = smem_desc_sw128(smem_u32(sX), 16, 1024);    // streamed tile as K-major B
+      const uint64_t dXmn = smem_desc_sw128(smem_u32(sX), BN * 128, 1024);  // streamed tile as MN-major B
+      const uint32_t tZ = tmem_base, tG = tmem_base + Cfg::G_COL, tAcc = tmem_base + ACC_COL,
+                     tS = tmem_base + Cfg::S_COL;
       int zi = blockIdx.x, zj = 0, gi = blockIdx.x, gj = 0;
       uint32_t zic = 0, cz = 0, gic = 0, cg = 0;
+      uint32_t zst = 0, zph = 0, zoff = 0;        // ring stage of the next logit tile, its phase, its offset
+      uint32_t gst = 0, goff = 0;                 // ring stage of the next gradient MMA, its offset
+      bool s_ready = false;                       // the current item's stationary tile is in place
       ItemInfo zit{}, git{};
       if (zi < n_items) zit = git = item_info<DP, kDH>(zi, n_valid, p);
-      // Z[cz % NZ] = S * X^T : both operands K-major, 128-byte swizzle
-      auto issue_next_z = [&]() -> bool {
-        if (zj == 0) {
-          if (!wait_bar(bar_sfull, zic & 1, wc, wait_tag(2, 0, zic))) return false;
-          tc_fence_after();
-        }
-        const uint32_t st = cz % NX, b = cz % NZ;
-        if (!wait_bar(bar_xfull + st, (cz / NX) & 1, wc, wait_tag(2, 2, cz))) return false;
-        if (!wait_bar(bar_zempty + b, ((cz / NZ) & 1) ^ 1, wc, wait_tag(2, 5, cz))) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < DP / 16; ++ks) {
-          const uint64_t a = smem_desc_sw128(sS_a + (ks >> 2) * (kTileM * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sX_a + st * X_BYTES + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
-          umma_bf16(tmem_base + b * BN, a, bd, idesc_z, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_zfull + b);
-        if (!kGrad) umma_commit(bar_xempty + st);
-        ++cz;
-        if (++zj == zit.n_x) {
-          umma_commit(bar_sempty);                 // the stationary tile is no longer read
-          zj = 0;
-          ++zic;
-          zi += gridDim.x;
-          if (zi < n_items) zit = item_info<DP, kDH>(zi, n_valid, p);
-        }
-        return true;
-      };
+      uint64_t idle_since = 0;
       bool ok = true;
-      if (!kGrad) {
-        while (ok && zi < n_items) ok = issue_next_z();
-      } else {
-        while (ok && gi < n_items) {
-          while (ok && zi < n_items && cz < cg + NZ) ok = issue_next_z();
-          if (!ok) break;
-          const uint32_t b = cg % NG, st = cg % NX;
-          if (!wait_bar(bar_gwritten + b, (cg / NG) & 1, wc, wait_tag(2, 6, cg)) ||
-              !wait_bar(bar_fixdone + b, (cg / NG) & 1, wc, wait_tag(2, 7, cg)))
-            break;
-          tc_fence_after();
-          if (gj == 0) {
-            if (!wait_bar(bar_accempty, (gic & 1) ^ 1, wc, wait_tag(2, 10, gic))) break;
+      while (ok && (zi < n_items || (kGrad && gi < n_items))) {
+        bool progressed = false;
+        // ---- logit tile Z(cz) into buffer cz & 1
+        if (zi < n_items) {
+          if (zj == 0 && !s_ready && test_bar_warp(bar_sfull, zic & 1)) {
             tc_fence_after();
-          }
-          // ACC += G[b] * X[st] : G K-major, X read MN-major (its rows are the K index)
+            s_ready = true;
+            if (Cfg::S_IN_TMEM) {
+              // stationary tile -> tensor memory once per item; its shared-memory buffer is then free
+              if (elect_one()) {
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t a = smem_desc_sw128(sG_a + b * G_BYTES + (ks >> 2) * (kTileM * 128) + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sX_a + st * X_BYTES + ks * 2048, BN * 128, 1024);
-            umma_bf16(tmem_base + ACC_COL, a, bd, idesc_acc, (gj > 0 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(bar_gempty + b);
-          umma_commit(bar_xempty + st);
-          ++cg;
-          if (++gj == git.n_x) {
-            umma_commit(bar_accfull);
-            gj = 0;
-            ++gic;
-            gi += gridDim.x;
-            if (gi < n_items) git = item_info<DP, kDH>(gi, n_valid, p);
-          }
-        }
-      }
-      // every MMA this thread issued has completed once the drain barrier flips
-      umma_commit(bar_drain);
-      wait_bar_drain(bar_drain, 0, p.timeout_ns);
-    }
-  } else if (warp == 2) {
-    // ============================================================ Y fix-up warp
-    if (kGrad) {
-      uint32_t cnt = 0;
-      bool ok = true;
-      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x) {
-        const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
-        PairCursor pc;
-        if (!kDH) {
-          // the item tile's pairs, ordered by position
-          pc.cur = __ldg(p.item_start + i);
-          pc.end = __ldg(p.item_start + i + 1);
-          pc.nxt = pc.cur < pc.end ? __ldg(p.srt_t + pc.cur) : 0x7fffffff;
-        } else {
-          // the 128 stationary positions' pairs, ordered by item, from the split's first item on
-          const int g0 = it.s_row0;
-          const int gs = __ldg(p.row_ptr + g0);
-          const int ge = __ldg(p.row_ptr + min(g0 + kGroupRows, n_valid));
-          pc.cur = lower_bound_idx(p.grp_v, gs, ge, it.x_tile0 * BN);
-          pc.end = ge;
-          pc.nxt = pc.cur < pc.end ? __ldg(p.grp_v + pc.cur) : 0x7fffffff;
-        }
-        for (int j = 0; j < it.n_x; ++j) {
-          const uint32_t c = cnt + j, b = c % NG;
-          const int x0 = kDH ? (it.x_tile0 + j) * BN : j * BN;   // first streamed row of the tile
-          // The previous use of this buffer (tile c - NG) must be consumed by the MMA first:
-          // that keeps this warp at most one phase ahead on gwritten[b] and fixdone[b], so a
-          // parity wait can never match a phase two uses ahead.
-          if (!wait_bar_warp(bar_gempty + b, ((c / NG) & 1) ^ 1, wc, wait_tag(3, 8, c))) {
-            ok = false;
-            break;
-          }
-          if (pc.nxt < x0 + BN) {
-            // positives fall in this tile: wait for the epilogue's sigmoid tile, then subtract 1
-            if (!wait_bar_warp(bar_gwritten + b, (c / NG) & 1, wc, wait_tag(3, 6, c))) {
-              ok = false;
-              break;
+                for (int ks = 0; ks < DP / 16; ++ks)
+                  tmem_cp_128x256b(tS + 8 * ks, dS + static_cast<uint32_t>((ks >> 2) * (kTileM * 8) + (ks & 3) * 2));
+                umma_commit(bar_sempty);
+              }
+              __syncwarp();
             }
-            uint8_t* G = sG + b * G_BYTES;
-            if (!kDH) fixup_apply<false>(pc, x0 + BN, x0, it.s_row0, G, p.srt_t, p.srt_v, lane);
-            else fixup_apply<true>(pc, x0 + BN, x0, it.s_row0, G, p.grp_v, p.grp_t, lane);
-            fence_proxy_async_smem();
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_fixdone + b);
+          const uint32_t b = cz & 1;
+          if ((zj > 0 || s_ready) && test_bar_warp(bar_xfull + zst, zph) &&
+              test_bar_warp(bar_zfree + b, ((cz >> 1) & 1) ^ 1)) {
+            tc_fence_after();
+            const uint64_t dB = dXk + zoff;
+            const uint32_t tD = tZ + b * BN;
+            if (elect_one()) {
+#pragma unroll
+              for (int ks = 0; ks < DP / 16; ++ks) {
+                const uint64_t bd = dB + static_cast<uint32_t>((ks >> 2) * (BN * 8) + (ks & 3) * 2);
+                if (Cfg::S_IN_TMEM) {
+                  umma_bf16_tmem_a(tD, tS + 8 * ks, bd, idesc_z, ks > 0 ? 1u : 0u);
+                } else {
+                  umma_bf16(tD, dS + static_cast<uint32_t>((ks >> 2) * (kTileM * 8) + (ks & 3) * 2), bd, idesc_z,
+                            ks > 0 ? 1u : 0u);
+                }
+              }
+              umma_commit(bar_zfull + b);
+              if (!kGrad) umma_commit(bar_xempty + zst);
+              if (!Cfg::S_IN_TMEM && zj + 1 == zit.n_x) umma_commit(bar_sempty);  // stationary tile no longer read
+            }
+            __syncwarp();
+            progressed = true;
+            ++cz;
+            zoff += kXStep;
+            if (++zst == static_cast<uint32_t>(NX)) {
+              zst = 0;
+              zoff = 0;
+              zph ^= 1;
+            }
+            if (++zj == zit.n_x) {
+              zj = 0;
+              ++zic;
+              s_ready = false;
+              zi += gridDim.x;
+              if (zi < n_items) zit = item_info<DP, kDH>(zi, n_valid, p);
+            }
+          }
         }
-        cnt += it.n_x;
+        // ---- gradient MMA G(cg): ACC += G[cg & 1] * X, G from tensor memory, X MN-major
+        if (kGrad && gi < n_items && cg < cz) {
+          const uint32_t b = cg & 1;
+          if (test_bar_warp(bar_gready + b, (cg >> 1) & 1) &&
+              (gj > 0 || test_bar_warp(bar_accempty, (gic & 1) ^ 1))) {
+            tc_fence_after();
+            const uint64_t dB = dXmn + goff;
+            const uint32_t tA = tG + b * Cfg::G_COLS;
+            const bool last = gj + 1 == git.n_x;
+            if (elect_one()) {
+#pragma unroll
+              for (int ks = 0; ks < BN / 16; ++ks)
+                umma_bf16_tmem_a(tAcc, tA + 8 * ks, dB + static_cast<uint32_t>(ks * 128), idesc_acc,
+                                 (gj > 0 || ks > 0) ? 1u : 0u);
+              umma_commit(bar_gfree + b);
+              umma_commit(bar_xempty + gst);
+              if (last) umma_commit(bar_accfull);
+            }
+            __syncwarp();
+            progressed = true;
+            ++cg;
+            goff += kXStep;
+            if (++gst == static_cast<uint32_t>(NX)) {
+              gst = 0;
+              goff = 0;
+            }
+            if (last) {
+              gj = 0;
+              ++gic;
+              gi += gridDim.x;
+              if (gi < n_items) git = item_info<DP, kDH>(gi, n_valid, p);
+            } else {
+              ++gj;
+            }
+          }
+        }
+        // ---- bounded: give up if nothing became ready within the limit
+        if (progressed) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = global_timer_ns();
+          if (idle_since == 0) idle_since = now;
+          int give_up = 0;
+          if (lane == 0) {
+            if (*abort_flag) {
+              give_up = 1;
+            } else if (static_cast<long long>(now - idle_since) > p.timeout_ns) {
+              *abort_flag = 1;
+              if (atomicCAS(&hdr->status, 0, kErrTimeout) == 0) {
+                hdr->wait_tag = wait_tag(2, 15, cz);
+                hdr->wait_block = static_cast<int>(blockIdx.x);
+              }
+              give_up = 1;
+            }
+          }
+          if (__shfl_sync(0xffffffffu, give_up, 0)) ok = false;
+        }
       }
+      // every MMA this warp issued has completed once the drain barrier flips
+      if (elect_one()) umma_commit(bar_drain);
+      __syncwarp();
+      if (lane == 0) wait_bar_drain(bar_drain, 0, p.timeout_ns);
+      __syncwarp();
     }
   } else if (warp >= kEpiWarp0) {
     // ============================================================ epilogue
-    // Warp w reads TMEM lanes 32*(w%4).. (its sub-partition's quarter) and one
-    // column slab of each tile: 4 warps per quarter keep the sub-partition's
-    // MUFU/FMA pipes fed while others wait on tensor-memory loads.
-    constexpr int kSlabs = kNumEpiWarps / 4;
-    constexpr int ZC = BN / kSlabs;               // Z columns per warp per tile (32 or 16)
-    constexpr int AC = DP / kSlabs;               // accumulator columns per warp (16 .. 64)
+    // Two groups of 8 warps take alternate tiles (group = tile counter & 1), so
+    // one group's tensor-memory traffic overlaps the other group's element math.
+    // In a group, warp w reads TMEM lanes 32*(w%4).. (its sub-partition's
+    // quarter) and one of two column slabs of the tile, and writes the same
+    // slab of the G tile.
+    constexpr int ZC = BN / 2;                    // Z columns per warp per tile (64 or 32)
+    constexpr int CH = 32;                        // columns per TMEM load
+    constexpr int AC = DP / 2;                    // accumulator columns per warp (32 .. 128)
+    const int ew = warp - kEpiWarp0;
+    const uint32_t grp = static_cast<uint32_t>(ew >> 3);   // tile-parity group
     const int q = warp & 3;                       // TMEM lane quarter
-    const int slab = (warp - kEpiWarp0) >> 2;     // column slab
+    const int slab = (ew >> 2) & 1;               // column slab within the group
     const int row = q * 32 + lane;                // stationary row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t sG_a = smem_u32(sG);
     const float gs = hdr->grad_scale;
+    const int* keys = kDH ? p.pair_v : p.csc_t;
     uint32_t cnt = 0, ic = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ic) {
       const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
       const int n = it.n_x;
       double item_acc = 0.0;
+      // this row's positives (y = 1), as keys along the streamed dimension
+      RowCursor rc{0, 0, 0x7fffffff};
+      if (kGrad) {
+        const int r = it.s_row0 + row;
+        if (!kDH) {
+          if (r < p.V) cursor_init(rc, keys, __ldg(p.csc_off + r), __ldg(p.csc_off + r + 1), 0);
+        } else {
+          if (r < n_valid) cursor_init(rc, keys, __ldg(p.row_ptr + r), __ldg(p.row_ptr + r + 1), it.x_tile0 * BN);
+        }
+      }
       for (int j = 0; j < n; ++j) {
         const uint32_t c = cnt + j, bz = c % NZ, bg = c % NG;
+        if ((c & 1) != grp) continue;             // the other group's tile
         if (!wait_bar_warp(bar_zfull + bz, (c / NZ) & 1, wc, wait_tag(4, 4, c))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t r[ZC];
-        tmem_ld<ZC>(tmem_base + lane_base + bz * BN + slab * ZC, r);
+        const int key0 = kDH ? (it.x_tile0 + j) * BN : j * BN;   // key of the tile's first column
+        float tile_mx = 0.f, tile_l2 = 0.f;
+        // all of this warp's logits of the tile are loaded at once (one wait), so
+        // the logit buffer goes back to the MMA issuer before any math is done
+        constexpr int NCH = ZC / CH;
+        uint32_t r[NCH][CH];
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) tmem_ld<CH>(tmem_base + lane_base + bz * BN + slab * ZC + ch * CH, r[ch]);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_zempty + bz);   // this warp's part of Z[bz] is in registers
-        uint32_t pk[ZC / 2];
-        float prod = 1.f, tile_mx = 0.f;
+        if (lane == 0) mbar_arrive(bar_zfree + bz);
 #pragma unroll
-        for (int e = 0; e < ZC; e += 2) {
-          float gpair[2];
+        for (int ch = 0; ch < NCH; ++ch) {
+          const int col0 = slab * ZC + ch * CH;
+          const uint32_t mask = kGrad ? cursor_take_mask(rc, keys, key0 + col0) : 0u;
+          const bool any_pos = kGrad && __any_sync(0xffffffffu, mask != 0u);
+          uint32_t pk[CH / 2];
+          float prod = 1.f;
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const float z = __uint_as_float(r[e + k]);
-            if (kLoss) {
-              const float u = ex2_approx(-fabsf(z) * kLog2e);   // e^{-|z|}
-              const float pz = 1.f + u;
-              prod *= pz;                                        // log1p batched: one lg2 per slab
-              tile_mx += fmaxf(z, 0.f);
-              if (kGrad) {
-                const float rp = rcp_approx(pz);                 // 1 / (1 + e^{-|z|})
-                gpair[k] = z >= 0.f ? rp : u * rp;               // sigmoid(z)
+          for (int e = 0; e < CH; e += 2) {
+            float g2[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const float z = __uint_as_float(r[ch][e + k]);
+              if (kLoss) {
+                const float u = ex2_approx(-fabsf(z) * kLog2e);   // e^{-|z|}
+                const float pz = 1.f + u;
+                prod *= pz;                                        // log1p batched: one lg2 per chunk
+                tile_mx += fmaxf(z, 0.f);
+                if (kGrad) {
+                  const float rp = rcp_approx(pz);                 // 1 / (1 + e^{-|z|})
+                  g2[k] = z >= 0.f ? rp : u * rp;                  // sigmoid(z)
+                }
+              } else {
+                g2[k] = fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);   // sigmoid(z)
               }
-            } else {
-              gpair[k] = fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);  // sigmoid(z)
+            }
+            if (kGrad) {
+              if (any_pos) {                                       // y = 1 at the masked columns
+                g2[0] -= static_cast<float>((mask >> e) & 1u);
+                g2[1] -= static_cast<float>((mask >> (e + 1)) & 1u);
+              }
+              pk[e >> 1] = pack_bf16x2(g2[0], g2[1]);
             }
           }
-          if (kGrad) pk[e >> 1] = pack_bf16x2(gpair[0], gpair[1]);
-        }
-        if (kGrad) {
-          if (!wait_bar_warp(bar_gempty + bg, ((c / NG) & 1) ^ 1, wc, wait_tag(4, 8, c))) {
-            ok = false;
-            break;
+          if (kLoss) tile_l2 += lg2_approx(prod);
+          if (kGrad) {
+            if (ch == 0 && !wait_bar_warp(bar_gfree + bg, ((c / NG) & 1) ^ 1, wc, wait_tag(4, 8, c))) {
+              ok = false;
+              break;
+            }
+            tmem_st16(tmem_base + lane_base + Cfg::G_COL + bg * Cfg::G_COLS + col0 / 2, pk);
           }
-          const int col0 = slab * ZC;
-          const uint32_t base = sG_a + bg * G_BYTES + (col0 >> 6) * (kTileM * 128) + row * 128;
-          const uint32_t j0 = (col0 & 63) >> 3;
-#pragma unroll
-          for (int k = 0; k < ZC / 8; ++k)
-            st_shared_v4(base + (((j0 + k) ^ (row & 7)) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
-                         pk[4 * k + 3]);
-          fence_proxy_async_smem();
+        }
+        if (!ok) break;
+        if (kGrad) {
+          tmem_st_wait();
+          tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_gwritten + bg);
+          if (lane == 0) mbar_arrive(bar_gready + bg);   // this warp's part of G is in place
         }
         if (kLoss) {
-          float tile_l2 = lg2_approx(prod);
           if (j == n - 1) {
             // zero rows of H_c past n_valid give z = 0 exactly: each adds log2(2) = 1 to tile_l2
             const int t0 = j * BN;
@@ -544,9 +590,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         double val = (it.s_row0 + row < p.V) ? item_acc : 0.0;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
-        if (lane == 0) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + (warp - kEpiWarp0)] = val;
+        if (lane == 0) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + ew] = val;
       }
-      if (kGrad) {
+      if (kGrad && ((cnt + n - 1) & 1) == grp) {
+        // the group that took the item's last tile reads the accumulator out
         if (!wait_bar_warp(bar_accfull, ic & 1, wc, wait_tag(4, 9, ic))) break;
         tc_fence_after();
 #pragma unroll 1
