@@ -33,7 +33,8 @@
  *    zero dH row and contributes nothing to dE; its ids are ignored entirely.
  *  - Every output and the workspace are owned by the caller.  The library
  *    never allocates or frees device memory and keeps no state between calls
- *    apart from cached device attributes.
+ *    apart from cached device attributes and the static scratch array of
+ *    cutbce_forward_fixed_scratch.
  *  - All compute calls are asynchronous on `stream`.  Errors a host can see
  *    (NULL pointers, sizes <= 0, unsupported D or dtype, a workspace that is
  *    too small, a device that is not sm_100) are returned before anything is
@@ -106,6 +107,40 @@ cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes);
  * 256-byte aligned. */
 cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_bytes,
                              double* loss, cutbce_stream_t stream);
+
+/* Size of the static device scratch array behind cutbce_forward_fixed_scratch
+ * (16 MiB, part of the library's device image on every device it runs on). */
+#define CUTBCE_FIXED_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* Loss only, like cutbce_forward, but with no workspace argument: the call
+ * uses a static scratch array of CUTBCE_FIXED_SCRATCH_BYTES bytes that lives in
+ * the library's own device image, so neither the caller nor the library
+ * allocates anything.  The paper has no counterpart to this entry; it exists
+ * for callers that cannot hand over device memory at the point of the call --
+ * for instance code that sized its device memory pool once at start-up and may
+ * not grow it, or a host runtime with no device allocator of its own, where a
+ * cudaMalloc would also stall the device until pending work drains.
+ *
+ * Limit: problems with cutbce_workspace_size() > CUTBCE_FIXED_SCRATCH_BYTES
+ * are rejected with CUTBCE_ERR_WORKSPACE before anything is launched (the
+ * workspace grows with T*K, S*T*D and V; small and medium problems fit).
+ * Setup: the first call on each device, with that device current, looks up
+ * the device address of the array (cudaGetSymbolAddress) and caches it; that
+ * lookup may load the library's device code on the device, so make the first
+ * call on each device before any stream capture begins.  A failed lookup
+ * returns CUTBCE_ERR_CUDA.
+ * Zeroing: nothing has to start at zero; each call clears the part of the
+ * array it needs cleared (the status header) on `stream` itself.
+ * Concurrency: all calls on one device share the one array, so two calls whose
+ * device work can overlap (different streams, or host threads without
+ * ordering between them) race on it and give wrong results; order them, for
+ * example by issuing them on one stream.
+ * Errors: host-visible errors are returned as for cutbce_forward.  The
+ * device status word sits in the static array, which the library does not
+ * expose, so a data error (an id out of range) is not reported by this entry
+ * (the loss is then unspecified); use cutbce_forward where it must be. */
+cutbce_status cutbce_forward_fixed_scratch(const cutbce_problem* prob, double* loss,
+                                           cutbce_stream_t stream);
 
 /* Gradients only (section III-B, Eq. (4)), recomputing the logits.
  * grad_loss: device float scalar g, or NULL for g = 1.

@@ -17,7 +17,8 @@ import torch
 
 __all__ = [
     "CutBCEError", "cutbce_problem", "load_library", "library_path", "declared_functions",
-    "cutbce_workspace_size", "cutbce_forward", "cutbce_backward", "cutbce_forward_backward",
+    "cutbce_workspace_size", "cutbce_forward", "cutbce_forward_fixed_scratch", "FIXED_SCRATCH_BYTES",
+    "cutbce_backward", "cutbce_forward_backward",
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
     "cutbce_selftest_wait_timeout", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
@@ -57,6 +58,7 @@ _vp, _sz, _i32, _i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.
 _SIGS = {
     "cutbce_workspace_size": (_i32, [_P, ctypes.POINTER(_sz)]),
     "cutbce_forward": (_i32, [_P, _vp, _sz, _vp, _vp]),
+    "cutbce_forward_fixed_scratch": (_i32, [_P, _vp, _vp]),
     "cutbce_backward": (_i32, [_P, _vp, _vp, _vp, _vp, _sz, _vp]),
     "cutbce_forward_backward": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "cutbce_host_buffer_size": (_i32, [_P, ctypes.POINTER(_sz)]),
@@ -143,6 +145,16 @@ def cutbce_workspace_size(prob: cutbce_problem) -> int:
 def cutbce_forward(prob, ws: torch.Tensor, loss: torch.Tensor, stream=None) -> None:
     _check(load_library().cutbce_forward(ctypes.byref(prob), ws.data_ptr(), ws.numel(), loss.data_ptr(),
                                          _stream(stream)), "cutbce_forward")
+
+
+# Size of the library's static scratch array (CUTBCE_FIXED_SCRATCH_BYTES in include/cutbce.h).
+FIXED_SCRATCH_BYTES = 16 << 20
+
+
+def cutbce_forward_fixed_scratch(prob, loss: torch.Tensor, stream=None) -> None:
+    """Loss only, with the library's static scratch array instead of a workspace (nothing is allocated)."""
+    _check(load_library().cutbce_forward_fixed_scratch(ctypes.byref(prob), loss.data_ptr(), _stream(stream)),
+           "cutbce_forward_fixed_scratch")
 
 
 def cutbce_backward(prob, grad_loss: Optional[torch.Tensor], dH: Optional[torch.Tensor],

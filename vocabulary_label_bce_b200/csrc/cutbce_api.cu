@@ -454,6 +454,33 @@ void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
   hl.total = o;
 }
 
+// ---------------------------------------------------------------- fixed scratch
+// Scratch of cutbce_forward_fixed_scratch: a static device array of the
+// library's own module, so that entry needs no caller workspace and allocates
+// nothing.  Every call on a device uses the same array: calls on one device
+// must not overlap in time (see the header).
+constexpr size_t kFixedScratchBytes = CUTBCE_FIXED_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_fixed_mutex;
+void* g_fixed_ptr[kMaxDevices] = {};
+
+// Device address of g_fixed_scratch on the current device, looked up once per
+// device (with that device current) and cached.
+cutbce_status fixed_scratch_ptr(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CUTBCE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_fixed_mutex);
+  if (g_fixed_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_fixed_scratch) != cudaSuccess || ptr == nullptr) return CUTBCE_ERR_CUDA;
+    g_fixed_ptr[dev] = ptr;
+  }
+  *out = g_fixed_ptr[dev];
+  return CUTBCE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -472,6 +499,19 @@ cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_byt
                              cutbce_stream_t stream) {
   if (loss == nullptr) return CUTBCE_ERR_INVALID_ARG;
   return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false}, ws, ws_bytes,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+cutbce_status cutbce_forward_fixed_scratch(const cutbce_problem* prob, double* loss, cutbce_stream_t stream) {
+  if (loss == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  cutbce_status s = check_problem(prob, true);
+  if (s != CUTBCE_OK) return s;
+  Plan pl;
+  make_plan(prob, pl);
+  if (pl.total > kFixedScratchBytes) return CUTBCE_ERR_WORKSPACE;   // the problem needs more than the fixed array
+  void* ws = nullptr;
+  if ((s = fixed_scratch_ptr(&ws)) != CUTBCE_OK) return s;
+  return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false}, ws, kFixedScratchBytes,
              reinterpret_cast<cudaStream_t>(stream));
 }
 
