@@ -79,8 +79,9 @@ def test_compute_calls_reject_before_launch():
 
 def test_launch_accounting():
     p = _prob()
-    # rows, scan, gather, 3 radix passes x 3 + item offsets, item pass, dH pass, finish
-    assert B.cutbce_kernel_launches(p, 2) == 16
+    # rows, scan, gather, sort keys, 2 radix passes x 3 (6844 item tiles: 13-bit keys),
+    # item-tile offsets, item pass, dH pass, finish
+    assert B.cutbce_kernel_launches(p, 2) == 14
     assert B.cutbce_kernel_launches(p, 0) == 5          # rows, scan, gather, item pass, finish
     assert B.cutbce_kernel_launches(p, 3) == -1
 

@@ -14,7 +14,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcutbce.so")
 SOURCES = ["cutbce_api.cu"]
-DEPS = ["cutbce_api.cu", "common.cuh", "prep_finish.cuh", "pair_sort.cuh", "tile_engine.cuh", "ptx_sm100.cuh", "probes.cuh"]
+DEPS = ["cutbce_api.cu", "common.cuh", "prep_finish.cuh", "pair_sort.cuh", "tile_engine.cuh", "ptx_sm100.cuh", "probes.cuh",
+        "elementwise.cuh"]
 
 
 def nvcc_path() -> str:

@@ -22,8 +22,8 @@ constexpr int kMaxDim = 256;          // feature width
 constexpr int kTileM = 128;           // stationary rows per tile = TMEM lanes
 constexpr int kMaxCtas = 256;         // upper bound of a persistent grid
 constexpr int kMaxSplits = 64;        // dH partial splits over the vocabulary
-constexpr int kTileThreads = 640;     // 20 warps: TMA, MMA, fix-up, idle, 16 epilogue
-constexpr int kEpiWarp0 = 4;
+constexpr int kTileThreads = 576;     // 18 warps: TMA producer, MMA issuer, 16 epilogue
+constexpr int kEpiWarp0 = 2;
 constexpr int kNumEpiWarps = 16;      // 2 groups x (4 TMEM lane quarters x 2 column slabs)
 constexpr int kEpiGroupWarps = 8;     // warps that take one tile
 
@@ -48,19 +48,21 @@ struct TileCfg {
   // (issued up to NZ-1 tiles early) until its gradient MMA completes, and the ring
   // must still cover the L2 -> shared memory latency of the next loads
   static constexpr int NX = DP == 64 ? 12 : DP == 128 ? 6 : DP == 192 ? 7 : 5;
-  static constexpr int NZ = 2;                               // fp32 logit tiles in tensor memory
-  static constexpr int NG = 2;                               // bf16 sigmoid tiles in tensor memory
+  // fp32 logit tiles in tensor memory.  The bf16 G tile of a logit tile is
+  // written over that tile's own columns (each warp over the slab it loaded),
+  // so a buffer holds Z, then G, and is free once the gradient MMA reading G
+  // has completed.
+  static constexpr int NZ = 3;
   static constexpr uint32_t S_BYTES = kTileM * DP * 2;       // stationary tile
   static constexpr uint32_t X_BYTES = BN * DP * 2;           // streamed tile
-  static constexpr int G_COL = NZ * BN;                      // TMEM column of the first G buffer
-  static constexpr int G_COLS = BN / 2;                      // a G tile: BN bf16 per lane, two per column
-  static constexpr int ACC_COL = G_COL + NG * G_COLS;        // TMEM column of the gradient accumulator
+  static constexpr int ZC = BN / 2;                          // logit columns per epilogue warp (one slab)
+  static constexpr int ACC_COL = NZ * BN;                    // TMEM column of the gradient accumulator
   static constexpr int TMEM_COLS = 512;
   // The stationary tile is copied into tensor memory (bf16 pairs, DP/2 columns)
   // when it fits, so the logit MMA reads only its B operand from shared memory.
   static constexpr int S_COL = ACC_COL + DP;
   static constexpr bool S_IN_TMEM = S_COL + DP / 2 <= TMEM_COLS;
-  static constexpr int NUM_BARS = 2 + 2 * NX + 2 * NZ + 2 * NG + 3;  // see the kernel for the list
+  static constexpr int NUM_BARS = 2 + 2 * NX + 3 * NZ + 3;  // see the kernel for the list
   static constexpr uint32_t SMEM_BYTES = 1024 + S_BYTES + NX * X_BYTES + NUM_BARS * 8 + 16 + 64;
   static_assert(ACC_COL + DP <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");

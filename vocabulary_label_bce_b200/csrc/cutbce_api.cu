@@ -49,6 +49,8 @@ cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
   if (p->dtype == CUTBCE_BF16 && (p->D % 8) != 0) return CUTBCE_ERR_UNSUPPORTED;
   if (p->V >= (int64_t(1) << 31) || p->T >= (int64_t(1) << 30) || p->T * p->K >= (int64_t(1) << 31))
     return CUTBCE_ERR_UNSUPPORTED;
+  // the item-owned pass packs a compacted position into 24 bits
+  if (p->dtype == CUTBCE_BF16 && round_up(p->T, kTileM) >= (int64_t(1) << kPairPosBits)) return CUTBCE_ERR_UNSUPPORTED;
   if (need_data) {
     if (p->H == nullptr || p->E == nullptr || p->targets == nullptr) return CUTBCE_ERR_INVALID_ARG;
     if (p->dtype == CUTBCE_BF16 &&
@@ -74,8 +76,8 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.n_gather_blocks = ceil_div(pl.Tpad, 8);
   {
     int bits = 0;
-    while ((int64_t(1) << bits) < p->V) ++bits;
-    pl.radix_passes = (bits + 7) / 8;     // 8-bit digits of the item id
+    while ((int64_t(1) << bits) < pl.n_vitems) ++bits;
+    pl.radix_passes = std::max(1, (bits + 7) / 8);     // 8-bit digits of the item-tile index
     pl.radix_blocks = static_cast<int>(std::max<int64_t>(1, ceil_div(p->T * p->K, kRadixTile)));
   }
   if (bf16) {
@@ -107,7 +109,7 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.o_pair_v = take(4 * TK);
   for (int k = 0; k < 4; ++k) pl.o_srt[k] = take(4 * TK);
   pl.o_ghist = take(4 * 256 * static_cast<size_t>(pl.radix_blocks));
-  pl.o_cscoff = take(4 * static_cast<size_t>(p->V + 1));
+  pl.o_cscoff = take(4 * static_cast<size_t>(pl.n_vitems + 1));
   pl.o_hc = take(pl.elem * static_cast<size_t>(pl.Tpad) * pl.DP);
   pl.o_lpart = take(8 * kNumEpiWarps * pl.n_vitems);
   pl.o_cpart = take(8 * pl.n_gather_blocks);
@@ -269,7 +271,7 @@ struct Want {
 int count_launches(const Plan& pl, Want w) {
   const bool bf16 = pl.dtype == CUTBCE_BF16;
   int n = 3;                                            // rows, scan, gather
-  if (bf16 && w.dE) n += 3 * pl.radix_passes + 1;       // radix passes and item offsets
+  if (bf16 && w.dE) n += 1 + 3 * pl.radix_passes + 1;   // sort keys, radix passes, item-tile offsets
   if (w.loss || w.dE) n += 1;                           // item-owned pass
   if (w.dH) n += 1;                                     // position-owned pass
   if (w.loss || w.dH) n += 1;                           // finish
@@ -339,26 +341,35 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
 
   const bool item_pass = w.loss || w.dE;
   if (bf16) {
-    const int* csc_v = pair_v;
-    const int* csc_t = pair_t;
+    const int* srt_key = pair_v;
+    const int* srt_val = pair_t;
     if (w.dE) {
-      // pairs ordered by (item, position): stable LSD radix sort on the item id, then offsets
+      // pairs grouped by item tile, ascending position inside a group: stable LSD
+      // radix sort of (item tile, packed row/position) starting from (position, item) order
       LaunchScope ls(CUTBCE_KERNEL_PAIR_SORT, st);
+      int* k0 = at<int>(ws, pl.o_srt[2]);
+      int* v0 = at<int>(ws, pl.o_srt[3]);
+      const int64_t TK = static_cast<int64_t>(T) * K;
+      k_pair_keys<<<static_cast<unsigned>(std::max<int64_t>(1, ceil_div(TK, 256))), 256, 0, st>>>(pair_v, pair_t,
+                                                                                                   hdr, k0, v0);
+      srt_key = k0;
+      srt_val = v0;
       for (int pass = 0; pass < pl.radix_passes; ++pass) {
-        int* out_v = at<int>(ws, pl.o_srt[2 * (pass & 1)]);
-        int* out_t = at<int>(ws, pl.o_srt[2 * (pass & 1) + 1]);
-        k_radix_hist<<<pl.radix_blocks, kRadixThreads, 0, st>>>(csc_v, hdr, 8 * pass, pl.radix_blocks, ghist);
+        int* out_k = at<int>(ws, pl.o_srt[2 * (pass & 1)]);
+        int* out_v = at<int>(ws, pl.o_srt[2 * (pass & 1) + 1]);
+        k_radix_hist<<<pl.radix_blocks, kRadixThreads, 0, st>>>(srt_key, hdr, 8 * pass, pl.radix_blocks, ghist);
         k_exclusive_scan<<<1, 1024, 0, st>>>(ghist, 256 * pl.radix_blocks);
-        k_radix_scatter<<<pl.radix_blocks, kRadixThreads, 0, st>>>(csc_v, csc_t, out_v, out_t, hdr, 8 * pass,
+        k_radix_scatter<<<pl.radix_blocks, kRadixThreads, 0, st>>>(srt_key, srt_val, out_k, out_v, hdr, 8 * pass,
                                                                    pl.radix_blocks, ghist);
-        csc_v = out_v;
-        csc_t = out_t;
+        srt_key = out_k;
+        srt_val = out_v;
       }
       CUTBCE_CK(cudaGetLastError());
     }
     if (w.dE) {
       LaunchScope ls(CUTBCE_KERNEL_CSC_OFFSETS, st);
-      k_csc_offsets<<<static_cast<unsigned>(ceil_div(V + 1, 256)), 256, 0, st>>>(csc_v, hdr, V, cscoff);
+      const int nkeys = static_cast<int>(pl.n_vitems);
+      k_key_offsets<<<static_cast<unsigned>(ceil_div(nkeys + 1, 256)), 256, 0, st>>>(srt_key, hdr, nkeys, cscoff);
       CUTBCE_CK(cudaGetLastError());
     }
     TileParams tp{};
@@ -368,8 +379,8 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     tp.hdr = hdr;
     tp.row_ptr = rowptr;
     tp.pair_v = pair_v;
-    tp.csc_off = cscoff;
-    tp.csc_t = csc_t;
+    tp.tile_pair_off = cscoff;
+    tp.tile_pairs = srt_val;
     tp.dE = dE;
     tp.loss_part = lpart;
     tp.dh_part = dhpart;

@@ -1,0 +1,82 @@
+// Per-logit BCE math of the tile engine, two logits at a time.
+//
+// For a logit z (section III-A, Eq. (2) of "Cut Binary Cross Entropy"):
+//   u = e^{-|z|} in (0, 1],   w = 1 + u in (1, 2]
+//   l(z, 0) = max(z, 0) + log(1 + e^{-|z|}) = max(z, 0) + ln 2 * log2(w)
+//   sigmoid(z) = 1 / w  (z >= 0),   u / w  (z < 0)      (Eq. (4): G = sigmoid(Z) - Y)
+//
+// Pipe budget on B200 (measured with the library's pipe probes): the SFU
+// (ex2, rcp, lg2, tanh) retires 16 results per clock per SM, the FMA pipe 128,
+// so one SFU operation costs as much as eight FMAs.  Each logit therefore gets
+// exactly one SFU operation (the exponential); the reciprocal runs on the FMA
+// pipe, and the logarithm is taken once per 32 logits of a row as the log2 of
+// the product of their w (each factor is in (1, 2], so 32 of them stay finite).
+//
+// Reciprocal: exponent-flip seed r0 = bits^-1(C - bits(w)) (the integer
+// subtraction negates the exponent and roughly reflects the mantissa; with
+// C = 0x7EF31000 the relative error |1 - w r0| is at most 0.0506 for every
+// normal w), then the cubically convergent step r1 = r0 (1 + e + e^2) with
+// e = 1 - w r0, which leaves |1 - w r1| = |e|^3 <= 1.3e-4, and optionally one
+// Newton step r2 = r1 (1 + e1) (error <= 1.7e-8).  The seed is formed from -w
+// (bits(-w) = bits(w) + 2^31), which the FMA pipe produces in the same
+// instruction as 1 + u, so no separate negation is needed.
+//
+// Packed fp32x2 instructions (two lanes of work per instruction) halve the
+// issue slots of the FMA-pipe part; the SFU and the selects stay scalar.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+#include "ptx_sm100.cuh"
+
+namespace cutbce {
+
+constexpr float kLog2eF = 1.4426950408889634f;
+constexpr float kLn2F = 0.6931471805599453f;
+constexpr uint32_t kRcpSeedNeg = 0x7EF31000u + 0x80000000u;   // C + 2^31: seed from bits(-w)
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// 1 / w from nw = -w (w normal and positive): seed plus cubic step, |rel err| <= 1.3e-4.
+__device__ __forceinline__ float2 rcp2_cubic(float2 nw) {
+  float2 r = f2(__uint_as_float(kRcpSeedNeg - __float_as_uint(nw.x)),
+                __uint_as_float(kRcpSeedNeg - __float_as_uint(nw.y)));
+  const float2 e = __ffma2_rn(nw, r, f2(1.f, 1.f));    // 1 - w r0
+  const float2 t = __ffma2_rn(e, e, e);                // e + e^2
+  return __ffma2_rn(r, t, r);                          // r0 (1 + e + e^2)
+}
+
+// Item-owned pass, loss and gradient: returns sigmoid(z) for both logits and
+// folds their loss terms into the running products `prod` (of w, sign-free
+// over an even count of factors per component) and the running sum `relu`
+// of max(z, 0).
+__device__ __forceinline__ float2 bce_pair_loss_grad(float2 z, float2& prod, float2& relu) {
+  const float2 u = f2(ex2_approx(-fabsf(z.x) * kLog2eF), ex2_approx(-fabsf(z.y) * kLog2eF));
+  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + u)
+  prod = __fmul2_rn(prod, nw);
+  relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
+  const float2 r = rcp2_cubic(nw);
+  const float2 ur = __fmul2_rn(u, r);
+  return f2(z.x >= 0.f ? r.x : ur.x, z.y >= 0.f ? r.y : ur.y);
+}
+
+// Item-owned pass, loss only.
+__device__ __forceinline__ void bce_pair_loss(float2 z, float2& prod, float2& relu) {
+  const float2 u = f2(ex2_approx(-fabsf(z.x) * kLog2eF), ex2_approx(-fabsf(z.y) * kLog2eF));
+  prod = __fmul2_rn(prod, __fadd2_rn(u, f2(1.f, 1.f)));
+  relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
+}
+
+// Gradient only (the position-owned pass, and the item pass without the
+// loss): sigmoid(z) = 1 / (1 + 2^{-z log2 e}) over the whole range, the
+// exponent clamped at 100 (below z = -69.3 the result is 2^-100 instead of
+// a smaller positive number).  Seed, cubic step and one Newton step:
+// |rel err| <= 1.7e-8 plus rounding.
+__device__ __forceinline__ float2 sigmoid_pair(float2 z) {
+  const float2 u = f2(ex2_approx(fminf(-z.x * kLog2eF, 100.f)), ex2_approx(fminf(-z.y * kLog2eF, 100.f)));
+  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + u)
+  const float2 r = rcp2_cubic(nw);
+  const float2 e = __ffma2_rn(nw, r, f2(1.f, 1.f));
+  return __ffma2_rn(r, e, r);                                        // Newton step
+}
+
+}  // namespace cutbce

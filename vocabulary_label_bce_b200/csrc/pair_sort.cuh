@@ -1,11 +1,13 @@
-// Item-major order of the (position, item) pairs (a CSC of the sparse target
-// matrix Y) for the item-owned tensor-core pass: every item's positives as an
-// ascending list of compacted positions, so that the epilogue thread owning an
-// item row walks them with a forward-only cursor as position tiles stream by.
+// Order of the (position, item) pairs for the item-owned tensor-core pass:
+// grouped by item tile (128 consecutive items, one stationary tile of that
+// pass), and within a group in ascending compacted position, so that the
+// epilogue warps of a CTA walk their item tile's positives with one forward
+// cursor as the position tiles stream by.
 //
 // The pairs are produced in (position, item) order; a stable LSD radix sort on
-// the item id therefore yields (item, position) order.  Every result is unique
-// (pairs are distinct), so the order is deterministic.
+// the item-tile index keeps that order inside each group.  The value carried
+// along packs the item's row within its tile and the compacted position:
+// (v mod 128) << 24 | t.  Every pair is unique, so the order is deterministic.
 #pragma once
 #include <cstdint>
 #include "common.cuh"
@@ -13,6 +15,7 @@
 namespace cutbce {
 
 constexpr int kRadixThreads = 256;
+constexpr int kPairPosBits = 24;                 // compacted positions below 2^24 fit the packed value
 constexpr int kRadixTile = 4096;                 // pairs per block
 constexpr int kRadixRounds = kRadixTile / kRadixThreads;
 
@@ -137,12 +140,22 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(const int* __re
   }
 }
 
-// csc_off[v] = first index of the item-sorted pairs whose item is >= v, for v in
-// [0, V]; item v owns [csc_off[v], csc_off[v+1]).
-__global__ void k_csc_offsets(const int* __restrict__ sorted_v, const WsHeader* hdr, int V,
+// Sort input: key = item tile v / 128, value = (v mod 128) << 24 | t.
+__global__ void k_pair_keys(const int* __restrict__ pair_v, const int* __restrict__ pair_t, const WsHeader* hdr,
+                            int* __restrict__ keys, int* __restrict__ vals) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= hdr->n_pairs) return;
+  const int v = pair_v[i];
+  keys[i] = v >> 7;
+  vals[i] = ((v & 127) << kPairPosBits) | pair_t[i];
+}
+
+// off[k] = first index of the sorted pairs whose key is >= k, for k in [0, nkeys];
+// key k owns [off[k], off[k+1]).
+__global__ void k_key_offsets(const int* __restrict__ sorted_v, const WsHeader* hdr, int nkeys,
                               int* __restrict__ csc_off) {
   const int v = blockIdx.x * blockDim.x + threadIdx.x;
-  if (v > V) return;
+  if (v > nkeys) return;
   int lo = 0, hi = hdr->n_pairs;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;

@@ -48,8 +48,11 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 #include "common.cuh"
 #include "ptx_sm100.cuh"
+#include "elementwise.cuh"
+#include "pair_sort.cuh"
 
 namespace cutbce {
 
@@ -60,8 +63,8 @@ struct TileParams {
   WsHeader* hdr;               // n_valid, grad scale, status
   const int* row_ptr;          // [n_valid + 1] pair offsets of compacted rows (CSR by position)
   const int* pair_v;           // CSR by position: items of each row, ascending
-  const int* csc_off;          // [V + 1] offsets into csc_t (CSC by item)
-  const int* csc_t;            // CSC by item: positions of each item, ascending
+  const int* tile_pair_off;    // [ceil(V/128) + 1] offsets into tile_pairs, one range per item tile
+  const int* tile_pairs;       // pairs grouped by item tile, ascending position: (v mod 128) << 24 | t
   float* dE;                   // item-owned pass output [V, D] (may be null when no gradient)
   double* loss_part;           // item-owned pass: one double per (item tile, epilogue warp)
   float* dh_part;              // position-owned pass output [S, Tpad, DP]
@@ -171,11 +174,12 @@ __device__ __forceinline__ void cursor_init(RowCursor& rc, const int* __restrict
   rc.nxt = c < end ? __ldg(keys + c) : 0x7fffffff;
 }
 
-// Bit e set for each positive whose key is lo + e, e in [0, 32); advances the cursor.
+// Bit e set for each positive whose key is lo + e, e in [0, 32); consumes every
+// key below lo + 32 (keys below lo belong to columns this thread does not own).
 __device__ __forceinline__ uint32_t cursor_take_mask(RowCursor& rc, const int* __restrict__ keys, int lo) {
   uint32_t mask = 0;
   while (rc.nxt < lo + 32) {
-    mask |= 1u << (rc.nxt - lo);
+    if (rc.nxt >= lo) mask |= 1u << (rc.nxt - lo);
     ++rc.cur;
     rc.nxt = rc.cur < rc.end ? __ldg(keys + rc.cur) : 0x7fffffff;
   }
@@ -190,13 +194,11 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   constexpr int NKB = Cfg::NKB;
   constexpr int NX = Cfg::NX;
   constexpr int NZ = Cfg::NZ;
-  constexpr int NG = Cfg::NG;
   constexpr uint32_t S_BYTES = Cfg::S_BYTES, X_BYTES = Cfg::X_BYTES;
   constexpr int ACC_COL = Cfg::ACC_COL;
   static_assert(!kDH || (kGrad && !kLoss), "the position-owned pass computes dH only");
   static_assert(kLoss || kGrad, "nothing to do");
-  constexpr float kLog2e = 1.4426950408889634f;
-  constexpr float kLn2 = 0.6931471805599453f;
+  constexpr float kLn2 = kLn2F;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -207,11 +209,11 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   uint64_t* bar_sempty = bars + 1;                // stationary tile free (MMA commit)
   uint64_t* bar_xfull = bars + 2;                 // [NX] streamed tile landed
   uint64_t* bar_xempty = bar_xfull + NX;          // [NX] streamed tile free
-  uint64_t* bar_zfull = bar_xempty + NX;          // [NZ] logit tile ready in TMEM
-  uint64_t* bar_zfree = bar_zfull + NZ;           // [NZ] logit tile loaded by the epilogue group
-  uint64_t* bar_gready = bar_zfree + NZ;          // [NG] G tile written by the epilogue group
-  uint64_t* bar_gfree = bar_gready + NG;          // [NG] G tile consumed by the gradient MMA
-  uint64_t* bar_accfull = bar_gfree + NG;         // gradient accumulator complete
+  uint64_t* bar_zfull = bar_xempty + NX;          // [NZ] logit tile ready in TMEM (MMA commit)
+  uint64_t* bar_zfree = bar_zfull + NZ;           // [NZ] buffer free: gradient MMA done (commit), or,
+                                                  //      without a gradient, logits loaded (epilogue group)
+  uint64_t* bar_gready = bar_zfree + NZ;          // [NZ] G tile written over the logits (epilogue group)
+  uint64_t* bar_accfull = bar_gready + NZ;        // gradient accumulator complete
   uint64_t* bar_accempty = bar_accfull + 1;       // gradient accumulator read out
   uint64_t* bar_drain = bar_accempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
@@ -256,11 +258,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
     for (int b = 0; b < NZ; ++b) {
       mbar_init(bar_zfull + b, 1);
-      mbar_init(bar_zfree + b, kEpiGroupWarps);
-    }
-    for (int b = 0; b < NG; ++b) {
+      mbar_init(bar_zfree + b, kGrad ? 1 : kEpiGroupWarps);
       mbar_init(bar_gready + b, kEpiGroupWarps);
-      mbar_init(bar_gfree + b, 1);
     }
     mbar_init(bar_accfull, 1);
     mbar_init(bar_accempty, kEpiGroupWarps);
@@ -320,11 +319,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     // ============================================================ MMA issuer
     // The whole warp runs this loop; lane 0 tests the barriers and shares the
     // answer, one elected lane issues each tcgen05 instruction.  It is an event
-    // loop over two in-order streams: logit tiles Z(c) (ready once their
-    // streamed tile has landed and their logit buffer has been loaded by the
-    // epilogue) and gradient MMAs G(c) (ready once the epilogue group has
-    // written the G tile).  Whichever is ready is issued, so a logit tile for
-    // one epilogue group never waits behind the other group's gradient tile.
+    // loop over two in-order streams: logit tiles Z(c) into buffer c mod NZ
+    // (ready once the streamed tile has landed and the buffer is free) and
+    // gradient MMAs G(c) (ready once the epilogue group has written the G tile
+    // over the logits of buffer c mod NZ).  Whichever is ready is issued.
     //
     // Shared-memory descriptors are built once and advanced by adding the byte
     // offset / 16 to their 14-bit start-address field (it cannot carry out:
@@ -333,16 +331,17 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       constexpr uint32_t idesc_z = idesc_bf16_f32(kTileM, BN, false, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kTileM, DP, false, true);
       constexpr uint32_t kXStep = X_BYTES >> 4;                       // one ring stage, in descriptor units
-      static_assert(NZ == 2 && NG == 2, "ring positions below use & 1");
+      constexpr int kKsPerSlab = Cfg::ZC / 16;                         // gradient K steps per epilogue slab
       const uint64_t dS = smem_desc_sw128(smem_u32(sS), 16, 1024);     // stationary tile, K-major
       const uint64_t dXk = smem_desc_sw128(smem_u32(sX), 16, 1024);    // streamed tile as K-major B
       const uint64_t dXmn = smem_desc_sw128(smem_u32(sX), BN * 128, 1024);  // streamed tile as MN-major B
-      const uint32_t tZ = tmem_base, tG = tmem_base + Cfg::G_COL, tAcc = tmem_base + ACC_COL,
-                     tS = tmem_base + Cfg::S_COL;
+      const uint32_t tZ = tmem_base, tAcc = tmem_base + ACC_COL, tS = tmem_base + Cfg::S_COL;
       int zi = blockIdx.x, zj = 0, gi = blockIdx.x, gj = 0;
       uint32_t zic = 0, cz = 0, gic = 0, cg = 0;
       uint32_t zst = 0, zph = 0, zoff = 0;        // ring stage of the next logit tile, its phase, its offset
       uint32_t gst = 0, goff = 0;                 // ring stage of the next gradient MMA, its offset
+      uint32_t zb = 0, zbph = 0;                  // logit buffer of the next Z, and its use parity
+      uint32_t gb = 0, gbph = 0;                  // logit buffer of the next G, and its use parity
       bool s_ready = false;                       // the current item's stationary tile is in place
       ItemInfo zit{}, git{};
       if (zi < n_items) zit = git = item_info<DP, kDH>(zi, n_valid, p);
@@ -350,9 +349,21 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       bool ok = true;
       while (ok && (zi < n_items || (kGrad && gi < n_items))) {
         bool progressed = false;
-        // ---- logit tile Z(cz) into buffer cz & 1
-        if (zi < n_items) {
-          if (zj == 0 && !s_ready && test_bar_warp(bar_sfull, zic & 1)) {
+        // Poll every barrier the next step may need at once: lane k tests one
+        // barrier, a single ballot gathers the answers (one shared-memory round
+        // trip per iteration instead of a chain of them).
+        const bool want_z = zi < n_items;
+        const bool want_g = kGrad && gi < n_items && cg < cz;
+        bool mine = false;
+        if (lane == 0 && want_z && zj == 0 && !s_ready) mine = mbar_test_wait(bar_sfull, zic & 1);
+        if (lane == 1 && want_z) mine = mbar_test_wait(bar_xfull + zst, zph);
+        if (lane == 2 && want_z) mine = mbar_test_wait(bar_zfree + zb, zbph ^ 1);
+        if (lane == 3 && want_g) mine = mbar_test_wait(bar_gready + gb, gbph);
+        if (lane == 4 && want_g && gj == 0) mine = mbar_test_wait(bar_accempty, (gic & 1) ^ 1);
+        const uint32_t ready = __ballot_sync(0xffffffffu, mine);
+        // ---- logit tile Z(cz) into buffer zb
+        if (want_z) {
+          if (zj == 0 && !s_ready && (ready & 1u)) {
             tc_fence_after();
             s_ready = true;
             if (Cfg::S_IN_TMEM) {
@@ -366,12 +377,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
               __syncwarp();
             }
           }
-          const uint32_t b = cz & 1;
-          if ((zj > 0 || s_ready) && test_bar_warp(bar_xfull + zst, zph) &&
-              test_bar_warp(bar_zfree + b, ((cz >> 1) & 1) ^ 1)) {
+          if ((zj > 0 || s_ready) && (ready & 6u) == 6u) {
             tc_fence_after();
             const uint64_t dB = dXk + zoff;
-            const uint32_t tD = tZ + b * BN;
+            const uint32_t tD = tZ + zb * BN;
             if (elect_one()) {
 #pragma unroll
               for (int ks = 0; ks < DP / 16; ++ks) {
@@ -383,7 +392,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                             ks > 0 ? 1u : 0u);
                 }
               }
-              umma_commit(bar_zfull + b);
+              umma_commit(bar_zfull + zb);
               if (!kGrad) umma_commit(bar_xempty + zst);
               if (!Cfg::S_IN_TMEM && zj + 1 == zit.n_x) umma_commit(bar_sempty);  // stationary tile no longer read
             }
@@ -396,6 +405,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
               zoff = 0;
               zph ^= 1;
             }
+            if (++zb == static_cast<uint32_t>(NZ)) {
+              zb = 0;
+              zbph ^= 1;
+            }
             if (++zj == zit.n_x) {
               zj = 0;
               ++zic;
@@ -405,21 +418,22 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             }
           }
         }
-        // ---- gradient MMA G(cg): ACC += G[cg & 1] * X, G from tensor memory, X MN-major
-        if (kGrad && gi < n_items && cg < cz) {
-          const uint32_t b = cg & 1;
-          if (test_bar_warp(bar_gready + b, (cg >> 1) & 1) &&
-              (gj > 0 || test_bar_warp(bar_accempty, (gic & 1) ^ 1))) {
+        // ---- gradient MMA G(cg): ACC += G[gb] * X, G from tensor memory, X MN-major
+        if (want_g) {
+          if ((ready & 8u) && (gj > 0 || (ready & 16u))) {
             tc_fence_after();
             const uint64_t dB = dXmn + goff;
-            const uint32_t tA = tG + b * Cfg::G_COLS;
+            const uint32_t tA = tZ + gb * BN;
             const bool last = gj + 1 == git.n_x;
             if (elect_one()) {
 #pragma unroll
-              for (int ks = 0; ks < BN / 16; ++ks)
-                umma_bf16_tmem_a(tAcc, tA + 8 * ks, dB + static_cast<uint32_t>(ks * 128), idesc_acc,
+              for (int ks = 0; ks < BN / 16; ++ks) {
+                // slab k of the G tile sits in the first half of the logit columns of slab k
+                const uint32_t a_col = (ks / kKsPerSlab) * Cfg::ZC + 8 * (ks % kKsPerSlab);
+                umma_bf16_tmem_a(tAcc, tA + a_col, dB + static_cast<uint32_t>(ks * 128), idesc_acc,
                                  (gj > 0 || ks > 0) ? 1u : 0u);
-              umma_commit(bar_gfree + b);
+              }
+              umma_commit(bar_zfree + gb);
               umma_commit(bar_xempty + gst);
               if (last) umma_commit(bar_accfull);
             }
@@ -430,6 +444,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             if (++gst == static_cast<uint32_t>(NX)) {
               gst = 0;
               goff = 0;
+            }
+            if (++gb == static_cast<uint32_t>(NZ)) {
+              gb = 0;
+              gbph ^= 1;
             }
             if (last) {
               gj = 0;
@@ -476,7 +494,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     // In a group, warp w reads TMEM lanes 32*(w%4).. (its sub-partition's
     // quarter) and one of two column slabs of the tile, and writes the same
     // slab of the G tile.
-    constexpr int ZC = BN / 2;                    // Z columns per warp per tile (64 or 32)
+    constexpr int ZC = Cfg::ZC;                   // Z columns per warp per tile (64 or 32)
     constexpr int CH = 32;                        // columns per TMEM load
     constexpr int AC = DP / 2;                    // accumulator columns per warp (32 .. 128)
     const int ew = warp - kEpiWarp0;
@@ -486,26 +504,69 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     const int row = q * 32 + lane;                // stationary row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float gs = hdr->grad_scale;
-    const int* keys = kDH ? p.pair_v : p.csc_t;
     uint32_t cnt = 0, ic = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ic) {
       const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
       const int n = it.n_x;
       double item_acc = 0.0;
-      // this row's positives (y = 1), as keys along the streamed dimension
+      // Positives (y = 1).  Position-owned pass: this thread's row (a position)
+      // has at most K of them, walked with a forward cursor over its items.
+      // Item-owned pass: the item tile's pairs, in ascending position, are
+      // walked by the whole warp, 32 at a time, one cursor per warp.
       RowCursor rc{0, 0, 0x7fffffff};
+      int seg = 0, seg_end = 0;
+      uint32_t win = 0xFFFFFFFFu;                 // item-owned pass: pairs seg .. seg + 31, one per lane
       if (kGrad) {
-        const int r = it.s_row0 + row;
-        if (!kDH) {
-          if (r < p.V) cursor_init(rc, keys, __ldg(p.csc_off + r), __ldg(p.csc_off + r + 1), 0);
+        if (kDH) {
+          const int r = it.s_row0 + row;
+          if (r < n_valid) cursor_init(rc, p.pair_v, __ldg(p.row_ptr + r), __ldg(p.row_ptr + r + 1), it.x_tile0 * BN);
         } else {
-          if (r < n_valid) cursor_init(rc, keys, __ldg(p.row_ptr + r), __ldg(p.row_ptr + r + 1), it.x_tile0 * BN);
+          seg = __ldg(p.tile_pair_off + i);
+          seg_end = __ldg(p.tile_pair_off + i + 1);
+          win = seg + lane < seg_end ? static_cast<uint32_t>(__ldg(p.tile_pairs + seg + lane)) : 0xFFFFFFFFu;
         }
       }
       for (int j = 0; j < n; ++j) {
-        const uint32_t c = cnt + j, bz = c % NZ, bg = c % NG;
+        const uint32_t c = cnt + j, bz = c % NZ;
         if ((c & 1) != grp) continue;             // the other group's tile
+        constexpr int NCH = ZC / CH;
+        uint32_t pmask[NCH];                      // item-owned pass: this row's positives per chunk
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) pmask[ch] = 0u;
+        if (kGrad && !kDH) {
+          // consume the item tile's pairs with position < end of this tile; keep
+          // those in this warp's rows and column slab (done before the logit wait,
+          // so the loads overlap it)
+          const int t_hi = (j + 1) * BN, t_lo = j * BN + slab * ZC;
+          while (true) {
+            const uint32_t val = win;
+            const int t = static_cast<int>(val & ((1u << kPairPosBits) - 1u));
+            const int rr = static_cast<int>(val >> kPairPosBits);
+            const unsigned below = __ballot_sync(0xffffffffu, t < t_hi);   // a prefix: positions ascend
+            unsigned mine = __ballot_sync(0xffffffffu, t < t_hi && t >= t_lo && t < t_lo + ZC && (rr >> 5) == q);
+            while (mine != 0u) {
+              const int k = __ffs(mine) - 1;
+              mine &= mine - 1u;
+              const int r_k = __shfl_sync(0xffffffffu, rr, k);
+              const int c_k = __shfl_sync(0xffffffffu, t - t_lo, k);
+              if (lane == (r_k & 31)) {
+#pragma unroll
+                for (int ch = 0; ch < NCH; ++ch)
+                  if ((c_k >> 5) == ch) pmask[ch] |= 1u << (c_k & 31);
+              }
+            }
+            const int nb = __popc(below);
+            seg += nb;
+            // the next window: loaded now, first read at this group's next tile
+            // (nothing to load while no pair was consumed, the common case)
+            if (nb > 0) {
+              const int pi = seg + lane;
+              win = pi < seg_end ? static_cast<uint32_t>(__ldg(p.tile_pairs + pi)) : 0xFFFFFFFFu;
+            }
+            if (nb < 32) break;
+          }
+        }
         if (!wait_bar_warp(bar_zfull + bz, (c / NZ) & 1, wc, wait_tag(4, 4, c))) {
           ok = false;
           break;
@@ -513,65 +574,58 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         tc_fence_after();
         const int key0 = kDH ? (it.x_tile0 + j) * BN : j * BN;   // key of the tile's first column
         float tile_mx = 0.f, tile_l2 = 0.f;
-        // all of this warp's logits of the tile are loaded at once (one wait), so
-        // the logit buffer goes back to the MMA issuer before any math is done
-        constexpr int NCH = ZC / CH;
-        uint32_t r[NCH][CH];
-#pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) tmem_ld<CH>(tmem_base + lane_base + bz * BN + slab * ZC + ch * CH, r[ch]);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_zfree + bz);
-#pragma unroll
+#pragma unroll 1
         for (int ch = 0; ch < NCH; ++ch) {
           const int col0 = slab * ZC + ch * CH;
-          const uint32_t mask = kGrad ? cursor_take_mask(rc, keys, key0 + col0) : 0u;
+          uint32_t r[CH];
+          tmem_ld<CH>(tmem_base + lane_base + bz * BN + col0, r);
+          tmem_ld_wait();
+          if (!kGrad && ch == NCH - 1) {          // no G: the buffer is free once loaded
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_zfree + bz);
+          }
+          const uint32_t mask = !kGrad ? 0u : kDH ? cursor_take_mask(rc, p.pair_v, key0 + col0)
+                                                 : (NCH == 1 || ch == 0) ? pmask[0] : pmask[NCH - 1];
           const bool any_pos = kGrad && __any_sync(0xffffffffu, mask != 0u);
           uint32_t pk[CH / 2];
-          float prod = 1.f;
+          float2 prod = f2(1.f, 1.f), relu = f2(0.f, 0.f);
+          // the chunk's element math; the y = 1 subtraction is compiled into a
+          // separate copy taken only by chunks that hold a positive (rare), so
+          // the common path has no per-element branch or bit test
+          auto chunk_math = [&](auto with_y) {
 #pragma unroll
-          for (int e = 0; e < CH; e += 2) {
-            float g2[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const float z = __uint_as_float(r[ch][e + k]);
-              if (kLoss) {
-                const float u = ex2_approx(-fabsf(z) * kLog2e);   // e^{-|z|}
-                const float pz = 1.f + u;
-                prod *= pz;                                        // log1p batched: one lg2 per chunk
-                tile_mx += fmaxf(z, 0.f);
-                if (kGrad) {
-                  const float rp = rcp_approx(pz);                 // 1 / (1 + e^{-|z|})
-                  g2[k] = z >= 0.f ? rp : u * rp;                  // sigmoid(z)
+            for (int e = 0; e < CH; e += 2) {
+              const float2 z = f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+              float2 g = f2(0.f, 0.f);
+              if (kLoss && kGrad) g = bce_pair_loss_grad(z, prod, relu);
+              else if (kLoss) bce_pair_loss(z, prod, relu);
+              else g = sigmoid_pair(z);
+              if (kGrad) {
+                if (decltype(with_y)::value) {                     // y = 1 at the masked columns
+                  g.x -= static_cast<float>((mask >> e) & 1u);
+                  g.y -= static_cast<float>((mask >> (e + 1)) & 1u);
                 }
-              } else {
-                g2[k] = fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);   // sigmoid(z)
+                pk[e >> 1] = pack_bf16x2(g.x, g.y);
               }
             }
-            if (kGrad) {
-              if (any_pos) {                                       // y = 1 at the masked columns
-                g2[0] -= static_cast<float>((mask >> e) & 1u);
-                g2[1] -= static_cast<float>((mask >> (e + 1)) & 1u);
-              }
-              pk[e >> 1] = pack_bf16x2(g2[0], g2[1]);
-            }
+          };
+          if (any_pos) chunk_math(std::true_type{});
+          else chunk_math(std::false_type{});
+          if (kLoss) {
+            // CH / 2 factors per component: the product of the -(1 + u) factors is positive
+            tile_l2 += lg2_approx(prod.x * prod.y);
+            tile_mx += relu.x + relu.y;
           }
-          if (kLoss) tile_l2 += lg2_approx(prod);
-          if (kGrad) {
-            if (ch == 0 && !wait_bar_warp(bar_gfree + bg, ((c / NG) & 1) ^ 1, wc, wait_tag(4, 8, c))) {
-              ok = false;
-              break;
-            }
-            tmem_st16(tmem_base + lane_base + Cfg::G_COL + bg * Cfg::G_COLS + col0 / 2, pk);
-          }
+          // G over the first half of this warp's own (already loaded) logit columns
+          if (kGrad) tmem_st16(tmem_base + lane_base + bz * BN + slab * ZC + ch * (CH / 2), pk);
         }
         if (!ok) break;
         if (kGrad) {
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_gready + bg);   // this warp's part of G is in place
+          if (lane == 0) mbar_arrive(bar_gready + bz);   // this warp's part of G is in place
         }
         if (kLoss) {
           if (j == n - 1) {
