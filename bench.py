@@ -38,7 +38,7 @@ METRIC = "fused BCE fwd+bwd tokens/s at V=876k,D=64 on 1 B200; % of roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
-TILE_SOURCES = ["tile_engine.cuh", "common.cuh", "ptx_sm100.cuh"]
+TILE_SOURCES = ["tile_engine.cuh", "common.cuh", "ptx_sm100.cuh", "elementwise.cuh", "pair_sort.cuh"]
 
 
 def parse_args():
@@ -85,22 +85,30 @@ def committed_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 50 ms; only those taken inside the timed window are kept."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.t0 = self.t1 = None
 
     def start(self):
+        """Start sampling (before the warm-up, so that the sampler is running when timing begins)."""
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+
+    def mark_begin(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
 
     def stop(self):
         if self.proc is None:
@@ -111,20 +119,25 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
-        sm, smax, reasons = [], None, set()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 10]
+        sm, smax, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             try:
-                sm.append(float(r[1]))
-                smax = float(r[2])
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f")
+                if self.t0 is not None and not (self.t0 <= ts <= self.t1):
+                    continue
+                sm.append(float(r[2]))
+                smax = float(r[3])
+                power.append(float(r[4]))
             except ValueError:
                 continue
-            for name, val in zip(names, r[5:9]):
+            for name, val in zip(names, r[6:10]):
                 if val.strip().lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w": statistics.median(power) if power else None}
 
 
 def sample_problem(p, n_items):
@@ -247,6 +260,8 @@ def run_ours(args):
     def step():
         B.cutbce_forward_backward(prob, None, loss, dH, dE, ws, stream)
 
+    sampler = ClockSampler(local)
+    sampler.start()
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -259,16 +274,16 @@ def run_ours(args):
     B.cutbce_profile_read(reset=True)
     B.cutbce_profile_enable(True)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    sampler = ClockSampler(local)
     barrier()
     torch.cuda.synchronize(dev)
-    sampler.start()
+    sampler.mark_begin()
     for s, e in ev:
         flush.zero_()
         s.record(stream)
         step()
         e.record(stream)
     torch.cuda.synchronize(dev)
+    sampler.mark_end()
     barrier()
     clocks = sampler.stop()
     B.cutbce_profile_enable(False)

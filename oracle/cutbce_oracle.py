@@ -23,14 +23,14 @@ The logits X = A E^T are formed here chunk by chunk over the vocabulary (the
 dense multi-hot Y inside the element loss (the Eq. (1)/(2) form), so that this
 file is a plain restatement and shares no arithmetic with the GPU design.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the paper is silent:
   * normalisation: MEAN_VALID_POSITIONS (default) divides the summed loss by the
     number of valid positions; SUM does not divide; MEAN_ELEMENTS divides by
     n_valid * V (Eq. (3)'s 1/V times section III-B's 1/BN);
   * duplicate ids in a row count once (Y is multi-hot, y in {0, 1});
   * -1 marks an empty slot; an id < -1 or >= V in a valid row is an error;
     id 0 is an ordinary item;
-  * the per-position `weights` of the pages' API is read as a {0, 1} mask: a
+  * the per-position `weights` of the paper's API is read as a {0, 1} mask: a
     masked row adds no loss, gets a zero dH row and adds nothing to dE; its ids
     are ignored entirely (not even range-checked);
   * the upstream gradient is one scalar g (default 1) multiplying dH and dE;

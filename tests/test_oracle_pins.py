@@ -1,6 +1,6 @@
 """Pins of the float64 oracle to things other than itself.
 
-Each test ties the oracle to a fact fixed by the pages' mathematics ("Cut Binary
+Each test ties the oracle to a fact fixed by the mathematics ("Cut Binary
 Cross Entropy", section III-A Eqs. (1)-(3), section III-B Eq. (4)) or by an
 independent implementation: the literal Eq. (1), closed forms at H = 0 and
 E = 0, central finite differences, torch's own binary_cross_entropy_with_logits
