@@ -25,7 +25,9 @@ constexpr int kMaxSplits = 64;        // dH partial splits over the vocabulary
 constexpr int kTileThreads = 576;     // 18 warps: TMA producer, MMA issuer, 16 epilogue
 constexpr int kEpiWarp0 = 2;
 constexpr int kNumEpiWarps = 16;      // 2 groups x (4 TMEM lane quarters x 2 column slabs)
-constexpr int kEpiGroupWarps = 8;     // warps that take one tile
+constexpr int kEpiGroups = 1;         // epilogue groups taking tiles in turn
+constexpr int kEpiGroupWarps = kNumEpiWarps / kEpiGroups;   // warps that take one tile
+constexpr int kEpiSlabs = kEpiGroupWarps / 4;               // column slabs of a tile (4 TMEM lane quarters each)
 
 // First 256 bytes of the workspace.
 struct WsHeader {
@@ -47,7 +49,7 @@ struct TileCfg {
   // stages of the streamed-operand ring: a streamed tile is held from its logit MMA
   // (issued up to NZ-1 tiles early) until its gradient MMA completes, and the ring
   // must still cover the L2 -> shared memory latency of the next loads
-  static constexpr int NX = DP == 64 ? 12 : DP == 128 ? 6 : DP == 192 ? 7 : 5;
+  static constexpr int NX = DP == 64 ? 12 : DP == 128 ? 5 : DP == 192 ? 7 : 4;
   // fp32 logit tiles in tensor memory.  The bf16 G tile of a logit tile is
   // written over that tile's own columns (each warp over the slab it loaded),
   // so a buffer holds Z, then G, and is free once the gradient MMA reading G
@@ -55,7 +57,7 @@ struct TileCfg {
   static constexpr int NZ = 3;
   static constexpr uint32_t S_BYTES = kTileM * DP * 2;       // stationary tile
   static constexpr uint32_t X_BYTES = BN * DP * 2;           // streamed tile
-  static constexpr int ZC = BN / 2;                          // logit columns per epilogue warp (one slab)
+  static constexpr int ZC = BN / kEpiSlabs;                  // logit columns per epilogue warp (one slab)
   static constexpr int ACC_COL = NZ * BN;                    // TMEM column of the gradient accumulator
   static constexpr int TMEM_COLS = 512;
   // The stationary tile is copied into tensor memory (bf16 pairs, DP/2 columns)
@@ -63,7 +65,10 @@ struct TileCfg {
   static constexpr int S_COL = ACC_COL + DP;
   static constexpr bool S_IN_TMEM = S_COL + DP / 2 <= TMEM_COLS;
   static constexpr int NUM_BARS = 2 + 2 * NX + 3 * NZ + 3;  // see the kernel for the list
-  static constexpr uint32_t SMEM_BYTES = 1024 + S_BYTES + NX * X_BYTES + NUM_BARS * 8 + 16 + 64;
+  // per epilogue warp: positives of its 32 rows, one word per 32 columns of its slab
+  static constexpr int MASK_WORDS = ZC >= 32 ? ZC / 32 : 1;
+  static constexpr uint32_t MASK_BYTES = kNumEpiWarps * 32 * MASK_WORDS * 4;
+  static constexpr uint32_t SMEM_BYTES = 1024 + S_BYTES + NX * X_BYTES + MASK_BYTES + NUM_BARS * 8 + 16 + 64;
   static_assert(ACC_COL + DP <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(SMEM_BYTES > 232448 / 2, "one CTA per SM keeps the TMEM allocation uncontended");

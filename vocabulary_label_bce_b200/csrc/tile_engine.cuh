@@ -204,7 +204,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sS = smem;
   uint8_t* sX = sS + S_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + NX * X_BYTES);
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sX + NX * X_BYTES);   // [16 warps][32 rows][MASK_WORDS]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + NX * X_BYTES + Cfg::MASK_BYTES);
   uint64_t* bar_sfull = bars + 0;                 // stationary tile landed (TMA)
   uint64_t* bar_sempty = bars + 1;                // stationary tile free (MMA commit)
   uint64_t* bar_xfull = bars + 2;                 // [NX] streamed tile landed
@@ -495,15 +496,19 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     // quarter) and one of two column slabs of the tile, and writes the same
     // slab of the G tile.
     constexpr int ZC = Cfg::ZC;                   // Z columns per warp per tile (64 or 32)
-    constexpr int CH = 32;                        // columns per TMEM load
-    constexpr int AC = DP / 2;                    // accumulator columns per warp (32 .. 128)
+    constexpr int CH = ZC < 32 ? ZC : 32;         // columns per TMEM load
+    constexpr int AC = DP / kEpiSlabs;            // accumulator columns per warp (16 .. 128)
     const int ew = warp - kEpiWarp0;
-    const uint32_t grp = static_cast<uint32_t>(ew >> 3);   // tile-parity group
+    const uint32_t grp = static_cast<uint32_t>(ew / kEpiGroupWarps);   // group: takes tiles c with c mod groups = grp
     const int q = warp & 3;                       // TMEM lane quarter
-    const int slab = (ew >> 2) & 1;               // column slab within the group
+    const int slab = (ew >> 2) % kEpiSlabs;       // column slab within the group
     const int row = q * 32 + lane;                // stationary row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float gs = hdr->grad_scale;
+    uint32_t* wmask = sMask + ew * 32 * Cfg::MASK_WORDS;   // this warp's positives scratch
+#pragma unroll
+    for (int k = 0; k < Cfg::MASK_WORDS; ++k) wmask[lane * Cfg::MASK_WORDS + k] = 0u;
+    __syncwarp();
     uint32_t cnt = 0, ic = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ic) {
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       }
       for (int j = 0; j < n; ++j) {
         const uint32_t c = cnt + j, bz = c % NZ;
-        if ((c & 1) != grp) continue;             // the other group's tile
+        if (c % kEpiGroups != grp) continue;      // another group's tile
         constexpr int NCH = ZC / CH;
         uint32_t pmask[NCH];                      // item-owned pass: this row's positives per chunk
 #pragma unroll
@@ -539,32 +544,60 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           // those in this warp's rows and column slab (done before the logit wait,
           // so the loads overlap it)
           const int t_hi = (j + 1) * BN, t_lo = j * BN + slab * ZC;
-          while (true) {
-            const uint32_t val = win;
+          bool any_pair = false;                  // this lane set a bit in the scratch
+          // one window of 32 pairs: set this warp's bits, return how many pairs lie below t_hi
+          auto take = [&](uint32_t val) -> int {
             const int t = static_cast<int>(val & ((1u << kPairPosBits) - 1u));
             const int rr = static_cast<int>(val >> kPairPosBits);
             const unsigned below = __ballot_sync(0xffffffffu, t < t_hi);   // a prefix: positions ascend
-            unsigned mine = __ballot_sync(0xffffffffu, t < t_hi && t >= t_lo && t < t_lo + ZC && (rr >> 5) == q);
-            while (mine != 0u) {
-              const int k = __ffs(mine) - 1;
-              mine &= mine - 1u;
-              const int r_k = __shfl_sync(0xffffffffu, rr, k);
-              const int c_k = __shfl_sync(0xffffffffu, t - t_lo, k);
-              if (lane == (r_k & 31)) {
+            // each lane holding one of this warp's pairs sets its bit in the row's
+            // word in shared memory (the lanes work in parallel)
+            if (t < t_hi && t >= t_lo && t < t_lo + ZC && (rr >> 5) == q) {
+              const int cc = t - t_lo;
+              atomicOr(wmask + (rr & 31) * Cfg::MASK_WORDS + (cc >> 5), 1u << (cc & 31));
+              any_pair = true;
+            }
+            return __popc(below);
+          };
+          const int seg0 = seg;
+          int nb = take(win);
+          seg += nb;
+          if (nb == 32) {
+            // a hot tile (more than one window of pairs): fetch four windows per
+            // round trip to memory instead of one
+            constexpr int kBatch = 4;
+            bool more = true;
+            while (more) {
+              uint32_t w[kBatch];
 #pragma unroll
-                for (int ch = 0; ch < NCH; ++ch)
-                  if ((c_k >> 5) == ch) pmask[ch] |= 1u << (c_k & 31);
+              for (int k = 0; k < kBatch; ++k) {
+                const int pi = seg + 32 * k + lane;
+                w[k] = pi < seg_end ? static_cast<uint32_t>(__ldg(p.tile_pairs + pi)) : 0xFFFFFFFFu;
+              }
+#pragma unroll
+              for (int k = 0; k < kBatch; ++k) {
+                if (!more) break;
+                nb = take(w[k]);
+                seg += nb;
+                more = nb == 32;
               }
             }
-            const int nb = __popc(below);
-            seg += nb;
-            // the next window: loaded now, first read at this group's next tile
-            // (nothing to load while no pair was consumed, the common case)
-            if (nb > 0) {
-              const int pi = seg + lane;
-              win = pi < seg_end ? static_cast<uint32_t>(__ldg(p.tile_pairs + pi)) : 0xFFFFFFFFu;
+          }
+          // the next window: loaded now, first read at this group's next tile
+          // (nothing to load while no pair was consumed, the common case)
+          if (seg != seg0) {
+            const int pi = seg + lane;
+            win = pi < seg_end ? static_cast<uint32_t>(__ldg(p.tile_pairs + pi)) : 0xFFFFFFFFu;
+          }
+          if (__any_sync(0xffffffffu, any_pair)) {
+            __syncwarp();
+            // this lane's row: take its words and clear them for the next tile
+#pragma unroll
+            for (int ch = 0; ch < NCH; ++ch) {
+              pmask[ch] = wmask[lane * Cfg::MASK_WORDS + ch];
+              wmask[lane * Cfg::MASK_WORDS + ch] = 0u;
             }
-            if (nb < 32) break;
+            __syncwarp();
           }
         }
         if (!wait_bar_warp(bar_zfull + bz, (c / NZ) & 1, wc, wait_tag(4, 4, c))) {
@@ -618,7 +651,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             tile_mx += relu.x + relu.y;
           }
           // G over the first half of this warp's own (already loaded) logit columns
-          if (kGrad) tmem_st16(tmem_base + lane_base + bz * BN + slab * ZC + ch * (CH / 2), pk);
+          if (kGrad) {
+            if constexpr (CH == 32) tmem_st16(tmem_base + lane_base + bz * BN + slab * ZC + ch * (CH / 2), pk);
+            else tmem_st8(tmem_base + lane_base + bz * BN + slab * ZC + ch * (CH / 2), pk);
+          }
         }
         if (!ok) break;
         if (kGrad) {
@@ -646,7 +682,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
         if (lane == 0) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + ew] = val;
       }
-      if (kGrad && ((cnt + n - 1) & 1) == grp) {
+      if (kGrad && (cnt + n - 1) % kEpiGroups == grp) {
         // the group that took the item's last tile reads the accumulator out
         if (!wait_bar_warp(bar_accfull, ic & 1, wc, wait_tag(4, 9, ic))) break;
         tc_fence_after();
