@@ -16,8 +16,7 @@
 // subtraction negates the exponent and roughly reflects the mantissa; with
 // C = 0x7EF31000 the relative error |1 - w r0| is at most 0.0506 for every
 // normal w), then the cubically convergent step r1 = r0 (1 + e + e^2) with
-// e = 1 - w r0, which leaves |1 - w r1| = |e|^3 <= 1.3e-4, and optionally one
-// Newton step r2 = r1 (1 + e1) (error <= 1.7e-8).  The seed is formed from -w
+// e = 1 - w r0, which leaves |1 - w r1| = |e|^3 <= 1.3e-4.  The seed is formed from -w
 // (bits(-w) = bits(w) + 2^31), which the FMA pipe produces in the same
 // instruction as 1 + u, so no separate negation is needed.
 //
@@ -69,14 +68,12 @@ __device__ __forceinline__ void bce_pair_loss(float2 z, float2& prod, float2& re
 // Gradient only (the position-owned pass, and the item pass without the
 // loss): sigmoid(z) = 1 / (1 + 2^{-z log2 e}) over the whole range, the
 // exponent clamped at 100 (below z = -69.3 the result is 2^-100 instead of
-// a smaller positive number).  Seed, cubic step and one Newton step:
-// |rel err| <= 1.7e-8 plus rounding.
+// a smaller positive number).  Seed and cubic step: |rel err| <= 1.3e-4 plus
+// rounding, well inside the bf16 rounding of G that follows (up to 2^-9).
 __device__ __forceinline__ float2 sigmoid_pair(float2 z) {
   const float2 u = f2(ex2_approx(fminf(-z.x * kLog2eF, 100.f)), ex2_approx(fminf(-z.y * kLog2eF, 100.f)));
   const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + u)
-  const float2 r = rcp2_cubic(nw);
-  const float2 e = __ffma2_rn(nw, r, f2(1.f, 1.f));
-  return __ffma2_rn(r, e, r);                                        // Newton step
+  return rcp2_cubic(nw);
 }
 
 }  // namespace cutbce

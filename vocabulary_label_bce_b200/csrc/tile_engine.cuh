@@ -636,8 +636,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
               else g = sigmoid_pair(z);
               if (kGrad) {
                 if (decltype(with_y)::value) {                     // y = 1 at the masked columns
-                  g.x -= static_cast<float>((mask >> e) & 1u);
-                  g.y -= static_cast<float>((mask >> (e + 1)) & 1u);
+                  if (mask & (1u << e)) g.x -= 1.f;                // a predicated add, no conversion
+                  if (mask & (1u << (e + 1))) g.y -= 1.f;
                 }
                 pk[e >> 1] = pack_bf16x2(g.x, g.y);
               }
