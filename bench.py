@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--workload", default="sasrec_876k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-items", type=int, default=16384)
+    ap.add_argument("--cpu-sample-items", type=int, default=32768)
     return ap.parse_args()
 
 

@@ -24,10 +24,12 @@ constexpr int kMaxCtas = 256;         // upper bound of a persistent grid
 constexpr int kMaxSplits = 64;        // dH partial splits over the vocabulary
 constexpr int kTileThreads = 576;     // 18 warps: TMA producer, MMA issuer, 16 epilogue
 constexpr int kEpiWarp0 = 2;
-constexpr int kNumEpiWarps = 16;      // 2 groups x (4 TMEM lane quarters x 2 column slabs)
-constexpr int kEpiGroups = 1;         // epilogue groups taking tiles in turn
-constexpr int kEpiGroupWarps = kNumEpiWarps / kEpiGroups;   // warps that take one tile
-constexpr int kEpiSlabs = kEpiGroupWarps / 4;               // column slabs of a tile (4 TMEM lane quarters each)
+constexpr int kNumEpiWarps = 16;      // groups x (4 TMEM lane quarters x column slabs)
+// Epilogue groups taking tiles in turn: two for the item-owned pass (one
+// group's tile handshakes overlap the other's math), one for the
+// position-owned pass (all 16 warps on every tile).
+template <bool kDH>
+__host__ __device__ constexpr int epi_groups() { return kDH ? 1 : 2; }
 
 // First 256 bytes of the workspace.
 struct WsHeader {
@@ -40,9 +42,13 @@ struct WsHeader {
   int wait_block;      // CTA of that wait
 };
 
-// Geometry of the tcgen05 tile engine for one padded feature width DP.
-template <int DP>
+// Geometry of the tcgen05 tile engine for one padded feature width DP and G
+// epilogue groups.
+template <int DP, int G = 1>
 struct TileCfg {
+  static constexpr int GROUPS = G;                           // epilogue groups taking tiles in turn
+  static constexpr int GROUP_WARPS = kNumEpiWarps / G;       // warps that take one tile
+  static constexpr int SLABS = GROUP_WARPS / 4;              // column slabs of a tile (4 TMEM lane quarters each)
   static_assert(DP % 64 == 0 && DP >= 64 && DP <= 256, "DP must be 64, 128, 192 or 256");
   static constexpr int BN = DP <= 128 ? 128 : 64;          // streamed rows per tile (Z columns)
   static constexpr int NKB = DP / 64;                        // 128-byte column blocks per row
@@ -57,7 +63,7 @@ struct TileCfg {
   static constexpr int NZ = 3;
   static constexpr uint32_t S_BYTES = kTileM * DP * 2;       // stationary tile
   static constexpr uint32_t X_BYTES = BN * DP * 2;           // streamed tile
-  static constexpr int ZC = BN / kEpiSlabs;                  // logit columns per epilogue warp (one slab)
+  static constexpr int ZC = BN / SLABS;                      // logit columns per epilogue warp (one slab)
   static constexpr int ACC_COL = NZ * BN;                    // TMEM column of the gradient accumulator
   static constexpr int TMEM_COLS = 512;
   // The stationary tile is copied into tensor memory (bf16 pairs, DP/2 columns)

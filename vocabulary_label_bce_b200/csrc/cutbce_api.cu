@@ -241,7 +241,7 @@ template <int DP, bool kLoss, bool kGrad, bool kDH>
 cudaError_t launch_tile(int grid, const CUtensorMap& s, const CUtensorMap& x, const TileParams& tp,
                         cudaStream_t st) {
   auto kern = k_tile<DP, kLoss, kGrad, kDH>;
-  constexpr uint32_t smem = TileCfg<DP>::SMEM_BYTES;
+  constexpr uint32_t smem = TileCfg<DP, epi_groups<kDH>()>::SMEM_BYTES;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -189,7 +189,7 @@ __device__ __forceinline__ uint32_t cursor_take_mask(RowCursor& rc, const int* _
 template <int DP, bool kLoss, bool kGrad, bool kDH>
 __global__ void __launch_bounds__(kTileThreads, 1)
     k_tile(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmX, TileParams p) {
-  using Cfg = TileCfg<DP>;
+  using Cfg = TileCfg<DP, epi_groups<kDH>()>;
   constexpr int BN = Cfg::BN;
   constexpr int NKB = Cfg::NKB;
   constexpr int NX = Cfg::NX;
@@ -259,11 +259,11 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
     for (int b = 0; b < NZ; ++b) {
       mbar_init(bar_zfull + b, 1);
-      mbar_init(bar_zfree + b, kGrad ? 1 : kEpiGroupWarps);
-      mbar_init(bar_gready + b, kEpiGroupWarps);
+      mbar_init(bar_zfree + b, kGrad ? 1 : Cfg::GROUP_WARPS);
+      mbar_init(bar_gready + b, Cfg::GROUP_WARPS);
     }
     mbar_init(bar_accfull, 1);
-    mbar_init(bar_accempty, kEpiGroupWarps);
+    mbar_init(bar_accempty, Cfg::GROUP_WARPS);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -497,11 +497,11 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     // slab of the G tile.
     constexpr int ZC = Cfg::ZC;                   // Z columns per warp per tile (64 or 32)
     constexpr int CH = ZC < 32 ? ZC : 32;         // columns per TMEM load
-    constexpr int AC = DP / kEpiSlabs;            // accumulator columns per warp (16 .. 128)
+    constexpr int AC = DP / Cfg::SLABS;            // accumulator columns per warp (16 .. 128)
     const int ew = warp - kEpiWarp0;
-    const uint32_t grp = static_cast<uint32_t>(ew / kEpiGroupWarps);   // group: takes tiles c with c mod groups = grp
+    const uint32_t grp = static_cast<uint32_t>(ew / Cfg::GROUP_WARPS);   // group: takes tiles c with c mod groups = grp
     const int q = warp & 3;                       // TMEM lane quarter
-    const int slab = (ew >> 2) % kEpiSlabs;       // column slab within the group
+    const int slab = (ew >> 2) % Cfg::SLABS;       // column slab within the group
     const int row = q * 32 + lane;                // stationary row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const float gs = hdr->grad_scale;
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       }
       for (int j = 0; j < n; ++j) {
         const uint32_t c = cnt + j, bz = c % NZ;
-        if (c % kEpiGroups != grp) continue;      // another group's tile
+        if (c % Cfg::GROUPS != grp) continue;      // another group's tile
         constexpr int NCH = ZC / CH;
         uint32_t pmask[NCH];                      // item-owned pass: this row's positives per chunk
 #pragma unroll
@@ -682,7 +682,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
         if (lane == 0) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + ew] = val;
       }
-      if (kGrad && (cnt + n - 1) % kEpiGroups == grp) {
+      if (kGrad && (cnt + n - 1) % Cfg::GROUPS == grp) {
         // the group that took the item's last tile reads the accumulator out
         if (!wait_bar_warp(bar_accfull, ic & 1, wc, wait_tag(4, 9, ic))) break;
         tc_fence_after();
