@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-items", type=int, default=32768)
+    ap.add_argument("--calls-only", type=int, default=0,
+                    help="run this many untimed fused calls on --workload and exit (a target for ncu)")
     return ap.parse_args()
 
 
@@ -380,8 +382,35 @@ def run_ours(args):
     return 0
 
 
+def run_calls_only(args):
+    """N plain fused calls, no timing and no output: the command ncu captures."""
+    import torch
+    from vocabulary_label_bce_b200 import binding as B
+    from vocabulary_label_bce_b200 import workloads as W
+    p = W.draw_config(args.workload, seed=0)
+    dev = torch.device("cuda", 0)
+    H = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    E = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    tg = torch.from_numpy(p.targets).to(dev)
+    m = torch.from_numpy(p.mask).to(dev)
+    prob = B.make_problem(H, E, tg, m, "mean")
+    ws = torch.empty(B.cutbce_workspace_size(prob), dtype=torch.uint8, device=dev)
+    loss = torch.empty((), dtype=torch.float64, device=dev)
+    dH = torch.empty((p.T, p.D), dtype=torch.float32, device=dev)
+    dE = torch.empty((p.V, p.D), dtype=torch.float32, device=dev)
+    for _ in range(args.calls_only):
+        B.cutbce_forward_backward(prob, None, loss, dH, dE, ws)
+    torch.cuda.synchronize(dev)
+    status = B.cutbce_read_status(ws)
+    if status != 0:
+        raise SystemExit(f"device status {B.cutbce_status_string(status)}")
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.calls_only > 0:
+        return run_calls_only(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
