@@ -1,11 +1,14 @@
-"""Host-side check of the reciprocal the tile engine uses for the sigmoid.
+"""Host-side check of the reciprocals the tile engine uses for the sigmoid.
 
-The kernels compute 1/w on the FMA pipe instead of the SFU: an exponent-flip
-seed r0 = bits^-1(C - bits(w)) with C = 0x7EF31000 (formed from -w, whose
-bits are bits(w) + 2^31), then one cubically convergent step
-r1 = r0 (1 + e + e^2), e = 1 - w r0.  This test replays the same float32
-operations (each fused multiply-add rounded once, as on the GPU) over the
-ranges the kernels use and checks the stated bound |1 - w r1| <= 1.3e-4.
+The kernels compute 1/w on the FMA pipe instead of the SFU: a seed, then one
+cubically convergent step r1 = r0 (1 + e + e^2), e = 1 - w r0.
+  * item pass, w in (1, 2]: linear minimax seed r0 = (24 - 8 w) / 17, one
+    fused multiply-add on -w; bound (1/17)^3 = 2.1e-4;
+  * gradient-only passes, w up to 2^100: exponent-flip seed
+    r0 = bits^-1(C - bits(w)), C = 0x7EF31000 (formed from -w, whose bits are
+    bits(w) + 2^31); bound 1.3e-4.
+This test replays the same float32 operations (each fused multiply-add
+rounded once, as on the GPU) over the ranges the kernels use.
 """
 import numpy as np
 
@@ -26,9 +29,21 @@ def rcp_cubic(w):
     return fma32(r, t, r)
 
 
+def rcp_linear_seed(w):
+    w = np.asarray(w, np.float32)
+    nw = -w
+    r = fma32(nw, np.float32(8.0 / 17.0), np.float32(24.0 / 17.0))
+    e = fma32(nw, r, np.float32(1.0))
+    t = fma32(e, e, e)
+    return fma32(r, t, r)
+
+
 def test_reciprocal_bound_item_range():
     # item pass: w = 1 + e^{-|z|} in (1, 2]
     w = np.linspace(1.0, 2.0, 400001, dtype=np.float32)[1:]
+    rel = np.abs(1.0 - w.astype(np.float64) * rcp_linear_seed(w).astype(np.float64))
+    assert rel.max() <= (1.0 / 17.0) ** 3 + 1e-6, rel.max()
+    # and the exponent-flip variant on the same range
     rel = np.abs(1.0 - w.astype(np.float64) * rcp_cubic(w).astype(np.float64))
     assert rel.max() <= 1.3e-4 + 1e-6, rel.max()
 

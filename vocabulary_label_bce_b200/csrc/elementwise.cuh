@@ -12,13 +12,16 @@
 // pipe, and the logarithm is taken once per 32 logits of a row as the log2 of
 // the product of their w (each factor is in (1, 2], so 32 of them stay finite).
 //
-// Reciprocal: exponent-flip seed r0 = bits^-1(C - bits(w)) (the integer
-// subtraction negates the exponent and roughly reflects the mantissa; with
-// C = 0x7EF31000 the relative error |1 - w r0| is at most 0.0506 for every
-// normal w), then the cubically convergent step r1 = r0 (1 + e + e^2) with
-// e = 1 - w r0, which leaves |1 - w r1| = |e|^3 <= 1.3e-4.  The seed is formed from -w
-// (bits(-w) = bits(w) + 2^31), which the FMA pipe produces in the same
-// instruction as 1 + u, so no separate negation is needed.
+// Reciprocal, on the FMA pipe: a seed, then the cubically convergent step
+// r1 = r0 (1 + e + e^2) with e = 1 - w r0, which leaves |1 - w r1| = |e|^3.
+//  * item pass, w in (1, 2]: linear minimax seed (24 - 8 w) / 17, |e| <= 1/17,
+//    so |1 - w r1| <= 2.1e-4;
+//  * gradient-only passes, w in (1, 2^100]: exponent-flip seed
+//    r0 = bits^-1(C - bits(w)) (the integer subtraction negates the exponent
+//    and roughly reflects the mantissa; with C = 0x7EF31000, |e| <= 0.0506 for
+//    every normal w), so |1 - w r1| <= 1.3e-4.
+// Both seeds are formed from -w, which the FMA pipe produces in the same
+// instruction as 1 + u (bits(-w) = bits(w) + 2^31 for the integer seed).
 //
 // Packed fp32x2 instructions (two lanes of work per instruction) halve the
 // issue slots of the FMA-pipe part; the SFU and the selects stay scalar.
@@ -44,23 +47,36 @@ __device__ __forceinline__ float2 rcp2_cubic(float2 nw) {
   return __ffma2_rn(r, t, r);                          // r0 (1 + e + e^2)
 }
 
+// 1 / w for w in [1, 2] from nw = -w: linear minimax seed r0 = (24 - 8 w) / 17
+// (|rel err| <= 1/17), one FFMA2 instead of two integer subtractions, then the
+// cubic step: |rel err| <= (1/17)^3 = 2.1e-4.
+__device__ __forceinline__ float2 rcp2_unit_interval(float2 nw) {
+  float2 r = __ffma2_rn(nw, f2(8.f / 17.f, 8.f / 17.f), f2(24.f / 17.f, 24.f / 17.f));
+  const float2 e = __ffma2_rn(nw, r, f2(1.f, 1.f));    // 1 - w r0
+  const float2 t = __ffma2_rn(e, e, e);                // e + e^2
+  return __ffma2_rn(r, t, r);                          // r0 (1 + e + e^2)
+}
+
 // Item-owned pass, loss and gradient: returns sigmoid(z) for both logits and
 // folds their loss terms into the running products `prod` (of w, sign-free
 // over an even count of factors per component) and the running sum `relu`
-// of max(z, 0).
+// of max(z, 0).  z log2 e is formed for both logits in one packed multiply;
+// the exponential takes -|.| of it as operand modifiers.
 __device__ __forceinline__ float2 bce_pair_loss_grad(float2 z, float2& prod, float2& relu) {
-  const float2 u = f2(ex2_approx(-fabsf(z.x) * kLog2eF), ex2_approx(-fabsf(z.y) * kLog2eF));
-  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + u)
+  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
+  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));   // e^{-|z|}
+  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));           // -(1 + u)
   prod = __fmul2_rn(prod, nw);
   relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
-  const float2 r = rcp2_cubic(nw);
+  const float2 r = rcp2_unit_interval(nw);
   const float2 ur = __fmul2_rn(u, r);
   return f2(z.x >= 0.f ? r.x : ur.x, z.y >= 0.f ? r.y : ur.y);
 }
 
 // Item-owned pass, loss only.
 __device__ __forceinline__ void bce_pair_loss(float2 z, float2& prod, float2& relu) {
-  const float2 u = f2(ex2_approx(-fabsf(z.x) * kLog2eF), ex2_approx(-fabsf(z.y) * kLog2eF));
+  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
+  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));
   prod = __fmul2_rn(prod, __fadd2_rn(u, f2(1.f, 1.f)));
   relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
 }
@@ -71,7 +87,8 @@ __device__ __forceinline__ void bce_pair_loss(float2 z, float2& prod, float2& re
 // a smaller positive number).  Seed and cubic step: |rel err| <= 1.3e-4 plus
 // rounding, well inside the bf16 rounding of G that follows (up to 2^-9).
 __device__ __forceinline__ float2 sigmoid_pair(float2 z) {
-  const float2 u = f2(ex2_approx(fminf(-z.x * kLog2eF, 100.f)), ex2_approx(fminf(-z.y * kLog2eF, 100.f)));
+  const float2 tz = __fmul2_rn(z, f2(-kLog2eF, -kLog2eF));
+  const float2 u = f2(ex2_approx(fminf(tz.x, 100.f)), ex2_approx(fminf(tz.y, 100.f)));
   const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + u)
   return rcp2_cubic(nw);
 }
