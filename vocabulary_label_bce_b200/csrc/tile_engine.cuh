@@ -607,7 +607,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         tc_fence_after();
         const int key0 = kDH ? (it.x_tile0 + j) * BN : j * BN;   // key of the tile's first column
         float tile_mx = 0.f, tile_l2 = 0.f;
-#pragma unroll 1
+#pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
           const int col0 = slab * ZC + ch * CH;
           uint32_t r[CH];
