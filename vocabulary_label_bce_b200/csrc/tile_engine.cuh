@@ -18,27 +18,35 @@
 //     Z = H_t E_v^T    -> sigmoid -> G (bf16, TMEM)
 //     dH_t += G E_v    (partial per split, reduced later in a fixed order)
 //
-// The sparse targets enter in registers: each epilogue thread owns one row of
-// the tile and walks that row's sorted positives with a forward-only cursor;
-// where a positive falls in the current 32-column chunk it subtracts 1 from
-// sigmoid(z) (y = 1).  The dense loss uses no Y at all (Eq. (2):
-// l(x,y) = l(x,0) - y x); the -y x part is the sparse correction summed in the
-// prep kernel.
+// The sparse targets (y = 1) are applied inside the tile, before G is rounded
+// to bf16, so that G = sigmoid(z) - y is rounded once:
+//   * position-owned pass: each epilogue thread owns one position row, which
+//     has at most K positives; it walks them with a forward-only cursor;
+//   * item-owned pass: the pairs are grouped by item tile in ascending
+//     position; each warp walks its item tile's pairs 32 at a time, and the
+//     lanes holding a pair of the warp's rows and slab set the bit in a
+//     per-warp shared-memory word (atomicOr), which the row's lane then takes.
+// Chunks holding a positive run a separate copy of the element loop with the
+// subtraction, so the common path has no per-element test.  The dense loss
+// uses no Y at all (Eq. (2): l(x,y) = l(x,0) - y x); the -y x part is the
+// sparse correction summed in the prep kernel.
 //
-// Warp roles (640 threads, one CTA per SM):
-//   warp 0      TMA producer (stationary tile, ring of streamed tiles)
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2-3   idle
-//   warps 4-19  epilogue, two groups of 8 taking alternate tiles; in a group,
-//               warp w reads TMEM lanes 32*(w%4).. and one of two column slabs
+// Warp roles (576 threads, one CTA per SM):
+//   warp 0      TMA producer (stationary tile, ring of NX streamed tiles)
+//   warp 1      TMEM allocator and MMA issuer: an event loop over the logit
+//               MMAs and the gradient MMAs, issued by one elected lane
+//   warps 2-17  epilogue.  Warp w reads TMEM lanes 32*(w%4).. (the quarter its
+//               sub-partition may access) and one column slab of the tile.
+//               Item-owned pass: two groups of 8 take alternate tiles (64-
+//               column slabs); position-owned pass: all 16 take every tile
+//               (32-column slabs).
 //
-// Tensor memory holds NZ fp32 logit buffers, NG bf16 G buffers, the gradient
-// accumulator and, where it fits, a copy of the stationary tile (the logit
-// MMA's A operand, so that only its B operand is read from shared memory).
-// A logit buffer is free again as soon as the epilogue group has loaded it; a
-// G buffer once the gradient MMA that reads it has completed.  With two groups
-// on alternate tiles, each group's next logit tile is computed while it still
-// works on the current one.
+// Tensor memory holds NZ = 3 fp32 logit buffers, the gradient accumulator and,
+// where it fits, a copy of the stationary tile (the logit MMA's A operand, so
+// that only its B operand is read from shared memory).  Each epilogue warp
+// writes its bf16 G slab over the first half of its own, already loaded,
+// logit columns; the gradient MMA reads G from there, and its completion frees
+// the buffer for the logit tile three tiles on.
 //
 // Every wait is bounded (global timer); on expiry the CTA records
 // CUTBCE_ERR_TIMEOUT and where it happened in the workspace header, the other
