@@ -40,6 +40,7 @@ struct WsHeader {
   double loss_scale;   // s
   float grad_scale;    // g * s
   int wait_block;      // CTA of that wait
+  int finish_count;    // blocks of the finish kernel done with their loss slice
 };
 
 // Geometry of the tcgen05 tile engine for one padded feature width DP and G

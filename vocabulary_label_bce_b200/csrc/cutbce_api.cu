@@ -28,6 +28,11 @@ constexpr int64_t kSplitItemsTarget = 16 * 148;        // about 16 dH work items
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Blocks of the finish kernel: one thread per dH element, and at least 256
+// blocks so that the loss partials are summed by many blocks.  Depends only on
+// T and D, so the summation order never depends on the device.
+int64_t finish_grid(int64_t T, int64_t D) { return std::max<int64_t>(256, ceil_div(T * D, kFinishThreads)); }
+
 struct Plan {
   int64_t T, V, D, K;
   int dtype, reduction;
@@ -37,7 +42,7 @@ struct Plan {
   int radix_passes, radix_blocks;
   size_t elem;
   size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_srt[4], o_ghist, o_cscoff, o_hc,
-      o_lpart, o_cpart, o_dhpart, total;
+      o_lpart, o_cpart, o_dhpart, o_fpart, total;
 };
 
 cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
@@ -114,6 +119,7 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.o_lpart = take(8 * kNumEpiWarps * pl.n_vitems);
   pl.o_cpart = take(8 * pl.n_gather_blocks);
   pl.o_dhpart = take(4 * static_cast<size_t>(pl.S) * pl.Tpad * pl.DP);
+  pl.o_fpart = take(16 * static_cast<size_t>(finish_grid(p->T, p->D)));
   pl.total = o;
 }
 
@@ -429,12 +435,12 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     }
   }
   if (w.loss || w.dH) {
-    const int64_t n = w.dH ? static_cast<int64_t>(T) * D : 1;
-    const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n, kFinishThreads)));
+    const unsigned grid = static_cast<unsigned>(finish_grid(T, D));
     LaunchScope ls(CUTBCE_KERNEL_FINISH, st);
     k_finish<<<grid, kFinishThreads, 0, st>>>(T, D, pl.DP, pl.Tpad, pl.S, cidx, dhpart, w.dH ? dH : nullptr, lpart,
                                              static_cast<int>(pl.n_vitems * kNumEpiWarps), cpart,
-                                             static_cast<int>(pl.n_gather_blocks), w.loss ? loss : nullptr, hdr);
+                                             static_cast<int>(pl.n_gather_blocks), at<double>(ws, pl.o_fpart),
+                                             w.loss ? loss : nullptr, hdr);
     CUTBCE_CK(cudaGetLastError());
   }
 #undef CUTBCE_CK

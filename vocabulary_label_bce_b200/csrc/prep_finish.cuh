@@ -209,8 +209,10 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
 
 // ------------------------------------------------------------------ finish
 // dH[t, d] = g*s * sum_{split} partial[split][c(t)][d] in split order (0 for
-// masked rows); the last block also forms loss = s * (dense - correction),
-// both sums taken in a fixed order.
+// masked rows).  The loss = s * (dense - correction) is summed in two levels:
+// every block reduces a fixed slice of the partials, and the last block to
+// finish (an atomic ticket in the workspace header, which each call clears)
+// sums the block results in block order, so the order is fixed.
 constexpr int kFinishThreads = 256;
 
 __device__ double block_sum_fixed(double v, double* red) {
@@ -229,9 +231,10 @@ __device__ double block_sum_fixed(double v, double* red) {
 __global__ void __launch_bounds__(kFinishThreads) k_finish(
     int T, int D, int DP, int64_t Tpad, int S, const int* __restrict__ cidx,
     const float* __restrict__ dh_part, float* __restrict__ dH, const double* __restrict__ loss_part,
-    int n_loss_part, const double* __restrict__ corr_part, int n_corr_part, double* __restrict__ loss,
-    const WsHeader* hdr) {
+    int n_loss_part, const double* __restrict__ corr_part, int n_corr_part, double* __restrict__ blk_part,
+    double* __restrict__ loss, WsHeader* hdr) {
   __shared__ double red[kFinishThreads];
+  __shared__ int ticket;
   const float gs = hdr->grad_scale;
   if (dH != nullptr) {
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -248,15 +251,37 @@ __global__ void __launch_bounds__(kFinishThreads) k_finish(
       dH[idx] = out;
     }
   }
-  if (loss != nullptr && blockIdx.x == gridDim.x - 1) {
+  if (loss != nullptr) {
+    // two levels, both in a fixed order: block b sums slice b of the partials
+    // (coalesced, thread-strided, then a fixed tree), the last block to finish
+    // sums the block results in block order
+    const int nb = static_cast<int>(gridDim.x);
+    const int per_a = (n_loss_part + nb - 1) / nb, per_b = (n_corr_part + nb - 1) / nb;
+    const int a0 = blockIdx.x * per_a, a1 = min(n_loss_part, a0 + per_a);
+    const int b0 = blockIdx.x * per_b, b1 = min(n_corr_part, b0 + per_b);
     double a = 0.0, b = 0.0;
-    const int per_a = (n_loss_part + blockDim.x - 1) / blockDim.x;
-    for (int i = threadIdx.x * per_a; i < min(n_loss_part, (threadIdx.x + 1) * per_a); ++i) a += loss_part[i];
-    const int per_b = (n_corr_part + blockDim.x - 1) / blockDim.x;
-    for (int i = threadIdx.x * per_b; i < min(n_corr_part, (threadIdx.x + 1) * per_b); ++i) b += corr_part[i];
-    const double dense = block_sum_fixed(a, red);
-    const double corr = block_sum_fixed(b, red);
-    if (threadIdx.x == 0) *loss = hdr->n_valid > 0 ? hdr->loss_scale * (dense - corr) : 0.0;
+    for (int i = a0 + threadIdx.x; i < a1; i += blockDim.x) a += loss_part[i];
+    for (int i = b0 + threadIdx.x; i < b1; i += blockDim.x) b += corr_part[i];
+    a = block_sum_fixed(a, red);
+    b = block_sum_fixed(b, red);
+    if (threadIdx.x == 0) {
+      blk_part[2 * blockIdx.x] = a;
+      blk_part[2 * blockIdx.x + 1] = b;
+      __threadfence();
+      ticket = atomicAdd(&hdr->finish_count, 1);
+    }
+    __syncthreads();
+    if (ticket == nb - 1) {
+      __threadfence();
+      double da = 0.0, db = 0.0;
+      for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        da += *reinterpret_cast<volatile double*>(blk_part + 2 * i);
+        db += *reinterpret_cast<volatile double*>(blk_part + 2 * i + 1);
+      }
+      const double dense = block_sum_fixed(da, red);
+      const double corr = block_sum_fixed(db, red);
+      if (threadIdx.x == 0) *loss = hdr->n_valid > 0 ? hdr->loss_scale * (dense - corr) : 0.0;
+    }
   }
 }
 
