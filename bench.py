@@ -174,6 +174,22 @@ def workload_config(p, n_valid, world, l2_note):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
+def reduce_max(x: float, world: int, device) -> float:
+    """The max of x over all ranks (the step time of a replicated run is its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(tokens_per_rank: int, world: int, step_ms_max: float) -> float:
+    """Whole-job throughput: every rank processes its own batch (replicas, weak scaling)."""
+    return world * tokens_per_rank / (step_ms_max * 1e-3)
+
+
 def roofline_times(n_valid, V, D, peaks, clock_mhz):
     f = (clock_mhz or peaks.get("sm_max_mhz", 1965.0)) * 1e6
     flops = 8.0 * n_valid * V * D
@@ -239,11 +255,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     peaks, peaks_src = load_peaks()
     p = W.draw_config(args.workload, seed=0)
@@ -296,7 +308,7 @@ def run_ours(args):
     step_ms_local = statistics.mean(s.elapsed_time(e) for s, e in ev)
     step_ms = max_over_ranks(step_ms_local)
     tokens = p.B * p.N
-    value = world * tokens / (step_ms * 1e-3)
+    value = aggregate_value(tokens, world, step_ms)
 
     # per-kernel durations (events inside the library, same stream)
     avg = {k: (ms / n if n else 0.0) for k, (ms, n) in prof.items()}
