@@ -84,7 +84,8 @@ typedef enum {
 /* Problem statement, after the paper's cut_binary_cross_entropy(activations,
  * embeddings, targets, weights) (section III-C, Listing 1), flattened to T rows. */
 typedef struct {
-  int64_t T;                 /* positions (B*N), >= 1 */
+  int64_t T;                 /* positions (B*N), >= 1; < 2^30, and for bf16 < 2^24 - 127
+                                (the item-owned pass packs a compacted position into 24 bits) */
   int64_t V;                 /* items, >= 1, < 2^31 */
   int64_t D;                 /* feature width, >= 1 */
   int64_t K;                 /* target slots per position, 1..128 */

@@ -54,6 +54,16 @@ def test_host_argument_errors(field, value, expect):
     assert e.value.status == expect
 
 
+def test_bf16_position_limit():
+    # the item-owned pass packs a compacted position into 24 bits
+    assert B.cutbce_workspace_size(_prob(T=(1 << 24) - 128, V=1000, K=1)) > 0
+    with pytest.raises(B.CutBCEError) as e:
+        B.cutbce_workspace_size(_prob(T=(1 << 24) - 127, V=1000, K=1))
+    assert e.value.status == B.ERR_UNSUPPORTED
+    # the fp32 path has no such limit
+    assert B.cutbce_workspace_size(_prob(T=(1 << 24), V=1000, K=1, dtype=B.F32)) > 0
+
+
 def test_compute_calls_reject_before_launch():
     lib = B.load_library()
     p = _prob(T=256, V=1000)

@@ -133,13 +133,6 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, co
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Warp-uniform non-blocking test of a barrier phase (lane 0 tests, the warp shares the answer).
-__device__ __forceinline__ bool test_bar_warp(uint64_t* bar, uint32_t parity) {
-  bool ok = false;
-  if ((threadIdx.x & 31) == 0) ok = mbar_test_wait(bar, parity);
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-}
-
 struct ItemInfo {
   int s_row0;     // first stationary row
   int x_tile0;    // first streamed tile (in units of BN rows)
