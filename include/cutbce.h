@@ -193,11 +193,11 @@ enum {
   CUTBCE_KERNEL_PREP_ROWS = 0,      /* mask and id rules per position */
   CUTBCE_KERNEL_PREP_SCAN = 1,      /* row compaction, pair offsets, scales */
   CUTBCE_KERNEL_PREP_GATHER = 2,    /* compacted H, pair lists, sparse correction */
-  CUTBCE_KERNEL_CSC_OFFSETS = 3,    /* first pair of every item in the item-sorted pairs */
+  CUTBCE_KERNEL_CSC_OFFSETS = 3,    /* first pair of every 128-item tile in the sorted pairs */
   CUTBCE_KERNEL_ITEM_PASS = 4,      /* tensor-core pass owning item tiles: loss and dE */
   CUTBCE_KERNEL_POSITION_PASS = 5,  /* tensor-core pass owning position tiles: dH partials */
   CUTBCE_KERNEL_FINISH = 6,         /* fixed-order dH reduction and the loss */
-  CUTBCE_KERNEL_PAIR_SORT = 7,      /* pairs sorted by (item, position): all radix passes */
+  CUTBCE_KERNEL_PAIR_SORT = 7,      /* pairs grouped by item tile, ascending position: sort keys and all radix passes */
   CUTBCE_NUM_KERNEL_KINDS = 8
 };
 
