@@ -166,7 +166,10 @@ cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes)
  * 256-byte aligned, caller-owned device memory) holds the device copies and the
  * workspace.  The call copies the inputs in, runs cutbce_forward_backward,
  * copies the results out and synchronises `stream`; on return the host outputs
- * are valid and the returned status includes the device status word. */
+ * are valid and the returned status includes the device status word.  dE is
+ * final once the item-owned pass ends, so its copy to the host runs on a second
+ * stream (created and destroyed by the call) while the dH pass still runs on
+ * `stream`; both streams are synchronised before the call returns. */
 cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float grad_loss,
                                            double* loss, float* dH, float* dE,
                                            void* dev_buf, size_t dev_bytes,

@@ -284,8 +284,10 @@ int count_launches(const Plan& pl, Want w) {
   return n;
 }
 
+// after_item: if not null, recorded on `st` right after the item-owned pass,
+// the point from which dE is final.
 cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss, float* dH, float* dE, Want w,
-                  void* ws, size_t ws_bytes, cudaStream_t st) {
+                  void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t after_item = nullptr) {
   cutbce_status s = check_problem(p, true);
   if (s != CUTBCE_OK) return s;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return CUTBCE_ERR_INVALID_ARG;
@@ -408,6 +410,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
       else e = launch_tile_dp<false, true, false>(pl.DP, grid, ms, mx, tp, st);
       CUTBCE_CK(e);
     }
+    if (item_pass && after_item != nullptr) CUTBCE_CK(cudaEventRecord(after_item, st));
     if (w.dH) {
       CUtensorMap ms, mx;
       if (!make_map(&ms, hc, pl.DP, pl.Tpad, pl.DP, kTileM) || !make_map(&mx, p->E, D, V, D, pl.BN))
@@ -427,6 +430,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
           w.loss ? lpart : nullptr);
       CUTBCE_CK(cudaGetLastError());
     }
+    if (item_pass && after_item != nullptr) CUTBCE_CK(cudaEventRecord(after_item, st));
     if (w.dH) {
       LaunchScope ls(CUTBCE_KERNEL_POSITION_PASS, st);
       k_simt_rows<<<static_cast<unsigned>(ceil_div(pl.Tpad, 128)), 128, 0, st>>>(
@@ -587,16 +591,40 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   dp.mask = prob->mask != nullptr ? reinterpret_cast<const uint8_t*>(b + hl.o_mask) : nullptr;
   float* ddH = dH ? reinterpret_cast<float*>(b + hl.o_dH) : nullptr;
   float* ddE = dE ? reinterpret_cast<float*>(b + hl.o_dE) : nullptr;
+  // dE is final once the item-owned pass ends: its copy to the host runs on a
+  // second stream while the position-owned pass and the finish run on `st`.
+  cudaStream_t s2 = nullptr;
+  cudaEvent_t item_done = nullptr;
+  if (dE != nullptr) {
+    if (cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking) != cudaSuccess) return CUTBCE_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&item_done, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(s2);
+      return CUTBCE_ERR_CUDA;
+    }
+  }
+  auto release = [&]() {
+    if (item_done != nullptr) cudaEventDestroy(item_done);
+    if (s2 != nullptr) cudaStreamDestroy(s2);
+  };
   s = run(&dp, reinterpret_cast<const float*>(b + hl.o_grad), reinterpret_cast<double*>(b + hl.o_loss), ddH, ddE,
-          Want{true, dE != nullptr, dH != nullptr}, b + hl.o_ws, pl.total, st);
-  if (s != CUTBCE_OK) return s;
+          Want{true, dE != nullptr, dH != nullptr}, b + hl.o_ws, pl.total, st, item_done);
+  if (s != CUTBCE_OK) {
+    if (s2 != nullptr) cudaStreamSynchronize(st);   // nothing may still use the buffers on return
+    release();
+    return s;
+  }
   int dev_status = 0;
-  if (cudaMemcpyAsync(loss, b + hl.o_loss, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      (dH && cudaMemcpyAsync(dH, ddH, 4 * prob->T * prob->D, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
-      (dE && cudaMemcpyAsync(dE, ddE, 4 * prob->V * prob->D, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
-      cudaMemcpyAsync(&dev_status, b + hl.o_ws + pl.o_hdr, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return CUTBCE_ERR_CUDA;
+  bool ok = true;
+  if (dE != nullptr)
+    ok = cudaStreamWaitEvent(s2, item_done, 0) == cudaSuccess &&
+         cudaMemcpyAsync(dE, ddE, 4 * prob->V * prob->D, cudaMemcpyDeviceToHost, s2) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(loss, b + hl.o_loss, 8, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
+       (!dH || cudaMemcpyAsync(dH, ddH, 4 * prob->T * prob->D, cudaMemcpyDeviceToHost, st) == cudaSuccess) &&
+       cudaMemcpyAsync(&dev_status, b + hl.o_ws + pl.o_hdr, 4, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+  // both streams are drained before returning, also after an error
+  const bool sync_ok = cudaStreamSynchronize(st) == cudaSuccess && (s2 == nullptr || cudaStreamSynchronize(s2) == cudaSuccess);
+  release();
+  if (!ok || !sync_ok) return CUTBCE_ERR_CUDA;
   return static_cast<cutbce_status>(dev_status);
 }
 
