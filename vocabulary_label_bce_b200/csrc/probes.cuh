@@ -68,9 +68,15 @@ __global__ void __launch_bounds__(kProbeThreads, 1) k_probe(int iters, unsigned 
       if (OP == kProbeTanh) a[k] = tanh_approx(a[k]);                // stays in (-1, 1)
       if (OP == kProbeLg2) a[k] = lg2_approx(a[k] + 2.0f);           // stays in [1, 2]
       if (OP == kProbeCvtBf16x2) a[k] = __uint_as_float(pack_bf16x2(a[k], a[k]));
-      if (OP == kProbeFmax) a[k] = fmaxf(a[k], 0.5f);
+      if (OP == kProbeFmax) {                                        // asm: the chain must not fold
+        asm volatile("max.f32 %0, %0, %1;" : "+f"(a[k]) : "f"(0.5f));
+      }
       if (OP == kProbeAdd2) a2[k] = fadd2(a2[k], c2);
-      if (OP == kProbeIadd) a[k] = __uint_as_float(__float_as_uint(a[k]) + 0x101u);
+      if (OP == kProbeIadd) {
+        uint32_t v = __float_as_uint(a[k]);
+        asm volatile("add.s32 %0, %0, 257;" : "+r"(v));
+        a[k] = __uint_as_float(v);
+      }
       if (OP == kProbePrmt) a[k] = __uint_as_float(__byte_perm(__float_as_uint(a[k]), 0x12345678u, 0x3726u));
     }
   }
