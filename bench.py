@@ -170,6 +170,8 @@ def blas_threads():
 
 def workload_config(p, n_valid, world, l2_note):
     return {"workload": p.name, "B": p.B, "N": p.N, "T": p.T, "n_valid": n_valid, "V": p.V, "D": p.D, "K": p.K,
+            "tokens": "value counts all B*N positions per step, padding included; valid_tokens_per_s counts "
+                      "the n_valid positions that carry work",
             "inputs": "bf16 H, E; int32 targets; uint8 mask", "seed": 0, "l2": l2_note,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
@@ -190,11 +192,27 @@ def aggregate_value(tokens_per_rank: int, world: int, step_ms_max: float) -> flo
     return world * tokens_per_rank / (step_ms_max * 1e-3)
 
 
-def roofline_times(n_valid, V, D, peaks, clock_mhz):
-    f = (clock_mhz or peaks.get("sm_max_mhz", 1965.0)) * 1e6
+DATASHEET_BF16_TFLOPS = 2250.0   # B200 dense bf16, nominal
+
+
+def probe_rates():
+    """SFU exponential and FMA-pipe rates (operations per clock per SM), measured live
+    by the library's own pipe probes on this GPU (median over SMs)."""
+    from vocabulary_label_bce_b200 import binding as B
+    return {"ex2": B.cutbce_probe_pipe_rate("ex2"), "ffma": B.cutbce_probe_pipe_rate("ffma"),
+            "ffma2": B.cutbce_probe_pipe_rate("ffma2")}
+
+
+def roofline_times(n_valid, V, D, peaks, rates, sms=148):
+    """Path roofline: the slower of the tensor-core time of 8*T*V*D FLOP at the
+    measured bf16 peak, and the time of T*V transcendental evaluations at the
+    SFU rate plus the FMA-pipe rate divided by the 8 FMA-pipe operations of one
+    polynomial exponential (rates per clock per SM from the live probes, at the
+    maximum SM clock)."""
+    f = peaks.get("sm_max_mhz", 1965.0) * 1e6
     flops = 8.0 * n_valid * V * D
     t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
-    r_mufu, r_fma = 16 * 148 * f, 128 * 148 * f
+    r_mufu, r_fma = rates["ex2"] * sms * f, rates["ffma"] * sms * f
     t_alu = n_valid * V / (r_mufu + r_fma / 8)
     return flops, t_tensor, t_alu
 
@@ -258,6 +276,8 @@ def run_ours(args):
         return reduce_max(x, world, dev)
 
     peaks, peaks_src = load_peaks()
+    rates = probe_rates()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     p = W.draw_config(args.workload, seed=0)
     H = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).to(dev)
     E = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -314,7 +334,7 @@ def run_ours(args):
     avg = {k: (ms / n if n else 0.0) for k, (ms, n) in prof.items()}
     dominant = max(("item_pass", "position_pass"), key=lambda k: avg[k])
     kern_ms = max_over_ranks(avg[dominant])
-    flops_path, t_tensor, t_alu = roofline_times(n_valid, p.V, p.D, peaks, None)
+    flops_path, t_tensor, t_alu = roofline_times(n_valid, p.V, p.D, peaks, rates, sms)
     kernel_flops = 4.0 * n_valid * p.V * p.D
     achieved = kernel_flops / (kern_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
@@ -377,9 +397,13 @@ def run_ours(args):
                          "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
                          "kernel_ms": kern_ms, "algorithmic_flops_per_launch": kernel_flops,
                          "peak_source": f"{peaks_src} bf16_tflops (burst)",
-                         "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak)},
+                         "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
+                         "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
             "path_roofline": {"flops": flops_path, "t_tensor_ms": t_tensor * 1e3, "t_alu_ms": t_alu * 1e3,
-                              "t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / step_ms},
+                              "t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / step_ms,
+                              "note": "headline fraction of the whole step: t_roof / measured step time; "
+                                      "t_alu from the live SFU (ex2) and FMA probe rates",
+                              "probe_rates_per_clk_per_sm": rates, "sms": sms},
             "kernels_ms": {k: round(v, 4) for k, v in avg.items()},
             "n_pairs": n_pairs,
             "gpu_launches": args.steps * B.cutbce_kernel_launches(prob, 2),

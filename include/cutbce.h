@@ -97,15 +97,27 @@ typedef struct {
   const uint8_t* mask;       /* [T] 1 = valid, or NULL = all valid (device) */
 } cutbce_problem;
 
-/* Bytes of device workspace that a compute call on this problem needs.  The
+/* Bytes of device workspace that a compute call on this problem needs, for
+ * every set of outputs (loss, dH and dE): enough for any compute call.  The
  * size has no T*V term: it is O(T*K + S*T*D + V) for a split count S <= 64
  * chosen from T.  Host-only; launches nothing.  Returns INVALID_ARG or
  * UNSUPPORTED for a problem the compute calls would reject. */
 cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes);
 
+/* Outputs of a compute call, as bits of `outputs` below. */
+enum { CUTBCE_OUT_LOSS = 1, CUTBCE_OUT_DH = 2, CUTBCE_OUT_DE = 4 };
+
+/* Bytes of device workspace for a call that computes only the given outputs
+ * (a bitwise or of CUTBCE_OUT_*): cutbce_forward needs CUTBCE_OUT_LOSS;
+ * cutbce_backward and cutbce_forward_backward need the bits of the outputs
+ * they are given non-NULL.  The dH split partials (O(S*T*D)) are counted only
+ * with CUTBCE_OUT_DH, and the pair-sort buffers (O(T*K)) only with
+ * CUTBCE_OUT_DE, so a loss-only workspace is O(T*K + T*D + V).  Host-only. */
+cutbce_status cutbce_workspace_size_for(const cutbce_problem* prob, int outputs, size_t* bytes);
+
 /* Loss only (section III-A).  loss: device double, written with the
- * normalised loss.  ws: device workspace of ws_bytes bytes (>= workspace size),
- * 256-byte aligned. */
+ * normalised loss.  ws: device workspace of ws_bytes bytes
+ * (>= cutbce_workspace_size_for(prob, CUTBCE_OUT_LOSS)), 256-byte aligned. */
 cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_bytes,
                              double* loss, cutbce_stream_t stream);
 
@@ -122,9 +134,12 @@ cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_byt
  * not grow it, or a host runtime with no device allocator of its own, where a
  * cudaMalloc would also stall the device until pending work drains.
  *
- * Limit: problems with cutbce_workspace_size() > CUTBCE_FIXED_SCRATCH_BYTES
- * are rejected with CUTBCE_ERR_WORKSPACE before anything is launched (the
- * workspace grows with T*K, S*T*D and V; small and medium problems fit).
+ * Limit: problems with cutbce_workspace_size_for(prob, CUTBCE_OUT_LOSS) >
+ * CUTBCE_FIXED_SCRATCH_BYTES are rejected with CUTBCE_ERR_WORKSPACE before
+ * anything is launched.  That loss-only workspace is about
+ * 16 T K + 2 T D' + 16 * 8 * ceil(V / 128) bytes (D' = D rounded up to 64), so
+ * for example T = 12,800 positions with K = 16 slots, D = 64 and V = 876,000
+ * items (about 6 MB) fits.
  * Setup: the first call on each device, with that device current, looks up
  * the device address of the array (cudaGetSymbolAddress) and caches it; that
  * lookup may load the library's device code on the device, so make the first
@@ -145,7 +160,8 @@ cutbce_status cutbce_forward_fixed_scratch(const cutbce_problem* prob, double* l
 
 /* Gradients only (section III-B, Eq. (4)), recomputing the logits.
  * grad_loss: device float scalar g, or NULL for g = 1.
- * dH: device float [T, D]; dE: device float [V, D]; either may be NULL to skip it. */
+ * dH: device float [T, D]; dE: device float [V, D]; either may be NULL to skip it.
+ * ws: >= cutbce_workspace_size_for(prob, outputs given) bytes, 256-byte aligned. */
 cutbce_status cutbce_backward(const cutbce_problem* prob, const float* grad_loss,
                               float* dH, float* dE, void* ws, size_t ws_bytes,
                               cutbce_stream_t stream);
@@ -168,8 +184,10 @@ cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes)
  * copies the results out and synchronises `stream`; on return the host outputs
  * are valid and the returned status includes the device status word.  dE is
  * final once the item-owned pass ends, so its copy to the host runs on a second
- * stream (created and destroyed by the call) while the dH pass still runs on
- * `stream`; both streams are synchronised before the call returns. */
+ * stream while the dH pass still runs on `stream`; both streams are
+ * synchronised before the call returns.  That second stream and its event are
+ * created by the first such calls on a device and kept in a per-device pool for
+ * the rest of the process (one pair per call in flight). */
 cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float grad_loss,
                                            double* loss, float* dH, float* dE,
                                            void* dev_buf, size_t dev_bytes,
@@ -228,7 +246,16 @@ enum {
   CUTBCE_PROBE_ADD2 = 8,    /* add.rn.f32x2, counted as two operations */
   CUTBCE_PROBE_IADD = 9,    /* add.s32 */
   CUTBCE_PROBE_PRMT = 10,   /* prmt.b32 */
-  CUTBCE_NUM_PROBES = 11
+  CUTBCE_PROBE_EX2_F16X2 = 11,   /* ex2.approx.f16x2 (two 16-bit results), counted per instruction */
+  CUTBCE_PROBE_EX2_BF16X2 = 12,  /* ex2.approx.ftz.bf16x2, counted per instruction */
+  CUTBCE_PROBE_TANH_F16X2 = 13,  /* tanh.approx.f16x2, counted per instruction */
+  CUTBCE_PROBE_HFMA2 = 14,       /* fma.rn.f16x2, counted per instruction */
+  CUTBCE_PROBE_CVT_F16X2 = 15,   /* cvt.rn.f16x2.f32, counted per instruction */
+  CUTBCE_PROBE_FFMA_SAT = 16,    /* fma.rn.sat.f32 */
+  CUTBCE_PROBE_SELECT = 17,      /* setp.ge.f32 + selp.f32, counted per select */
+  CUTBCE_PROBE_LOP = 18,         /* and.b32 */
+  CUTBCE_PROBE_FMUL2 = 19,       /* mul.rn.f32x2, counted as two operations */
+  CUTBCE_NUM_PROBES = 20
 };
 
 /* Bytes of device scratch cutbce_probe_pipe_rate needs. */

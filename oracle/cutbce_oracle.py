@@ -202,10 +202,16 @@ def dE_rows(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np
     rows = np.nonzero(tg.valid)[0]
     Hv = H64[rows]
     s = scale_factor(reduction, len(rows), V)
+    # the valid rows (indices into rows) that hold each positive item
+    holders: dict = {}
+    for r, t in enumerate(rows):
+        for v in tg.sets[t].tolist():
+            holders.setdefault(v, []).append(r)
     out = np.zeros((len(items), H64.shape[1]), dtype=np.float64)
     for i, v in enumerate(items):
         z = Hv @ np.asarray(E[v], dtype=np.float64)
-        y = np.array([1.0 if np.any(tg.sets[t] == v) else 0.0 for t in rows])
+        y = np.zeros(len(rows), dtype=np.float64)
+        y[holders.get(int(v), [])] = 1.0
         out[i] = grad_loss * s * ((sigmoid(z) - y) @ Hv)
     return out
 

@@ -68,7 +68,7 @@ def test_compute_calls_reject_before_launch():
     lib = B.load_library()
     p = _prob(T=256, V=1000)
     n = ctypes.c_size_t()
-    assert lib.cutbce_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    assert lib.cutbce_workspace_size_for(ctypes.byref(p), B.OUT_LOSS, ctypes.byref(n)) == 0
     loss = ctypes.c_void_p(0x20000)
     # null workspace, small workspace, misaligned workspace, null loss, null problem pointers
     assert lib.cutbce_forward(ctypes.byref(p), None, n.value, loss, None) == B.ERR_INVALID_ARG
@@ -85,6 +85,23 @@ def test_compute_calls_reject_before_launch():
     assert lib.cutbce_backward(ctypes.byref(p), None, None, None, ctypes.c_void_p(0x40000), n.value,
                                None) == B.ERR_INVALID_ARG
     assert lib.cutbce_selftest_wait_timeout(0, ctypes.c_void_p(0x40000), None) == B.ERR_INVALID_ARG
+
+
+def test_workspace_size_per_outputs():
+    p = _prob()
+    full = B.cutbce_workspace_size(p)
+    assert full == B.cutbce_workspace_size_for(p, B.OUT_LOSS | B.OUT_DH | B.OUT_DE)
+    loss_only = B.cutbce_workspace_size_for(p, B.OUT_LOSS)
+    dh = B.cutbce_workspace_size_for(p, B.OUT_DH)
+    de = B.cutbce_workspace_size_for(p, B.OUT_DE)
+    assert loss_only < dh < full and loss_only < de < full
+    # the loss-only layout holds neither the dH split partials nor the pair-sort buffers
+    assert full - loss_only >= 16 * 12800 * 16 + 4 * 12800 * 64
+    assert loss_only < 16 << 20
+    for bad in (0, 8, -1):
+        with pytest.raises(B.CutBCEError) as e:
+            B.cutbce_workspace_size_for(p, bad)
+        assert e.value.status == B.ERR_INVALID_ARG
 
 
 def test_launch_accounting():

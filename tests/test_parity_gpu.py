@@ -180,3 +180,43 @@ def test_autograd_wrapper():
     assert rel_fro(Hb.grad.float().cpu().numpy(), ref.dH) < GRAD_RTOL + 4e-3   # bf16 output rounding
     assert rel_fro(Eb.grad.float().cpu().numpy(), ref.dE) < GRAD_RTOL + 4e-3
     del Hf, Ef
+
+
+@pytest.mark.parametrize("outputs", ["loss", "dH", "dE", "all"])
+def test_canary_guards_untouched(outputs):
+    # a tiny, unaligned case (T and V not multiples of a tile, D padded to 64):
+    # every byte past the workspace the call asked for, and past the [T, D] and
+    # [V, D] outputs, must keep its canary value
+    p = W.draw(T=65, V=2047, D=40, K=3, dtype="bf16", seed=14, ids="zipf", mask="random", mask_frac=0.1)
+    H, E, tg, m = to_device(p)
+    prob = B.make_problem(H, E, tg, m, "mean")
+    bits = {"loss": B.OUT_LOSS, "dH": B.OUT_DH, "dE": B.OUT_DE, "all": B.OUT_LOSS | B.OUT_DH | B.OUT_DE}[outputs]
+    n = B.cutbce_workspace_size_for(prob, bits)
+    guard = 64 << 10
+    ws_all = torch.full((n + guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    dH_all = torch.full((p.T * p.D + guard // 4,), 12345.0, dtype=torch.float32, device="cuda")
+    dE_all = torch.full((p.V * p.D + guard // 4,), 12345.0, dtype=torch.float32, device="cuda")
+    loss = torch.full((), float("nan"), dtype=torch.float64, device="cuda")
+    dH = dH_all[:p.T * p.D].view(p.T, p.D) if bits & B.OUT_DH else None
+    dE = dE_all[:p.V * p.D].view(p.V, p.D) if bits & B.OUT_DE else None
+    ws = ws_all[:n]
+    if bits == B.OUT_LOSS:
+        B.cutbce_forward(prob, ws, loss)
+    elif not bits & B.OUT_LOSS:
+        B.cutbce_backward(prob, None, dH, dE, ws)
+    else:
+        B.cutbce_forward_backward(prob, None, loss, dH, dE, ws)
+    assert B.cutbce_read_status(ws) == 0
+    torch.cuda.synchronize()
+    assert bool(torch.all(ws_all[n:] == 0xA5)), "workspace guard overwritten"
+    assert bool(torch.all(dH_all[p.T * p.D:] == 12345.0)), "dH guard overwritten"
+    assert bool(torch.all(dE_all[p.V * p.D:] == 12345.0)), "dE guard overwritten"
+    if dH is None:
+        assert bool(torch.all(dH_all == 12345.0)), "dH written although not asked for"
+    if dE is None:
+        assert bool(torch.all(dE_all == 12345.0)), "dE written although not asked for"
+    got = {"status": 0, "prob": prob, "ws": ws,
+           "loss": float(loss.item()) if bits & B.OUT_LOSS else None,
+           "dH": dH.cpu().numpy().astype(np.float64) if dH is not None else None,
+           "dE": dE.cpu().numpy().astype(np.float64) if dE is not None else None}
+    check_against_oracle(p, got, "mean")

@@ -56,7 +56,8 @@ def forward_backward(H: torch.Tensor, E: torch.Tensor, targets: torch.Tensor, ma
     H2, tg, m = _flat(H, targets, mask)
     E = E.contiguous()
     prob = B.make_problem(H2, E, tg, m, reduction)
-    ws = workspace if workspace is not None else _WS.get(B.cutbce_workspace_size(prob), H2.device)
+    outs = (B.OUT_LOSS if want_loss else 0) | (B.OUT_DH if want_dH else 0) | (B.OUT_DE if want_dE else 0)
+    ws = workspace if workspace is not None else _WS.get(B.cutbce_workspace_size_for(prob, outs), H2.device)
     loss = torch.empty((), dtype=torch.float64, device=H2.device) if want_loss else None
     dH = torch.empty(H2.shape, dtype=torch.float32, device=H2.device) if want_dH else None
     dE = torch.empty(E.shape, dtype=torch.float32, device=E.device) if want_dE else None
@@ -71,7 +72,7 @@ def forward(H, E, targets, mask=None, reduction: str = "mean", workspace=None) -
     H2, tg, m = _flat(H, targets, mask)
     E = E.contiguous()
     prob = B.make_problem(H2, E, tg, m, reduction)
-    ws = workspace if workspace is not None else _WS.get(B.cutbce_workspace_size(prob), H2.device)
+    ws = workspace if workspace is not None else _WS.get(B.cutbce_workspace_size_for(prob, B.OUT_LOSS), H2.device)
     loss = torch.empty((), dtype=torch.float64, device=H2.device)
     B.cutbce_forward(prob, ws, loss)
     return loss
@@ -82,7 +83,8 @@ def backward(H, E, targets, mask=None, reduction: str = "mean", grad_loss=None, 
     H2, tg, m = _flat(H, targets, mask)
     E = E.contiguous()
     prob = B.make_problem(H2, E, tg, m, reduction)
-    ws = workspace if workspace is not None else _WS.get(B.cutbce_workspace_size(prob), H2.device)
+    outs = (B.OUT_DH if want_dH else 0) | (B.OUT_DE if want_dE else 0)
+    ws = workspace if workspace is not None else _WS.get(B.cutbce_workspace_size_for(prob, outs), H2.device)
     dH = torch.empty(H2.shape, dtype=torch.float32, device=H2.device) if want_dH else None
     dE = torch.empty(E.shape, dtype=torch.float32, device=E.device) if want_dE else None
     g = grad_loss.to(torch.float32).reshape(()) if grad_loss is not None else None

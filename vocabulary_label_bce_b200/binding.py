@@ -17,7 +17,7 @@ import torch
 
 __all__ = [
     "CutBCEError", "cutbce_problem", "load_library", "library_path", "declared_functions",
-    "cutbce_workspace_size", "cutbce_forward", "cutbce_forward_fixed_scratch", "FIXED_SCRATCH_BYTES",
+    "cutbce_workspace_size", "cutbce_workspace_size_for", "OUT_LOSS", "OUT_DH", "OUT_DE", "cutbce_forward", "cutbce_forward_fixed_scratch", "FIXED_SCRATCH_BYTES",
     "cutbce_backward", "cutbce_forward_backward",
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
@@ -27,6 +27,7 @@ __all__ = [
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TARGET_RANGE, ERR_TIMEOUT, ERR_CUDA = range(7)
 BF16, F32 = 0, 1
+OUT_LOSS, OUT_DH, OUT_DE = 1, 2, 4
 REDUCTIONS = {"mean": 0, "sum": 1, "mean_elements": 2}
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -57,6 +58,7 @@ _P = ctypes.POINTER(cutbce_problem)
 _vp, _sz, _i32, _i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
 _SIGS = {
     "cutbce_workspace_size": (_i32, [_P, ctypes.POINTER(_sz)]),
+    "cutbce_workspace_size_for": (_i32, [_P, ctypes.c_int, ctypes.POINTER(_sz)]),
     "cutbce_forward": (_i32, [_P, _vp, _sz, _vp, _vp]),
     "cutbce_forward_fixed_scratch": (_i32, [_P, _vp, _vp]),
     "cutbce_backward": (_i32, [_P, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -75,7 +77,8 @@ _SIGS = {
     "cutbce_probe_mma": (_i32, [ctypes.c_int, ctypes.c_int, _i64, _vp, _sz, ctypes.POINTER(ctypes.c_double),
                                 ctypes.POINTER(ctypes.c_double), _vp]),
 }
-PROBES = ["ffma", "ffma2", "ex2", "rcp", "tanh", "lg2", "cvt_bf16x2", "fmax", "add2", "iadd", "prmt"]
+PROBES = ["ffma", "ffma2", "ex2", "rcp", "tanh", "lg2", "cvt_bf16x2", "fmax", "add2", "iadd", "prmt",
+          "ex2_f16x2", "ex2_bf16x2", "tanh_f16x2", "hfma2", "cvt_f16x2", "ffma_sat", "select", "lop", "fmul2"]
 KERNEL_KINDS = ["prep_rows", "prep_scan", "prep_gather", "csc_offsets", "item_pass", "position_pass", "finish",
                 "pair_sort"]
 
@@ -139,6 +142,14 @@ def make_problem(H: torch.Tensor, E: torch.Tensor, targets: torch.Tensor, mask: 
 def cutbce_workspace_size(prob: cutbce_problem) -> int:
     n = _sz(0)
     _check(load_library().cutbce_workspace_size(ctypes.byref(prob), ctypes.byref(n)), "cutbce_workspace_size")
+    return int(n.value)
+
+
+def cutbce_workspace_size_for(prob: cutbce_problem, outputs: int) -> int:
+    """Workspace bytes for a call computing only `outputs` (a bitwise or of OUT_LOSS, OUT_DH, OUT_DE)."""
+    n = _sz(0)
+    _check(load_library().cutbce_workspace_size_for(ctypes.byref(prob), int(outputs), ctypes.byref(n)),
+           "cutbce_workspace_size_for")
     return int(n.value)
 
 

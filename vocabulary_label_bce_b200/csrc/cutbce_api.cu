@@ -7,6 +7,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -32,6 +33,16 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // blocks so that the loss partials are summed by many blocks.  Depends only on
 // T and D, so the summation order never depends on the device.
 int64_t finish_grid(int64_t T, int64_t D) { return std::max<int64_t>(256, ceil_div(T * D, kFinishThreads)); }
+
+// Outputs one call computes; the workspace plan holds only what they need.
+struct Want {
+  bool loss, dE, dH;
+};
+constexpr Want kWantAll{true, true, true};
+
+Want want_from_mask(int outputs) {
+  return Want{(outputs & CUTBCE_OUT_LOSS) != 0, (outputs & CUTBCE_OUT_DE) != 0, (outputs & CUTBCE_OUT_DH) != 0};
+}
 
 struct Plan {
   int64_t T, V, D, K;
@@ -65,7 +76,11 @@ cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
   return CUTBCE_OK;
 }
 
-void make_plan(const cutbce_problem* p, Plan& pl) {
+// Workspace layout.  The header and the per-position arrays come first, at the
+// same offsets for every set of outputs (cutbce_read_status and
+// cutbce_read_counts rely on that); the pair-sort buffers (dE only) and the dH
+// split partials (dH only) are laid out only when those outputs are wanted.
+void make_plan(const cutbce_problem* p, Want w, Plan& pl) {
   pl.T = p->T;
   pl.V = p->V;
   pl.D = p->D;
@@ -112,14 +127,15 @@ void make_plan(const cutbce_problem* p, Plan& pl) {
   pl.o_ids = take(4 * TK);
   pl.o_pair_t = take(4 * TK);
   pl.o_pair_v = take(4 * TK);
-  for (int k = 0; k < 4; ++k) pl.o_srt[k] = take(4 * TK);
-  pl.o_ghist = take(4 * 256 * static_cast<size_t>(pl.radix_blocks));
-  pl.o_cscoff = take(4 * static_cast<size_t>(pl.n_vitems + 1));
   pl.o_hc = take(pl.elem * static_cast<size_t>(pl.Tpad) * pl.DP);
   pl.o_lpart = take(8 * kNumEpiWarps * pl.n_vitems);
   pl.o_cpart = take(8 * pl.n_gather_blocks);
-  pl.o_dhpart = take(4 * static_cast<size_t>(pl.S) * pl.Tpad * pl.DP);
   pl.o_fpart = take(16 * static_cast<size_t>(finish_grid(p->T, p->D)));
+  const bool sort = bf16 && w.dE;
+  for (int k = 0; k < 4; ++k) pl.o_srt[k] = sort ? take(4 * TK) : 0;
+  pl.o_ghist = sort ? take(4 * 256 * static_cast<size_t>(pl.radix_blocks)) : 0;
+  pl.o_cscoff = sort ? take(4 * static_cast<size_t>(pl.n_vitems + 1)) : 0;
+  pl.o_dhpart = w.dH ? take(4 * static_cast<size_t>(pl.S) * pl.Tpad * pl.DP) : 0;
   pl.total = o;
 }
 
@@ -248,11 +264,17 @@ cudaError_t launch_tile(int grid, const CUtensorMap& s, const CUtensorMap& x, co
                         cudaStream_t st) {
   auto kern = k_tile<DP, kLoss, kGrad, kDH>;
   constexpr uint32_t smem = TileCfg<DP, epi_groups<kDH>()>::SMEM_BYTES;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // the attribute belongs to the current device: set it once per device
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = uint64_t(1) << dev;
+  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   kern<<<grid, kTileThreads, smem, st>>>(s, x, tp);
   return cudaGetLastError();
@@ -269,10 +291,6 @@ cudaError_t launch_tile_dp(int DP, int grid, const CUtensorMap& s, const CUtenso
     default: return cudaErrorInvalidValue;
   }
 }
-
-struct Want {
-  bool loss, dE, dH;
-};
 
 int count_launches(const Plan& pl, Want w) {
   const bool bf16 = pl.dtype == CUTBCE_BF16;
@@ -293,7 +311,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return CUTBCE_ERR_INVALID_ARG;
   if (w.loss && loss == nullptr) return CUTBCE_ERR_INVALID_ARG;
   Plan pl;
-  make_plan(p, pl);
+  make_plan(p, w, pl);
   if (ws_bytes < pl.total) return CUTBCE_ERR_WORKSPACE;
   DeviceFacts dev;
   if ((s = device_facts(dev)) != CUTBCE_OK) return s;
@@ -475,6 +493,46 @@ void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
   hl.total = o;
 }
 
+// ---------------------------------------------------------------- host-entry side streams
+// The host-buffer entry copies dE out on a second stream, ordered after the
+// item-owned pass by an event.  Streams and events are created once per device
+// and pooled: each call takes one pair for its duration, so concurrent calls
+// never share an event.
+struct SideStream {
+  int dev;
+  cudaStream_t s;
+  cudaEvent_t ev;
+};
+std::mutex g_side_mu;
+std::vector<SideStream> g_side_free;
+
+cutbce_status take_side_stream(SideStream& out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CUTBCE_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    for (size_t i = 0; i < g_side_free.size(); ++i) {
+      if (g_side_free[i].dev == dev) {
+        out = g_side_free[i];
+        g_side_free.erase(g_side_free.begin() + static_cast<std::ptrdiff_t>(i));
+        return CUTBCE_OK;
+      }
+    }
+  }
+  out.dev = dev;
+  if (cudaStreamCreateWithFlags(&out.s, cudaStreamNonBlocking) != cudaSuccess) return CUTBCE_ERR_CUDA;
+  if (cudaEventCreateWithFlags(&out.ev, cudaEventDisableTiming) != cudaSuccess) {
+    cudaStreamDestroy(out.s);
+    return CUTBCE_ERR_CUDA;
+  }
+  return CUTBCE_OK;
+}
+
+void give_side_stream(const SideStream& s) {
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  g_side_free.push_back(s);
+}
+
 // ---------------------------------------------------------------- fixed scratch
 // Scratch of cutbce_forward_fixed_scratch: a static device array of the
 // library's own module, so that entry needs no caller workspace and allocates
@@ -507,11 +565,16 @@ cutbce_status fixed_scratch_ptr(void** out) {
 extern "C" {
 
 cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes) {
-  if (bytes == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  return cutbce_workspace_size_for(prob, CUTBCE_OUT_LOSS | CUTBCE_OUT_DH | CUTBCE_OUT_DE, bytes);
+}
+
+cutbce_status cutbce_workspace_size_for(const cutbce_problem* prob, int outputs, size_t* bytes) {
+  if (bytes == nullptr || outputs <= 0 || outputs > (CUTBCE_OUT_LOSS | CUTBCE_OUT_DH | CUTBCE_OUT_DE))
+    return CUTBCE_ERR_INVALID_ARG;
   const cutbce_status s = check_problem(prob, false);
   if (s != CUTBCE_OK) return s;
   Plan pl;
-  make_plan(prob, pl);
+  make_plan(prob, want_from_mask(outputs), pl);
   *bytes = pl.total;
   return CUTBCE_OK;
 }
@@ -528,7 +591,7 @@ cutbce_status cutbce_forward_fixed_scratch(const cutbce_problem* prob, double* l
   cutbce_status s = check_problem(prob, true);
   if (s != CUTBCE_OK) return s;
   Plan pl;
-  make_plan(prob, pl);
+  make_plan(prob, Want{true, false, false}, pl);                   // the loss-only layout that run() uses
   if (pl.total > kFixedScratchBytes) return CUTBCE_ERR_WORKSPACE;   // the problem needs more than the fixed array
   void* ws = nullptr;
   if ((s = fixed_scratch_ptr(&ws)) != CUTBCE_OK) return s;
@@ -555,7 +618,7 @@ cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes)
   const cutbce_status s = check_problem(prob, false);
   if (s != CUTBCE_OK) return s;
   Plan pl;
-  make_plan(prob, pl);
+  make_plan(prob, kWantAll, pl);
   HostLayout hl;
   host_layout(prob, pl, hl);
   *bytes = hl.total;
@@ -569,21 +632,25 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   if (loss == nullptr || dev_buf == nullptr || (reinterpret_cast<uintptr_t>(dev_buf) & 255) != 0)
     return CUTBCE_ERR_INVALID_ARG;
   Plan pl;
-  make_plan(prob, pl);
+  make_plan(prob, kWantAll, pl);     // the largest layout: the buffer size query covers every set of outputs
   HostLayout hl;
   host_layout(prob, pl, hl);
   if (dev_bytes < hl.total) return CUTBCE_ERR_WORKSPACE;
+  // dE is final once the item-owned pass ends: its copy to the host runs on a
+  // second stream while the position-owned pass and the finish run on `st`.
+  // The stream and its event come from a per-device pool (created on first use).
+  SideStream side{};
+  if (dE != nullptr && (s = take_side_stream(side)) != CUTBCE_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* b = static_cast<uint8_t*>(dev_buf);
   const size_t szH = pl.elem * prob->T * prob->D, szE = pl.elem * prob->V * prob->D;
-  if (cudaMemcpyAsync(b + hl.o_H, prob->H, szH, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(b + hl.o_E, prob->E, szE, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(b + hl.o_tg, prob->targets, 4 * prob->T * prob->K, cudaMemcpyHostToDevice, st) !=
-          cudaSuccess ||
-      (prob->mask != nullptr &&
-       cudaMemcpyAsync(b + hl.o_mask, prob->mask, prob->T, cudaMemcpyHostToDevice, st) != cudaSuccess) ||
-      cudaMemcpyAsync(b + hl.o_grad, &grad_loss, 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return CUTBCE_ERR_CUDA;
+  bool copied = cudaMemcpyAsync(b + hl.o_H, prob->H, szH, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+                cudaMemcpyAsync(b + hl.o_E, prob->E, szE, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+                cudaMemcpyAsync(b + hl.o_tg, prob->targets, 4 * prob->T * prob->K, cudaMemcpyHostToDevice, st) ==
+                    cudaSuccess &&
+                (prob->mask == nullptr ||
+                 cudaMemcpyAsync(b + hl.o_mask, prob->mask, prob->T, cudaMemcpyHostToDevice, st) == cudaSuccess) &&
+                cudaMemcpyAsync(b + hl.o_grad, &grad_loss, 4, cudaMemcpyHostToDevice, st) == cudaSuccess;
   cutbce_problem dp = *prob;
   dp.H = b + hl.o_H;
   dp.E = b + hl.o_E;
@@ -591,39 +658,26 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   dp.mask = prob->mask != nullptr ? reinterpret_cast<const uint8_t*>(b + hl.o_mask) : nullptr;
   float* ddH = dH ? reinterpret_cast<float*>(b + hl.o_dH) : nullptr;
   float* ddE = dE ? reinterpret_cast<float*>(b + hl.o_dE) : nullptr;
-  // dE is final once the item-owned pass ends: its copy to the host runs on a
-  // second stream while the position-owned pass and the finish run on `st`.
-  cudaStream_t s2 = nullptr;
-  cudaEvent_t item_done = nullptr;
-  if (dE != nullptr) {
-    if (cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking) != cudaSuccess) return CUTBCE_ERR_CUDA;
-    if (cudaEventCreateWithFlags(&item_done, cudaEventDisableTiming) != cudaSuccess) {
-      cudaStreamDestroy(s2);
-      return CUTBCE_ERR_CUDA;
-    }
-  }
-  auto release = [&]() {
-    if (item_done != nullptr) cudaEventDestroy(item_done);
-    if (s2 != nullptr) cudaStreamDestroy(s2);
-  };
-  s = run(&dp, reinterpret_cast<const float*>(b + hl.o_grad), reinterpret_cast<double*>(b + hl.o_loss), ddH, ddE,
-          Want{true, dE != nullptr, dH != nullptr}, b + hl.o_ws, pl.total, st, item_done);
+  s = copied ? run(&dp, reinterpret_cast<const float*>(b + hl.o_grad), reinterpret_cast<double*>(b + hl.o_loss),
+                   ddH, ddE, Want{true, dE != nullptr, dH != nullptr}, b + hl.o_ws, pl.total, st, side.ev)
+             : CUTBCE_ERR_CUDA;
   if (s != CUTBCE_OK) {
-    if (s2 != nullptr) cudaStreamSynchronize(st);   // nothing may still use the buffers on return
-    release();
+    cudaStreamSynchronize(st);   // no copy from or to the caller's host memory may still run on return
+    if (dE != nullptr) give_side_stream(side);
     return s;
   }
   int dev_status = 0;
   bool ok = true;
   if (dE != nullptr)
-    ok = cudaStreamWaitEvent(s2, item_done, 0) == cudaSuccess &&
-         cudaMemcpyAsync(dE, ddE, 4 * prob->V * prob->D, cudaMemcpyDeviceToHost, s2) == cudaSuccess;
+    ok = cudaStreamWaitEvent(side.s, side.ev, 0) == cudaSuccess &&
+         cudaMemcpyAsync(dE, ddE, 4 * prob->V * prob->D, cudaMemcpyDeviceToHost, side.s) == cudaSuccess;
   ok = ok && cudaMemcpyAsync(loss, b + hl.o_loss, 8, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
        (!dH || cudaMemcpyAsync(dH, ddH, 4 * prob->T * prob->D, cudaMemcpyDeviceToHost, st) == cudaSuccess) &&
        cudaMemcpyAsync(&dev_status, b + hl.o_ws + pl.o_hdr, 4, cudaMemcpyDeviceToHost, st) == cudaSuccess;
   // both streams are drained before returning, also after an error
-  const bool sync_ok = cudaStreamSynchronize(st) == cudaSuccess && (s2 == nullptr || cudaStreamSynchronize(s2) == cudaSuccess);
-  release();
+  const bool sync_ok = cudaStreamSynchronize(st) == cudaSuccess &&
+                       (dE == nullptr || cudaStreamSynchronize(side.s) == cudaSuccess);
+  if (dE != nullptr) give_side_stream(side);
   if (!ok || !sync_ok) return CUTBCE_ERR_CUDA;
   return static_cast<cutbce_status>(dev_status);
 }
@@ -643,7 +697,7 @@ cutbce_status cutbce_read_counts(const cutbce_problem* prob, const void* ws, int
   if (s != CUTBCE_OK) return s;
   if (ws == nullptr || n_valid == nullptr || n_pairs == nullptr) return CUTBCE_ERR_INVALID_ARG;
   Plan pl;
-  make_plan(prob, pl);
+  make_plan(prob, kWantAll, pl);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   WsHeader h;
   const uint8_t* b = static_cast<const uint8_t*>(ws);
@@ -660,7 +714,7 @@ cutbce_status cutbce_read_counts(const cutbce_problem* prob, const void* ws, int
 int cutbce_kernel_launches(const cutbce_problem* prob, int entry) {
   if (check_problem(prob, false) != CUTBCE_OK || entry < 0 || entry > 2) return -1;
   Plan pl;
-  make_plan(prob, pl);
+  make_plan(prob, kWantAll, pl);
   const Want w = entry == 0 ? Want{true, false, false} : entry == 1 ? Want{false, true, true} : Want{true, true, true};
   return count_launches(pl, w);
 }
@@ -720,7 +774,16 @@ cutbce_status cutbce_probe_pipe_rate(int op, void* scratch, size_t scratch_bytes
     case kProbeFmax: launch(k_probe<kProbeFmax>); break;
     case kProbeAdd2: launch(k_probe<kProbeAdd2>); break;
     case kProbeIadd: launch(k_probe<kProbeIadd>); break;
-    default: launch(k_probe<kProbePrmt>); break;
+    case kProbePrmt: launch(k_probe<kProbePrmt>); break;
+    case kProbeEx2F16x2: launch(k_probe<kProbeEx2F16x2>); break;
+    case kProbeEx2Bf16x2: launch(k_probe<kProbeEx2Bf16x2>); break;
+    case kProbeTanhF16x2: launch(k_probe<kProbeTanhF16x2>); break;
+    case kProbeHfma2: launch(k_probe<kProbeHfma2>); break;
+    case kProbeCvtF16x2: launch(k_probe<kProbeCvtF16x2>); break;
+    case kProbeFfmaSat: launch(k_probe<kProbeFfmaSat>); break;
+    case kProbeSelp: launch(k_probe<kProbeSelp>); break;
+    case kProbeLop3: launch(k_probe<kProbeLop3>); break;
+    default: launch(k_probe<kProbeFmul2>); break;
   }
   if (e != cudaSuccess) return CUTBCE_ERR_CUDA;
   std::vector<unsigned long long> h(grid);
@@ -728,7 +791,8 @@ cutbce_status cutbce_probe_pipe_rate(int op, void* scratch, size_t scratch_bytes
       cudaStreamSynchronize(st) != cudaSuccess)
     return CUTBCE_ERR_CUDA;
   std::sort(h.begin(), h.end());
-  const double ops = static_cast<double>(kProbeThreads) * kIters * kProbeChains * ((op == kProbeFfma2 || op == kProbeAdd2) ? 2 : 1);
+  const bool two = op == kProbeFfma2 || op == kProbeAdd2 || op == kProbeFmul2;   // fp32x2: two operations each
+  const double ops = static_cast<double>(kProbeThreads) * kIters * kProbeChains * (two ? 2 : 1);
   *ops_per_clock_per_sm = h[grid / 2] > 0 ? ops / static_cast<double>(h[grid / 2]) : 0.0;
   return CUTBCE_OK;
 }

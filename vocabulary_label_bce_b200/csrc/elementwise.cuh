@@ -93,4 +93,96 @@ __device__ __forceinline__ float2 sigmoid_pair(float2 z) {
   return rcp2_cubic(nw);
 }
 
+// ---------------------------------------------------------------- variants under measurement
+#ifndef CUTBCE_ITEM_MATH
+#define CUTBCE_ITEM_MATH 0
+#endif
+#ifndef CUTBCE_POS_MATH
+#define CUTBCE_POS_MATH 0
+#endif
+#ifndef CUTBCE_POS_POLY_PAIRS
+#define CUTBCE_POS_POLY_PAIRS 0
+#endif
+
+// 1 for t >= 0, 0 for t < 0, on the FMA pipe: saturate(t * 2^100 + 1).  Only for
+// |t| < 2^-100 is the result strictly between 0 and 1.
+__device__ __forceinline__ float nonneg_mask(float t) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(t), "f"(0x1p100f), "f"(1.0f));
+  return r;
+}
+
+// n / w for w = -nw in [1, 2]: linear minimax seed r0 = (24 - 8 w) / 17, then the
+// cubic step applied to the quotient: q = n r0 (1 + e + e^2), e = 1 - w r0, so
+// |q / (n / w) - 1| = |e|^3 <= (1/17)^3 = 2.1e-4.
+__device__ __forceinline__ float2 quot2_unit_interval(float2 n, float2 nw) {
+  const float2 r = __ffma2_rn(nw, f2(8.f / 17.f, 8.f / 17.f), f2(24.f / 17.f, 24.f / 17.f));
+  const float2 e = __ffma2_rn(nw, r, f2(1.f, 1.f));
+  const float2 t = __ffma2_rn(e, e, e);
+  const float2 q = __fmul2_rn(n, r);
+  return __ffma2_rn(q, t, q);
+}
+
+// Item-owned pass, select-free: the sign of z enters through the FMA-pipe mask
+// s = [z >= 0], which also forms max(z, 0) = z s in one packed FMA.
+__device__ __forceinline__ float2 bce_pair_loss_grad_mask(float2 z, float2& prod, float2& relu) {
+  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
+  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));   // e^{-|z|}
+  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));           // -(1 + u)
+  prod = __fmul2_rn(prod, nw);
+  const float2 s = f2(nonneg_mask(tz.x), nonneg_mask(tz.y));
+  relu = __ffma2_rn(z, s, relu);
+#if CUTBCE_ITEM_MATH == 2
+  const float2 n = f2(fmaxf(u.x, s.x), fmaxf(u.y, s.y));                     // 1 (z >= 0) or u
+#else
+  const float2 omu = __ffma2_rn(u, f2(-1.f, -1.f), f2(1.f, 1.f));            // 1 - u
+  const float2 n = __ffma2_rn(s, omu, u);                                    // 1 (z >= 0) or u
+#endif
+  return quot2_unit_interval(n, nw);
+}
+
+// 2^x for x in [-100, 100] on the FMA pipe: x = j + f with j = rint(x) taken from
+// the low mantissa bits of x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial fitted by a Remez exchange for minimum relative error on
+// [-1/2, 1/2] (max relative error 7.5e-5, float32 Horner included); the
+// exponent j is added to the result's exponent field with one integer
+// multiply-add (bits(j_shifted) * 2^23 keeps j's low 9 bits, two's complement).
+__device__ __forceinline__ float2 exp2_poly3_pair(float2 x) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  const float2 j = __fadd2_rn(x, f2(kShift, kShift));
+  const float2 jr = __fadd2_rn(j, f2(-kShift, -kShift));             // rint(x), exact
+  const float2 f = __ffma2_rn(jr, f2(-1.f, -1.f), x);                // x - rint(x), exact
+  float2 p = __ffma2_rn(f2(0.0551716685f, 0.0551716685f), f, f2(0.2426111251f, 0.2426111251f));
+  p = __ffma2_rn(p, f, f2(0.6932609677f, 0.6932609677f));
+  p = __ffma2_rn(p, f, f2(0.9999280572f, 0.9999280572f));
+  uint32_t rx, ry;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(rx) : "r"(__float_as_uint(j.x)), "r"(1u << 23), "r"(__float_as_uint(p.x)));
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(ry) : "r"(__float_as_uint(j.y)), "r"(1u << 23), "r"(__float_as_uint(p.y)));
+  return f2(__uint_as_float(rx), __uint_as_float(ry));
+}
+
+// Gradient only, saturating clamp on the FMA pipe: x = clamp(-z log2 e, -100, 100)
+// formed as 200 * saturate(-z log2 e / 200 + 1/2) - 100 (error <= 200 * 2^-25 in x,
+// 4e-6 relative in 2^x), then sigmoid = 1 / (1 + 2^x) with the exponent-flip
+// seed and the cubic step.  kPoly: 2^x on the FMA pipe instead of the SFU.
+template <bool kPoly>
+__device__ __forceinline__ float2 sigmoid_pair_sat(float2 z) {
+  float ax, ay;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ax) : "f"(z.x), "f"(-kLog2eF / 200.f), "f"(0.5f));
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ay) : "f"(z.y), "f"(-kLog2eF / 200.f), "f"(0.5f));
+  const float2 x = __ffma2_rn(f2(ax, ay), f2(200.f, 200.f), f2(-100.f, -100.f));
+  const float2 v = kPoly ? exp2_poly3_pair(x) : f2(ex2_approx(x.x), ex2_approx(x.y));
+  const float2 nw = __ffma2_rn(v, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + v)
+  return rcp2_cubic(nw);
+}
+
+// Gradient only, symmetric form: u = 2^{-|z| log2 e}, n = [z >= 0] or u, q = n / (1 + u).
+__device__ __forceinline__ float2 sigmoid_pair_sym(float2 z) {
+  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
+  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));
+  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));
+  const float2 n = f2(fmaxf(u.x, nonneg_mask(tz.x)), fmaxf(u.y, nonneg_mask(tz.y)));
+  return quot2_unit_interval(n, nw);
+}
+
 }  // namespace cutbce

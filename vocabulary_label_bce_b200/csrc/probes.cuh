@@ -25,7 +25,16 @@ enum : int {
   kProbeAdd2 = 8,     // add.rn.f32x2 (two additions per instruction)
   kProbeIadd = 9,     // add.s32
   kProbePrmt = 10,    // prmt.b32
-  kProbeCount = 11
+  kProbeEx2F16x2 = 11,   // ex2.approx.f16x2 (+ one packed add to stay in range), counted per instruction
+  kProbeEx2Bf16x2 = 12,  // ex2.approx.ftz.bf16x2 (+ one packed add), counted per instruction
+  kProbeTanhF16x2 = 13,  // tanh.approx.f16x2, counted per instruction
+  kProbeHfma2 = 14,      // fma.rn.f16x2, counted per instruction
+  kProbeCvtF16x2 = 15,   // cvt.rn.f16x2.f32, counted per instruction
+  kProbeFfmaSat = 16,    // fma.rn.sat.f32
+  kProbeSelp = 17,       // setp.ge.f32 + selp.f32 (one select), counted per select
+  kProbeLop3 = 18,       // and.b32 with a register operand
+  kProbeFmul2 = 19,      // mul.rn.f32x2, counted as two operations
+  kProbeCount = 20
 };
 
 constexpr int kProbeThreads = 1024;
@@ -34,6 +43,12 @@ constexpr int kProbeChains = 8;
 __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm volatile("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t fmul2_u(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm volatile("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 
@@ -49,7 +64,7 @@ __global__ void __launch_bounds__(kProbeThreads, 1) k_probe(int iters, unsigned 
 #pragma unroll
   for (int k = 0; k < kProbeChains; ++k) a[k] = 0.25f + 1e-4f * static_cast<float>((threadIdx.x + 37 * k) & 255);
   uint64_t a2[kProbeChains];
-  if (OP == kProbeFfma2 || OP == kProbeAdd2) {
+  if (OP == kProbeFfma2 || OP == kProbeAdd2 || OP == kProbeFmul2) {
 #pragma unroll
     for (int k = 0; k < kProbeChains; ++k)
       a2[k] = (static_cast<uint64_t>(__float_as_uint(a[k])) << 32) | __float_as_uint(a[k] + 0.5f);
@@ -78,6 +93,38 @@ __global__ void __launch_bounds__(kProbeThreads, 1) k_probe(int iters, unsigned 
         a[k] = __uint_as_float(v);
       }
       if (OP == kProbePrmt) a[k] = __uint_as_float(__byte_perm(__float_as_uint(a[k]), 0x12345678u, 0x3726u));
+      if (OP == kProbeEx2F16x2 || OP == kProbeEx2Bf16x2 || OP == kProbeTanhF16x2 || OP == kProbeHfma2) {
+        // two 16-bit lanes in one register; values stay in a small range
+        uint32_t v = __float_as_uint(a[k]);
+        if (OP == kProbeEx2F16x2) {
+          asm volatile("ex2.approx.f16x2 %0, %0;" : "+r"(v));
+          asm volatile("sub.f16x2 %0, %0, %1;" : "+r"(v) : "r"(0x3E003E00u));          // - 1.5
+        } else if (OP == kProbeEx2Bf16x2) {
+          asm volatile("ex2.approx.ftz.bf16x2 %0, %0;" : "+r"(v));
+          asm volatile("sub.bf16x2 %0, %0, %1;" : "+r"(v) : "r"(0x3FC03FC0u));         // - 1.5
+        } else if (OP == kProbeTanhF16x2) {
+          asm volatile("tanh.approx.f16x2 %0, %0;" : "+r"(v));
+        } else {
+          asm volatile("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(v) : "r"(0x3BFF3BFFu), "r"(0x1A001A00u));
+        }
+        a[k] = __uint_as_float(v);
+      }
+      if (OP == kProbeCvtF16x2) {
+        uint32_t v;
+        asm volatile("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(a[k]), "f"(a[k]));
+        a[k] = __uint_as_float(v & 0x3FFFFFFFu);
+      }
+      if (OP == kProbeFfmaSat) asm volatile("fma.rn.sat.f32 %0, %0, %1, %2;" : "+f"(a[k]) : "f"(0.999f), "f"(1e-3f));
+      if (OP == kProbeSelp) {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ge.f32 p, %0, %1;\n\tselp.f32 %0, %2, %0, p;\n\t}"
+                     : "+f"(a[k]) : "f"(0.5f), "f"(0.25f));
+      }
+      if (OP == kProbeLop3) {
+        uint32_t v = __float_as_uint(a[k]);
+        asm volatile("and.b32 %0, %0, %1;" : "+r"(v) : "r"(0xFFFFFF7Fu + static_cast<uint32_t>(k)));
+        a[k] = __uint_as_float(v);
+      }
+      if (OP == kProbeFmul2) a2[k] = fmul2_u(a2[k], m2);
     }
   }
   __syncthreads();
@@ -85,7 +132,8 @@ __global__ void __launch_bounds__(kProbeThreads, 1) k_probe(int iters, unsigned 
   float s = 0.f;
 #pragma unroll
   for (int k = 0; k < kProbeChains; ++k)
-    s += (OP == kProbeFfma2 || OP == kProbeAdd2) ? __uint_as_float(static_cast<uint32_t>(a2[k])) : a[k];
+    s += (OP == kProbeFfma2 || OP == kProbeAdd2 || OP == kProbeFmul2) ? __uint_as_float(static_cast<uint32_t>(a2[k]))
+                                                                     : a[k];
   if (s == 12345.678f) sink[threadIdx.x] = s;
   if (threadIdx.x == 0) cycles[blockIdx.x] = static_cast<unsigned long long>(t1 - t0);
 }

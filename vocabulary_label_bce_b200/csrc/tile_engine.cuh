@@ -632,9 +632,21 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             for (int e = 0; e < CH; e += 2) {
               const float2 z = f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
               float2 g = f2(0.f, 0.f);
-              if (kLoss && kGrad) g = bce_pair_loss_grad(z, prod, relu);
-              else if (kLoss) bce_pair_loss(z, prod, relu);
-              else g = sigmoid_pair(z);
+              if (kLoss && kGrad) {
+                g = CUTBCE_ITEM_MATH == 0 ? bce_pair_loss_grad(z, prod, relu) : bce_pair_loss_grad_mask(z, prod, relu);
+              } else if (kLoss) {
+                bce_pair_loss(z, prod, relu);
+              } else {
+#if CUTBCE_POS_MATH == 0
+                g = sigmoid_pair(z);
+#elif CUTBCE_POS_MATH == 1
+                // CUTBCE_POS_POLY_PAIRS of the 16 pairs of a chunk, spread evenly, on the FMA pipe
+                if (((e >> 1) * CUTBCE_POS_POLY_PAIRS) % 16 < CUTBCE_POS_POLY_PAIRS) g = sigmoid_pair_sat<true>(z);
+                else g = sigmoid_pair_sat<false>(z);
+#else
+                g = sigmoid_pair_sym(z);
+#endif
+              }
               if (kGrad) {
                 if (decltype(with_y)::value) {                     // y = 1 at the masked columns
                   if (mask & (1u << e)) g.x -= 1.f;                // a predicated add, no conversion
