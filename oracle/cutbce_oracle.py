@@ -37,7 +37,8 @@ Readings where the paper is silent:
   * with no valid position the loss and both gradients are 0.
 
 Every function here is pinned by tests/test_oracle_pins.py against identities,
-closed forms, finite differences and torch's own BCE-with-logits.
+closed forms, finite differences, torch's own BCE-with-logits, brute-force
+enumeration on tiny inputs and scikit-learn's classification metrics.
 """
 from __future__ import annotations
 
@@ -258,3 +259,51 @@ def loss_sum_slice(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Opti
         Z = Hv @ np.asarray(E[c0:c1], dtype=np.float64).T
         total += float(bce_eq2(Z, _multi_hot(sets_v, c0, c1)).sum())
     return total
+
+
+# ---------------------------------------------------------------- Cut Metrics (section III-D)
+# Confusion counts per position over the whole vocabulary, computed from the
+# logits without keeping them.  The pages give the four counts of shape [B, N]
+# and say accuracy, precision, recall and F_beta follow from them; they do not
+# state the decision threshold.  Reading: item v is predicted positive for
+# position t iff sigmoid(x_tv) > 1/2, i.e. x_tv > 0 (a logit of exactly 0 is a
+# predicted negative).  A masked position has all four counts 0.
+
+def cut_metrics(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np.ndarray] = None,
+                chunk: int = 8192) -> np.ndarray:
+    """int64 [T, 4]: (TP, FP, FN, TN) of each position, from the dense logits chunk by chunk."""
+    H64 = np.asarray(H, dtype=np.float64)
+    V = E.shape[0]
+    tg = positive_sets(targets, mask, V)
+    rows = np.nonzero(tg.valid)[0]
+    Hv = H64[rows]
+    sets_v = [tg.sets[t] for t in rows]
+    counts = np.zeros((H64.shape[0], 4), dtype=np.int64)
+    if len(rows) == 0:
+        return counts
+    acc = np.zeros((len(rows), 4), dtype=np.int64)
+    for c0 in range(0, V, chunk):
+        c1 = min(V, c0 + chunk)
+        Z = Hv @ np.asarray(E[c0:c1], dtype=np.float64).T
+        pred = Z > 0.0
+        y = _multi_hot(sets_v, c0, c1) > 0.5
+        acc[:, 0] += np.sum(pred & y, axis=1)
+        acc[:, 1] += np.sum(pred & ~y, axis=1)
+        acc[:, 2] += np.sum(~pred & y, axis=1)
+        acc[:, 3] += np.sum(~pred & ~y, axis=1)
+    counts[rows] = acc
+    return counts
+
+
+def metrics_from_counts(counts: np.ndarray, beta: float = 1.0) -> dict:
+    """Binary accuracy, precision, recall and F_beta of the counts summed over positions
+    (a ratio with a zero denominator is 0)."""
+    tp, fp, fn, tn = (float(x) for x in np.asarray(counts, dtype=np.int64).reshape(-1, 4).sum(axis=0))
+    total = tp + fp + fn + tn
+    precision = tp / (tp + fp) if tp + fp > 0 else 0.0
+    recall = tp / (tp + fn) if tp + fn > 0 else 0.0
+    b2 = beta * beta
+    denom = b2 * precision + recall
+    fbeta = (1.0 + b2) * precision * recall / denom if denom > 0 else 0.0
+    return {"accuracy": (tp + tn) / total if total > 0 else 0.0, "precision": precision, "recall": recall,
+            "fbeta": fbeta}
