@@ -30,9 +30,11 @@ Readings where the paper is silent:
   * duplicate ids in a row count once (Y is multi-hot, y in {0, 1});
   * -1 marks an empty slot; an id < -1 or >= V in a valid row is an error;
     id 0 is an ordinary item;
-  * the per-position `weights` of the paper's API is read as a {0, 1} mask: a
-    masked row adds no loss, gets a zero dH row and adds nothing to dE; its ids
-    are ignored entirely (not even range-checked);
+  * a masked row adds no loss, gets a zero dH row and adds nothing to dE; its
+    ids are ignored entirely (not even range-checked);
+  * the per-position `weights` of the paper's API multiply the position's loss
+    row and its row of G; a zero weight makes the position padding (excluded
+    from the mean, like a masked one), so {0, 1} weights are the mask;
   * the upstream gradient is one scalar g (default 1) multiplying dH and dE;
   * with no valid position the loss and both gradients are 0.
 
@@ -77,20 +79,32 @@ class Targets:
         return int(self.row_counts.sum())
 
 
-def positive_sets(targets: np.ndarray, mask: Optional[np.ndarray], V: int) -> Targets:
-    """Apply the mask and the id rules: P_t = set of ids >= 0 in a valid row."""
+def positive_sets(targets: np.ndarray, mask: Optional[np.ndarray], V: int,
+                  weights: Optional[np.ndarray] = None, vocab_offset: int = 0,
+                  V_total: Optional[int] = None) -> Targets:
+    """Apply the mask, the weights and the id rules: P_t = set of ids >= 0 in a valid row.
+
+    A position is valid iff its mask entry is nonzero and its weight (if given) is
+    nonzero.  With a vocabulary shard (vocab_offset, V_total), ids are global: an
+    id outside [-1, V_total) is an error, an id outside [vocab_offset,
+    vocab_offset + V) is not in this shard and is dropped, and the kept ids are
+    returned shard-local (id - vocab_offset)."""
     targets = np.asarray(targets)
     T = targets.shape[0]
+    Vt = V if V_total is None else int(V_total)
     valid = np.ones(T, dtype=bool) if mask is None else (np.asarray(mask) != 0)
+    if weights is not None:
+        valid = valid & (np.asarray(weights, dtype=np.float64) != 0.0)
     sets = []
     for t in range(T):
         if not valid[t]:
             sets.append(np.zeros(0, dtype=np.int64))
             continue
         row = targets[t].astype(np.int64)
-        if np.any(row < -1) or np.any(row >= V):
-            raise TargetRangeError(f"row {t}: id outside [-1, {V})")
-        sets.append(np.unique(row[row >= 0]))
+        if np.any(row < -1) or np.any(row >= Vt):
+            raise TargetRangeError(f"row {t}: id outside [-1, {Vt})")
+        local = row[(row >= vocab_offset) & (row < vocab_offset + V)] - vocab_offset
+        sets.append(np.unique(local))
     return Targets(valid=valid, sets=sets)
 
 
@@ -154,20 +168,35 @@ class Result:
 
 def forward_backward(H: np.ndarray, E: np.ndarray, targets: np.ndarray,
                      mask: Optional[np.ndarray] = None, reduction: int = MEAN_VALID_POSITIONS,
-                     grad_loss: float = 1.0, chunk: int = 8192, want_grad: bool = True) -> Result:
+                     grad_loss: float = 1.0, chunk: int = 8192, want_grad: bool = True,
+                     weights: Optional[np.ndarray] = None, vocab_offset: int = 0,
+                     V_total: Optional[int] = None) -> Result:
     """Loss and gradients of the fused BCE, computed densely chunk by chunk over V.
 
     H [T, D] and E [V, D] are taken as given (the exact input values, widened to
     float64); targets [T, K] int ids with -1 empty; mask [T] (nonzero = valid).
+
+    weights [T] (the per-position weights of the paper's API, section III-C
+    Listing 1): position t's loss row and its row of G are multiplied by w_t, so
+    loss = s sum_t w_t sum_v l(x_tv, y_tv), G = diag(w) (sigmoid(X) - Y); a
+    position with w_t = 0 is padding (not counted in the mean).
+
+    vocab_offset, V_total: E holds items [vocab_offset, vocab_offset + V) of a
+    vocabulary of V_total items (one shard of a vocabulary-parallel split): the
+    result is this shard's share of the loss sum and of dH (the shares of all
+    shards add up to the unsharded result) and the shard's rows of dE.  The
+    MEAN_ELEMENTS normalisation uses V_total.
     """
     H64 = np.asarray(H, dtype=np.float64)
     E64 = np.asarray(E, dtype=np.float64)
     T, D = H64.shape
     V = E64.shape[0]
-    tg = positive_sets(targets, mask, V)
+    Vt = V if V_total is None else int(V_total)
+    tg = positive_sets(targets, mask, V, weights, vocab_offset, Vt)
     rows = np.nonzero(tg.valid)[0]
     Hv = H64[rows]
     sets_v = [tg.sets[t] for t in rows]
+    w = np.ones(len(rows)) if weights is None else np.asarray(weights, dtype=np.float64)[rows]
 
     total = 0.0
     dHv = np.zeros_like(Hv) if want_grad else None
@@ -178,12 +207,12 @@ def forward_backward(H: np.ndarray, E: np.ndarray, targets: np.ndarray,
             Ec = E64[c0:c1]
             Z = Hv @ Ec.T                                  # chunk logits, then discarded
             Y = _multi_hot(sets_v, c0, c1)
-            total += float(bce_eq2(Z, Y).sum())            # Eq. (2), summed as in Eq. (3)
+            total += float((w[:, None] * bce_eq2(Z, Y)).sum())   # Eq. (2), summed as in Eq. (3)
             if want_grad:
-                G = sigmoid(Z) - Y                         # Eq. (4)
+                G = w[:, None] * (sigmoid(Z) - Y)          # Eq. (4), row t scaled by w_t
                 dHv += G @ Ec
                 dE[c0:c1] = G.T @ Hv
-    s = scale_factor(reduction, len(rows), V)
+    s = scale_factor(reduction, len(rows), Vt)
     dH = None
     if want_grad:
         dH = np.zeros((T, D), dtype=np.float64)
@@ -270,11 +299,16 @@ def loss_sum_slice(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Opti
 # predicted negative).  A masked position has all four counts 0.
 
 def cut_metrics(H: np.ndarray, E: np.ndarray, targets: np.ndarray, mask: Optional[np.ndarray] = None,
-                chunk: int = 8192) -> np.ndarray:
-    """int64 [T, 4]: (TP, FP, FN, TN) of each position, from the dense logits chunk by chunk."""
+                chunk: int = 8192, weights: Optional[np.ndarray] = None, vocab_offset: int = 0,
+                V_total: Optional[int] = None) -> np.ndarray:
+    """int64 [T, 4]: (TP, FP, FN, TN) of each position, from the dense logits chunk by chunk.
+
+    The counts are not weighted; a position with weight 0 is padding (all zero).
+    On a vocabulary shard the counts cover the shard's items only (the counts of
+    all shards add up to the unsharded counts)."""
     H64 = np.asarray(H, dtype=np.float64)
     V = E.shape[0]
-    tg = positive_sets(targets, mask, V)
+    tg = positive_sets(targets, mask, V, weights, vocab_offset, V if V_total is None else V_total)
     rows = np.nonzero(tg.valid)[0]
     Hv = H64[rows]
     sets_v = [tg.sets[t] for t in rows]
