@@ -105,13 +105,15 @@ typedef struct {
 cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes);
 
 /* Outputs of a compute call, as bits of `outputs` below. */
-enum { CUTBCE_OUT_LOSS = 1, CUTBCE_OUT_DH = 2, CUTBCE_OUT_DE = 4 };
+enum { CUTBCE_OUT_LOSS = 1, CUTBCE_OUT_DH = 2, CUTBCE_OUT_DE = 4, CUTBCE_OUT_METRICS = 8 };
 
 /* Bytes of device workspace for a call that computes only the given outputs
  * (a bitwise or of CUTBCE_OUT_*): cutbce_forward needs CUTBCE_OUT_LOSS;
  * cutbce_backward and cutbce_forward_backward need the bits of the outputs
- * they are given non-NULL.  The dH split partials (O(S*T*D)) are counted only
- * with CUTBCE_OUT_DH, and the pair-sort buffers (O(T*K)) only with
+ * they are given non-NULL; cutbce_forward_backward_ex adds CUTBCE_OUT_METRICS
+ * when it is given a metrics output.  The dH split partials (O(S*T*D)) are
+ * counted only with CUTBCE_OUT_DH, the metrics partials (O(S*T)) only with
+ * CUTBCE_OUT_METRICS, and the pair-sort buffers (O(T*K)) only with
  * CUTBCE_OUT_DE, so a loss-only workspace is O(T*K + T*D + V).  Host-only. */
 cutbce_status cutbce_workspace_size_for(const cutbce_problem* prob, int outputs, size_t* bytes);
 
@@ -171,6 +173,67 @@ cutbce_status cutbce_backward(const cutbce_problem* prob, const float* grad_loss
 cutbce_status cutbce_forward_backward(const cutbce_problem* prob, const float* grad_loss,
                                       double* loss, float* dH, float* dE,
                                       void* ws, size_t ws_bytes, cutbce_stream_t stream);
+
+/* dtype of the dH and dE outputs of cutbce_forward_backward_ex. */
+enum { CUTBCE_GRAD_F32 = 0, CUTBCE_GRAD_BF16 = 1 };
+/* Bits of cutbce_options.accumulate. */
+enum { CUTBCE_ACCUMULATE_DH = 1, CUTBCE_ACCUMULATE_DE = 2 };
+
+/* Options of cutbce_forward_backward_ex; a zero-initialised struct gives the
+ * behaviour of cutbce_forward_backward. */
+typedef struct {
+  /* Cut Metrics (section III-D): [T, 4] int32 device output, 16-byte aligned, or
+   * NULL.  Row t holds (TP, FP, FN, TN) of position t over the vocabulary of this
+   * call, item v counted as predicted positive iff sigmoid(x_tv) > 1/2, i.e.
+   * x_tv > 0 as the kernel computes x_tv (fp32 accumulation of the products; a
+   * logit of exactly 0, or one below the smallest normal float, is a predicted
+   * negative).  TP + FP + FN + TN = V; invalid positions get (0, 0, 0, 0).  The
+   * counts are not weighted.  They come from a position-owned pass over the
+   * logits: fused into the dH pass when dH is requested, a count-only pass
+   * otherwise. */
+  int32_t* metrics;
+  /* Per-position weights w (the `weights` argument of section III-C, Listing 1):
+   * float [T] device array, 4-byte aligned, or NULL for w = 1.  Position t's loss
+   * row and its row of G = sigmoid(X) - Y are multiplied by w_t:
+   *   loss = s sum_t w_t sum_v l(x_tv, y_tv),  dH_t = g s w_t sum_v (sigmoid - y) e_v,
+   *   dE_v = g s sum_t w_t (sigmoid - y) h_t.
+   * A position with w_t = 0 is padding, exactly like a masked one: it is not
+   * counted in the mean and gets a zero dH row.  With weights the loss is
+   * summed in the position-owned pass (one weight per row) and the item-owned
+   * pass scales each column of G by its weight. */
+  const float* weights;
+  /* CUTBCE_GRAD_F32 (default) or CUTBCE_GRAD_BF16: dtype of the dH and dE
+   * outputs (bf16 is rounded to nearest even from the fp32 result). */
+  int32_t grad_dtype;
+  /* Bitwise or of CUTBCE_ACCUMULATE_DH / _DE: add the gradient to what the
+   * output already holds instead of overwriting it (the sum is formed in fp32
+   * and rounded once; masked rows of dH keep their value). */
+  int32_t accumulate;
+  /* Vocabulary sharding (section III-C, the vocabulary-parallel split): E holds
+   * items [vocab_offset, vocab_offset + V) of a vocabulary of V_total items
+   * (V_total = 0 means V, and then vocab_offset must be 0).  Target ids are
+   * global: an id in [0, V_total) outside this shard is not a positive of this
+   * call (and not an error); an id < -1 or >= V_total in a valid row is
+   * CUTBCE_ERR_TARGET_RANGE.  The loss and dH are this shard's shares (the sums
+   * over all shards are the unsharded results, with the same normalisation s;
+   * MEAN_ELEMENTS uses V_total), dE holds this shard's rows, and the metrics
+   * count this shard's items. */
+  int64_t vocab_offset;
+  int64_t V_total;
+} cutbce_options;
+
+/* cutbce_forward_backward with options (see cutbce_options).  dH and dE point
+ * to fp32 or bf16 arrays according to opts->grad_dtype.  At least one of loss,
+ * dH, dE and opts->metrics must be non-NULL; ws must hold
+ * cutbce_workspace_size_ex(prob, opts, the bits of those outputs) bytes. */
+cutbce_status cutbce_forward_backward_ex(const cutbce_problem* prob, const cutbce_options* opts,
+                                         const float* grad_loss, double* loss, void* dH, void* dE,
+                                         void* ws, size_t ws_bytes, cutbce_stream_t stream);
+
+/* Workspace bytes of cutbce_forward_backward_ex for these options and outputs
+ * (bits CUTBCE_OUT_*); opts may be NULL.  Host-only. */
+cutbce_status cutbce_workspace_size_ex(const cutbce_problem* prob, const cutbce_options* opts, int outputs,
+                                       size_t* bytes);
 
 /* Bytes of device memory that cutbce_forward_backward_host needs in dev_buf. */
 cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes);

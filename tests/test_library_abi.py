@@ -98,7 +98,9 @@ def test_workspace_size_per_outputs():
     # the loss-only layout holds neither the dH split partials nor the pair-sort buffers
     assert full - loss_only >= 16 * 12800 * 16 + 4 * 12800 * 64
     assert loss_only < 16 << 20
-    for bad in (0, 8, -1):
+    met = B.cutbce_workspace_size_for(p, B.OUT_LOSS | B.OUT_METRICS)
+    assert met - loss_only >= 8 * 12800            # one (count, TP) pair per position and split slot
+    for bad in (0, 16, -1):
         with pytest.raises(B.CutBCEError) as e:
             B.cutbce_workspace_size_for(p, bad)
         assert e.value.status == B.ERR_INVALID_ARG

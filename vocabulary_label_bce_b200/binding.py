@@ -17,7 +17,9 @@ import torch
 
 __all__ = [
     "CutBCEError", "cutbce_problem", "load_library", "library_path", "declared_functions",
-    "cutbce_workspace_size", "cutbce_workspace_size_for", "OUT_LOSS", "OUT_DH", "OUT_DE", "cutbce_forward", "cutbce_forward_fixed_scratch", "FIXED_SCRATCH_BYTES",
+    "cutbce_workspace_size", "cutbce_workspace_size_for", "OUT_LOSS", "OUT_DH", "OUT_DE", "OUT_METRICS",
+    "cutbce_options", "make_options", "cutbce_forward_backward_ex", "cutbce_workspace_size_ex",
+    "GRAD_F32", "GRAD_BF16", "ACCUMULATE_DH", "ACCUMULATE_DE", "cutbce_forward", "cutbce_forward_fixed_scratch", "FIXED_SCRATCH_BYTES",
     "cutbce_backward", "cutbce_forward_backward",
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
@@ -27,7 +29,7 @@ __all__ = [
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TARGET_RANGE, ERR_TIMEOUT, ERR_CUDA = range(7)
 BF16, F32 = 0, 1
-OUT_LOSS, OUT_DH, OUT_DE = 1, 2, 4
+OUT_LOSS, OUT_DH, OUT_DE, OUT_METRICS = 1, 2, 4, 8
 REDUCTIONS = {"mean": 0, "sum": 1, "mean_elements": 2}
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -44,6 +46,29 @@ class cutbce_problem(ctypes.Structure):
         ("dtype", ctypes.c_int32), ("reduction", ctypes.c_int32),
         ("H", ctypes.c_void_p), ("E", ctypes.c_void_p), ("targets", ctypes.c_void_p), ("mask", ctypes.c_void_p),
     ]
+
+
+class cutbce_options(ctypes.Structure):
+    _fields_ = [("metrics", ctypes.c_void_p), ("weights", ctypes.c_void_p), ("grad_dtype", ctypes.c_int32),
+                ("accumulate", ctypes.c_int32), ("vocab_offset", ctypes.c_int64), ("V_total", ctypes.c_int64)]
+
+
+GRAD_F32, GRAD_BF16 = 0, 1
+ACCUMULATE_DH, ACCUMULATE_DE = 1, 2
+
+
+def make_options(metrics: Optional[torch.Tensor] = None, weights: Optional[torch.Tensor] = None,
+                 grad_dtype: int = GRAD_F32, accumulate: int = 0, vocab_offset: int = 0,
+                 V_total: int = 0) -> cutbce_options:
+    """Options of cutbce_forward_backward_ex (see include/cutbce.h): metrics is an int32 [T, 4]
+    device tensor, weights a float32 [T] device tensor."""
+    if metrics is not None and (metrics.dtype != torch.int32 or not metrics.is_contiguous()):
+        raise ValueError("metrics must be a contiguous int32 [T, 4] tensor")
+    if weights is not None and (weights.dtype != torch.float32 or not weights.is_contiguous()):
+        raise ValueError("weights must be a contiguous float32 [T] tensor")
+    return cutbce_options(metrics.data_ptr() if metrics is not None else None,
+                          weights.data_ptr() if weights is not None else None,
+                          int(grad_dtype), int(accumulate), int(vocab_offset), int(V_total))
 
 
 class CutBCEError(RuntimeError):
@@ -63,6 +88,8 @@ _SIGS = {
     "cutbce_forward_fixed_scratch": (_i32, [_P, _vp, _vp]),
     "cutbce_backward": (_i32, [_P, _vp, _vp, _vp, _vp, _sz, _vp]),
     "cutbce_forward_backward": (_i32, [_P, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cutbce_forward_backward_ex": (_i32, [_P, ctypes.POINTER(cutbce_options), _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cutbce_workspace_size_ex": (_i32, [_P, ctypes.POINTER(cutbce_options), ctypes.c_int, ctypes.POINTER(_sz)]),
     "cutbce_host_buffer_size": (_i32, [_P, ctypes.POINTER(_sz)]),
     "cutbce_forward_backward_host": (_i32, [_P, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     "cutbce_read_status": (_i32, [_vp, _vp]),
@@ -153,6 +180,13 @@ def cutbce_workspace_size_for(prob: cutbce_problem, outputs: int) -> int:
     return int(n.value)
 
 
+def cutbce_workspace_size_ex(prob: cutbce_problem, opts: Optional[cutbce_options], outputs: int) -> int:
+    n = _sz(0)
+    _check(load_library().cutbce_workspace_size_ex(ctypes.byref(prob), ctypes.byref(opts) if opts is not None else None,
+                                                   int(outputs), ctypes.byref(n)), "cutbce_workspace_size_ex")
+    return int(n.value)
+
+
 def cutbce_forward(prob, ws: torch.Tensor, loss: torch.Tensor, stream=None) -> None:
     _check(load_library().cutbce_forward(ctypes.byref(prob), ws.data_ptr(), ws.numel(), loss.data_ptr(),
                                          _stream(stream)), "cutbce_forward")
@@ -184,6 +218,16 @@ def cutbce_forward_backward(prob, grad_loss: Optional[torch.Tensor], loss: Optio
         loss.data_ptr() if loss is not None else None, dH.data_ptr() if dH is not None else None,
         dE.data_ptr() if dE is not None else None, ws.data_ptr(), ws.numel(), _stream(stream)),
         "cutbce_forward_backward")
+
+
+def cutbce_forward_backward_ex(prob, opts: cutbce_options, grad_loss: Optional[torch.Tensor],
+                               loss: Optional[torch.Tensor], dH: Optional[torch.Tensor], dE: Optional[torch.Tensor],
+                               ws: torch.Tensor, stream=None) -> None:
+    _check(load_library().cutbce_forward_backward_ex(
+        ctypes.byref(prob), ctypes.byref(opts), grad_loss.data_ptr() if grad_loss is not None else None,
+        loss.data_ptr() if loss is not None else None, dH.data_ptr() if dH is not None else None,
+        dE.data_ptr() if dE is not None else None, ws.data_ptr(), ws.numel(), _stream(stream)),
+        "cutbce_forward_backward_ex")
 
 
 def cutbce_host_buffer_size(prob: cutbce_problem) -> int:

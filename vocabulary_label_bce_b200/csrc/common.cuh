@@ -31,8 +31,11 @@ constexpr int kNumEpiWarps = 16;      // groups x (4 TMEM lane quarters x column
 #ifndef CUTBCE_POS_GROUPS
 #define CUTBCE_POS_GROUPS 1
 #endif
+#ifndef CUTBCE_ITEM_GROUPS
+#define CUTBCE_ITEM_GROUPS 2
+#endif
 template <bool kDH>
-__host__ __device__ constexpr int epi_groups() { return kDH ? CUTBCE_POS_GROUPS : 2; }
+__host__ __device__ constexpr int epi_groups() { return kDH ? CUTBCE_POS_GROUPS : CUTBCE_ITEM_GROUPS; }
 
 // First 256 bytes of the workspace.
 struct WsHeader {

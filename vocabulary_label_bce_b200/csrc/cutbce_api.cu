@@ -36,13 +36,52 @@ int64_t finish_grid(int64_t T, int64_t D) { return std::max<int64_t>(256, ceil_d
 
 // Outputs one call computes; the workspace plan holds only what they need.
 struct Want {
-  bool loss, dE, dH;
+  bool loss, dE, dH, met;
 };
-constexpr Want kWantAll{true, true, true};
+constexpr Want kWantAll{true, true, true, false};
+constexpr int kAllOutputs = CUTBCE_OUT_LOSS | CUTBCE_OUT_DH | CUTBCE_OUT_DE | CUTBCE_OUT_METRICS;
 
 Want want_from_mask(int outputs) {
-  return Want{(outputs & CUTBCE_OUT_LOSS) != 0, (outputs & CUTBCE_OUT_DE) != 0, (outputs & CUTBCE_OUT_DH) != 0};
+  return Want{(outputs & CUTBCE_OUT_LOSS) != 0, (outputs & CUTBCE_OUT_DE) != 0, (outputs & CUTBCE_OUT_DH) != 0,
+              (outputs & CUTBCE_OUT_METRICS) != 0};
 }
+
+// Options of one call, validated (see cutbce_options in the header).
+struct Opts {
+  int32_t* metrics = nullptr;
+  const float* weights = nullptr;
+  bool grad_bf16 = false, acc_dH = false, acc_dE = false;
+  int64_t v_off = 0, V_total = 0;   // V_total resolved: the problem's V when not sharded
+};
+
+cutbce_status resolve_opts(const cutbce_problem* p, const cutbce_options* o, Opts& out) {
+  out = Opts{};
+  out.V_total = p->V;
+  if (o == nullptr) return CUTBCE_OK;
+  out.metrics = o->metrics;
+  out.weights = o->weights;
+  if (o->grad_dtype != CUTBCE_GRAD_F32 && o->grad_dtype != CUTBCE_GRAD_BF16) return CUTBCE_ERR_UNSUPPORTED;
+  if (o->accumulate < 0 || o->accumulate > (CUTBCE_ACCUMULATE_DH | CUTBCE_ACCUMULATE_DE)) return CUTBCE_ERR_INVALID_ARG;
+  out.grad_bf16 = o->grad_dtype == CUTBCE_GRAD_BF16;
+  out.acc_dH = (o->accumulate & CUTBCE_ACCUMULATE_DH) != 0;
+  out.acc_dE = (o->accumulate & CUTBCE_ACCUMULATE_DE) != 0;
+  if (o->V_total == 0) {
+    if (o->vocab_offset != 0) return CUTBCE_ERR_INVALID_ARG;
+  } else {
+    if (o->vocab_offset < 0 || o->V_total < 0 || o->vocab_offset + p->V > o->V_total ||
+        o->V_total >= (int64_t(1) << 31))
+      return CUTBCE_ERR_INVALID_ARG;
+    out.v_off = o->vocab_offset;
+    out.V_total = o->V_total;
+  }
+  if (out.weights != nullptr && (reinterpret_cast<uintptr_t>(out.weights) & 3) != 0) return CUTBCE_ERR_INVALID_ARG;
+  if (out.metrics != nullptr && (reinterpret_cast<uintptr_t>(out.metrics) & 15) != 0) return CUTBCE_ERR_INVALID_ARG;
+  return CUTBCE_OK;
+}
+
+// (group, column slab) combinations of the position-owned pass's epilogue: one
+// metrics partial per split and combination.
+constexpr int kMetSlotsPerSplit = kNumEpiWarps / 4;
 
 struct Plan {
   int64_t T, V, D, K;
@@ -53,7 +92,8 @@ struct Plan {
   int radix_passes, radix_blocks;
   size_t elem;
   size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_srt[4], o_ghist, o_cscoff, o_hc,
-      o_lpart, o_cpart, o_dhpart, o_fpart, total;
+      o_lpart, o_cpart, o_dhpart, o_fpart, o_metpart, o_wc, total;
+  int met_slots;
 };
 
 cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
@@ -80,7 +120,7 @@ cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
 // same offsets for every set of outputs (cutbce_read_status and
 // cutbce_read_counts rely on that); the pair-sort buffers (dE only) and the dH
 // split partials (dH only) are laid out only when those outputs are wanted.
-void make_plan(const cutbce_problem* p, Want w, Plan& pl) {
+void make_plan(const cutbce_problem* p, Want w, Plan& pl, bool weighted = false) {
   pl.T = p->T;
   pl.V = p->V;
   pl.D = p->D;
@@ -128,7 +168,12 @@ void make_plan(const cutbce_problem* p, Want w, Plan& pl) {
   pl.o_pair_t = take(4 * TK);
   pl.o_pair_v = take(4 * TK);
   pl.o_hc = take(pl.elem * static_cast<size_t>(pl.Tpad) * pl.DP);
-  pl.o_lpart = take(8 * kNumEpiWarps * pl.n_vitems);
+  // dense loss partials: per item tile, or (weighted loss on the tensor-core path)
+  // per position-owned work item
+  const int64_t n_loss_items = (weighted && bf16 && w.loss) ? std::max<int64_t>(pl.n_vitems, int64_t(pl.S) * (pl.Tpad / kTileM))
+                                                           : pl.n_vitems;
+  pl.o_lpart = take(8 * kNumEpiWarps * static_cast<size_t>(n_loss_items));
+  pl.o_wc = weighted ? take(4 * static_cast<size_t>(pl.Tpad)) : 0;
   pl.o_cpart = take(8 * pl.n_gather_blocks);
   pl.o_fpart = take(16 * static_cast<size_t>(finish_grid(p->T, p->D)));
   const bool sort = bf16 && w.dE;
@@ -136,6 +181,8 @@ void make_plan(const cutbce_problem* p, Want w, Plan& pl) {
   pl.o_ghist = sort ? take(4 * 256 * static_cast<size_t>(pl.radix_blocks)) : 0;
   pl.o_cscoff = sort ? take(4 * static_cast<size_t>(pl.n_vitems + 1)) : 0;
   pl.o_dhpart = w.dH ? take(4 * static_cast<size_t>(pl.S) * pl.Tpad * pl.DP) : 0;
+  pl.met_slots = bf16 ? pl.S * kMetSlotsPerSplit : 1;
+  pl.o_metpart = w.met ? take(8 * static_cast<size_t>(pl.met_slots) * pl.Tpad) : 0;
   pl.total = o;
 }
 
@@ -259,10 +306,10 @@ struct LaunchScope {
 };
 
 // ---------------------------------------------------------------- tile-engine dispatch
-template <int DP, bool kLoss, bool kGrad, bool kDH>
+template <int DP, bool kLoss, bool kGrad, bool kDH, bool kMet>
 cudaError_t launch_tile(int grid, const CUtensorMap& s, const CUtensorMap& x, const TileParams& tp,
                         cudaStream_t st) {
-  auto kern = k_tile<DP, kLoss, kGrad, kDH>;
+  auto kern = k_tile<DP, kLoss, kGrad, kDH, kMet>;
   constexpr uint32_t smem = TileCfg<DP, epi_groups<kDH>()>::SMEM_BYTES;
   // the attribute belongs to the current device: set it once per device
   static std::atomic<uint64_t> configured{0};
@@ -280,14 +327,14 @@ cudaError_t launch_tile(int grid, const CUtensorMap& s, const CUtensorMap& x, co
   return cudaGetLastError();
 }
 
-template <bool kLoss, bool kGrad, bool kDH>
+template <bool kLoss, bool kGrad, bool kDH, bool kMet = false>
 cudaError_t launch_tile_dp(int DP, int grid, const CUtensorMap& s, const CUtensorMap& x, const TileParams& tp,
                            cudaStream_t st) {
   switch (DP) {
-    case 64: return launch_tile<64, kLoss, kGrad, kDH>(grid, s, x, tp, st);
-    case 128: return launch_tile<128, kLoss, kGrad, kDH>(grid, s, x, tp, st);
-    case 192: return launch_tile<192, kLoss, kGrad, kDH>(grid, s, x, tp, st);
-    case 256: return launch_tile<256, kLoss, kGrad, kDH>(grid, s, x, tp, st);
+    case 64: return launch_tile<64, kLoss, kGrad, kDH, kMet>(grid, s, x, tp, st);
+    case 128: return launch_tile<128, kLoss, kGrad, kDH, kMet>(grid, s, x, tp, st);
+    case 192: return launch_tile<192, kLoss, kGrad, kDH, kMet>(grid, s, x, tp, st);
+    case 256: return launch_tile<256, kLoss, kGrad, kDH, kMet>(grid, s, x, tp, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -297,21 +344,24 @@ int count_launches(const Plan& pl, Want w) {
   int n = 3;                                            // rows, scan, gather
   if (bf16 && w.dE) n += 1 + 3 * pl.radix_passes + 1;   // sort keys, radix passes, item-tile offsets
   if (w.loss || w.dE) n += 1;                           // item-owned pass
-  if (w.dH) n += 1;                                     // position-owned pass
-  if (w.loss || w.dH) n += 1;                           // finish
+  if (w.dH || w.met) n += 1;                            // position-owned pass (dH and/or metrics)
+  if (w.loss || w.dH || w.met) n += 1;                  // finish
   return n;
 }
 
 // after_item: if not null, recorded on `st` right after the item-owned pass,
 // the point from which dE is final.
-cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss, float* dH, float* dE, Want w,
-                  void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t after_item = nullptr) {
+cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss, void* dH, void* dE, Want w,
+                  void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t after_item = nullptr,
+                  Opts o = Opts{}) {
+  if (o.V_total == 0) o.V_total = p->V;   // not sharded
   cutbce_status s = check_problem(p, true);
   if (s != CUTBCE_OK) return s;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return CUTBCE_ERR_INVALID_ARG;
-  if (w.loss && loss == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  if ((w.loss && loss == nullptr) || (w.met && o.metrics == nullptr)) return CUTBCE_ERR_INVALID_ARG;
+  const bool weighted = o.weights != nullptr;
   Plan pl;
-  make_plan(p, w, pl);
+  make_plan(p, w, pl, weighted);
   if (ws_bytes < pl.total) return CUTBCE_ERR_WORKSPACE;
   DeviceFacts dev;
   if ((s = device_facts(dev)) != CUTBCE_OK) return s;
@@ -333,6 +383,8 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   int* cscoff = at<int>(ws, pl.o_cscoff);
   int* ghist = at<int>(ws, pl.o_ghist);
   float* dhpart = at<float>(ws, pl.o_dhpart);
+  int2* metpart = w.met ? at<int2>(ws, pl.o_metpart) : nullptr;
+  float* wc = weighted ? at<float>(ws, pl.o_wc) : nullptr;
 
 #define CUTBCE_CK(x)                           \
   do {                                         \
@@ -342,13 +394,14 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   CUTBCE_CK(cudaMemsetAsync(hdr, 0, 256, st));
   {
   LaunchScope ls(CUTBCE_KERNEL_PREP_ROWS, st);
-  k_prep_rows<<<static_cast<unsigned>(ceil_div(T, 128)), 128, 0, st>>>(p->targets, p->mask, T, K, V, ids, rowcnt,
-                                                                        hdr);
+  k_prep_rows<<<static_cast<unsigned>(ceil_div(T, 128)), 128, 0, st>>>(p->targets, p->mask, o.weights, T, K, V,
+                                                                        o.v_off, o.V_total, ids, rowcnt, hdr);
   CUTBCE_CK(cudaGetLastError());
   }
   {
   LaunchScope ls(CUTBCE_KERNEL_PREP_SCAN, st);
-  k_prep_scan<<<1, kScanThreads, 0, st>>>(p->mask, rowcnt, T, V, p->reduction, grad_loss, cidx, orig, rowptr, hdr);
+  k_prep_scan<<<1, kScanThreads, 0, st>>>(p->mask, o.weights, rowcnt, T, o.V_total, p->reduction, grad_loss, cidx,
+                                          orig, rowptr, hdr);
   CUTBCE_CK(cudaGetLastError());
   }
   {
@@ -356,16 +409,22 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   if (bf16) {
     k_prep_gather<__nv_bfloat16><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(p->H), static_cast<const __nv_bfloat16*>(p->E), D, pl.DP, K, pl.Tpad,
-        orig, ids, rowcnt, rowptr, hdr, at<__nv_bfloat16>(ws, pl.o_hc), pair_t, pair_v, cpart);
+        orig, ids, rowcnt, rowptr, hdr, o.weights, wc, at<__nv_bfloat16>(ws, pl.o_hc), pair_t, pair_v, cpart);
   } else {
     k_prep_gather<float><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
         static_cast<const float*>(p->H), static_cast<const float*>(p->E), D, pl.DP, K, pl.Tpad, orig, ids, rowcnt,
-        rowptr, hdr, at<float>(ws, pl.o_hc), pair_t, pair_v, cpart);
+        rowptr, hdr, o.weights, wc, at<float>(ws, pl.o_hc), pair_t, pair_v, cpart);
   }
   CUTBCE_CK(cudaGetLastError());
   }
 
-  const bool item_pass = w.loss || w.dE;
+  // With per-position weights the tensor-core path sums the loss in the
+  // position-owned pass (one weight per row there); the item-owned pass then
+  // computes dE only.  The fp32 path sums it per item with the column weights.
+  const bool loss_in_pos = bf16 && weighted && w.loss;
+  const bool item_loss = w.loss && !loss_in_pos;
+  const bool item_pass = item_loss || w.dE;
+  const bool pos_pass = w.dH || w.met || loss_in_pos;
   if (bf16) {
     const int* srt_key = pair_v;
     const int* srt_val = pair_t;
@@ -407,9 +466,13 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     tp.pair_v = pair_v;
     tp.tile_pair_off = cscoff;
     tp.tile_pairs = srt_val;
-    tp.dE = dE;
+    tp.dE = static_cast<float*>(dE);
+    tp.de_bf16 = o.grad_bf16 ? 1 : 0;
+    tp.de_acc = o.acc_dE ? 1 : 0;
+    tp.wc = wc;
     tp.loss_part = lpart;
     tp.dh_part = dhpart;
+    tp.met_part = metpart;
     tp.nsplit = pl.S;
     tp.tiles_per_split = pl.tps;
     tp.n_item_tiles_bn = pl.n_vtiles_bn;
@@ -423,13 +486,13 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
                                                            static_cast<int64_t>(kMaxCtas)}));
       cudaError_t e;
       LaunchScope ls(CUTBCE_KERNEL_ITEM_PASS, st);
-      if (w.loss && w.dE) e = launch_tile_dp<true, true, false>(pl.DP, grid, ms, mx, tp, st);
-      else if (w.loss) e = launch_tile_dp<true, false, false>(pl.DP, grid, ms, mx, tp, st);
+      if (item_loss && w.dE) e = launch_tile_dp<true, true, false>(pl.DP, grid, ms, mx, tp, st);
+      else if (item_loss) e = launch_tile_dp<true, false, false>(pl.DP, grid, ms, mx, tp, st);
       else e = launch_tile_dp<false, true, false>(pl.DP, grid, ms, mx, tp, st);
       CUTBCE_CK(e);
     }
     if (item_pass && after_item != nullptr) CUTBCE_CK(cudaEventRecord(after_item, st));
-    if (w.dH) {
+    if (pos_pass) {
       CUtensorMap ms, mx;
       if (!make_map(&ms, hc, pl.DP, pl.Tpad, pl.DP, kTileM) || !make_map(&mx, p->E, D, V, D, pl.BN))
         return CUTBCE_ERR_CUDA;
@@ -437,32 +500,65 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
       const int grid = static_cast<int>(
           std::min<int64_t>({static_cast<int64_t>(dev.sms), items_max, static_cast<int64_t>(kMaxCtas)}));
       LaunchScope ls(CUTBCE_KERNEL_POSITION_PASS, st);
-      CUTBCE_CK((launch_tile_dp<false, true, true>(pl.DP, grid, ms, mx, tp, st)));
+      const int kind = (loss_in_pos ? 4 : 0) | (w.dH ? 2 : 0) | (w.met ? 1 : 0);
+      cudaError_t e;
+      switch (kind) {
+        case 1: e = launch_tile_dp<false, false, true, true>(pl.DP, grid, ms, mx, tp, st); break;
+        case 2: e = launch_tile_dp<false, true, true, false>(pl.DP, grid, ms, mx, tp, st); break;
+        case 3: e = launch_tile_dp<false, true, true, true>(pl.DP, grid, ms, mx, tp, st); break;
+        case 4: e = launch_tile_dp<true, false, true, false>(pl.DP, grid, ms, mx, tp, st); break;
+        case 5: e = launch_tile_dp<true, false, true, true>(pl.DP, grid, ms, mx, tp, st); break;
+        case 6: e = launch_tile_dp<true, true, true, false>(pl.DP, grid, ms, mx, tp, st); break;
+        default: e = launch_tile_dp<true, true, true, true>(pl.DP, grid, ms, mx, tp, st); break;
+      }
+      CUTBCE_CK(e);
     }
   } else {
     const float* hc = at<float>(ws, pl.o_hc);
     if (item_pass) {
       LaunchScope ls(CUTBCE_KERNEL_ITEM_PASS, st);
       k_simt_items<<<static_cast<unsigned>(pl.n_vitems), 128, 0, st>>>(
-          hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, w.dE ? dE : nullptr,
-          w.loss ? lpart : nullptr);
+          hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, wc, w.dE ? dE : nullptr,
+          o.grad_bf16 ? 1 : 0, o.acc_dE ? 1 : 0, w.loss ? lpart : nullptr);
       CUTBCE_CK(cudaGetLastError());
     }
     if (item_pass && after_item != nullptr) CUTBCE_CK(cudaEventRecord(after_item, st));
-    if (w.dH) {
+    if (w.dH || w.met) {
       LaunchScope ls(CUTBCE_KERNEL_POSITION_PASS, st);
       k_simt_rows<<<static_cast<unsigned>(ceil_div(pl.Tpad, 128)), 128, 0, st>>>(
-          hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, dhpart);
+          hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, w.dH ? dhpart : nullptr, metpart);
       CUTBCE_CK(cudaGetLastError());
     }
   }
-  if (w.loss || w.dH) {
+  if (w.loss || w.dH || w.met) {
     const unsigned grid = static_cast<unsigned>(finish_grid(T, D));
+    FinishParams fp{};
+    fp.T = T;
+    fp.D = D;
+    fp.DP = pl.DP;
+    fp.S = pl.S;
+    fp.V = V;
+    fp.Tpad = pl.Tpad;
+    fp.cidx = cidx;
+    fp.dh_part = dhpart;
+    fp.dH = w.dH ? dH : nullptr;
+    fp.dh_bf16 = o.grad_bf16 ? 1 : 0;
+    fp.dh_acc = o.acc_dH ? 1 : 0;
+    fp.weights = o.weights;
+    fp.loss_part = lpart;
+    fp.n_loss_part = static_cast<int>(pl.n_vitems * kNumEpiWarps);
+    fp.loss_pos_splits = loss_in_pos ? pl.S : 0;
+    fp.corr_part = cpart;
+    fp.n_corr_part = static_cast<int>(pl.n_gather_blocks);
+    fp.blk_part = at<double>(ws, pl.o_fpart);
+    fp.loss = w.loss ? loss : nullptr;
+    fp.met_part = metpart;
+    fp.met_slots = pl.met_slots;
+    fp.metrics = w.met ? o.metrics : nullptr;
+    fp.row_cnt = rowcnt;
+    fp.hdr = hdr;
     LaunchScope ls(CUTBCE_KERNEL_FINISH, st);
-    k_finish<<<grid, kFinishThreads, 0, st>>>(T, D, pl.DP, pl.Tpad, pl.S, cidx, dhpart, w.dH ? dH : nullptr, lpart,
-                                             static_cast<int>(pl.n_vitems * kNumEpiWarps), cpart,
-                                             static_cast<int>(pl.n_gather_blocks), at<double>(ws, pl.o_fpart),
-                                             w.loss ? loss : nullptr, hdr);
+    k_finish<<<grid, kFinishThreads, 0, st>>>(fp);
     CUTBCE_CK(cudaGetLastError());
   }
 #undef CUTBCE_CK
@@ -569,8 +665,7 @@ cutbce_status cutbce_workspace_size(const cutbce_problem* prob, size_t* bytes) {
 }
 
 cutbce_status cutbce_workspace_size_for(const cutbce_problem* prob, int outputs, size_t* bytes) {
-  if (bytes == nullptr || outputs <= 0 || outputs > (CUTBCE_OUT_LOSS | CUTBCE_OUT_DH | CUTBCE_OUT_DE))
-    return CUTBCE_ERR_INVALID_ARG;
+  if (bytes == nullptr || outputs <= 0 || outputs > kAllOutputs) return CUTBCE_ERR_INVALID_ARG;
   const cutbce_status s = check_problem(prob, false);
   if (s != CUTBCE_OK) return s;
   Plan pl;
@@ -582,7 +677,7 @@ cutbce_status cutbce_workspace_size_for(const cutbce_problem* prob, int outputs,
 cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_bytes, double* loss,
                              cutbce_stream_t stream) {
   if (loss == nullptr) return CUTBCE_ERR_INVALID_ARG;
-  return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false}, ws, ws_bytes,
+  return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false, false}, ws, ws_bytes,
              reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -591,26 +686,51 @@ cutbce_status cutbce_forward_fixed_scratch(const cutbce_problem* prob, double* l
   cutbce_status s = check_problem(prob, true);
   if (s != CUTBCE_OK) return s;
   Plan pl;
-  make_plan(prob, Want{true, false, false}, pl);                   // the loss-only layout that run() uses
+  make_plan(prob, Want{true, false, false, false}, pl);                   // the loss-only layout that run() uses
   if (pl.total > kFixedScratchBytes) return CUTBCE_ERR_WORKSPACE;   // the problem needs more than the fixed array
   void* ws = nullptr;
   if ((s = fixed_scratch_ptr(&ws)) != CUTBCE_OK) return s;
-  return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false}, ws, kFixedScratchBytes,
+  return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false, false}, ws, kFixedScratchBytes,
              reinterpret_cast<cudaStream_t>(stream));
 }
 
 cutbce_status cutbce_backward(const cutbce_problem* prob, const float* grad_loss, float* dH, float* dE, void* ws,
                               size_t ws_bytes, cutbce_stream_t stream) {
   if (dH == nullptr && dE == nullptr) return CUTBCE_ERR_INVALID_ARG;
-  return run(prob, grad_loss, nullptr, dH, dE, Want{false, dE != nullptr, dH != nullptr}, ws, ws_bytes,
+  return run(prob, grad_loss, nullptr, dH, dE, Want{false, dE != nullptr, dH != nullptr, false}, ws, ws_bytes,
              reinterpret_cast<cudaStream_t>(stream));
 }
 
 cutbce_status cutbce_forward_backward(const cutbce_problem* prob, const float* grad_loss, double* loss, float* dH,
                                       float* dE, void* ws, size_t ws_bytes, cutbce_stream_t stream) {
   if (loss == nullptr && dH == nullptr && dE == nullptr) return CUTBCE_ERR_INVALID_ARG;
-  return run(prob, grad_loss, loss, dH, dE, Want{loss != nullptr, dE != nullptr, dH != nullptr}, ws, ws_bytes,
+  return run(prob, grad_loss, loss, dH, dE, Want{loss != nullptr, dE != nullptr, dH != nullptr, false}, ws, ws_bytes,
              reinterpret_cast<cudaStream_t>(stream));
+}
+
+cutbce_status cutbce_forward_backward_ex(const cutbce_problem* prob, const cutbce_options* opts,
+                                         const float* grad_loss, double* loss, void* dH, void* dE, void* ws,
+                                         size_t ws_bytes, cutbce_stream_t stream) {
+  cutbce_status s = check_problem(prob, false);
+  if (s != CUTBCE_OK) return s;
+  Opts o;
+  if ((s = resolve_opts(prob, opts, o)) != CUTBCE_OK) return s;
+  if (loss == nullptr && dH == nullptr && dE == nullptr && o.metrics == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  return run(prob, grad_loss, loss, dH, dE, Want{loss != nullptr, dE != nullptr, dH != nullptr, o.metrics != nullptr},
+             ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, o);
+}
+
+cutbce_status cutbce_workspace_size_ex(const cutbce_problem* prob, const cutbce_options* opts, int outputs,
+                                       size_t* bytes) {
+  if (bytes == nullptr || outputs <= 0 || outputs > kAllOutputs) return CUTBCE_ERR_INVALID_ARG;
+  cutbce_status s = check_problem(prob, false);
+  if (s != CUTBCE_OK) return s;
+  Opts o;
+  if ((s = resolve_opts(prob, opts, o)) != CUTBCE_OK) return s;
+  Plan pl;
+  make_plan(prob, want_from_mask(outputs), pl, o.weights != nullptr);
+  *bytes = pl.total;
+  return CUTBCE_OK;
 }
 
 cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes) {
@@ -659,7 +779,7 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   float* ddH = dH ? reinterpret_cast<float*>(b + hl.o_dH) : nullptr;
   float* ddE = dE ? reinterpret_cast<float*>(b + hl.o_dE) : nullptr;
   s = copied ? run(&dp, reinterpret_cast<const float*>(b + hl.o_grad), reinterpret_cast<double*>(b + hl.o_loss),
-                   ddH, ddE, Want{true, dE != nullptr, dH != nullptr}, b + hl.o_ws, pl.total, st, side.ev)
+                   ddH, ddE, Want{true, dE != nullptr, dH != nullptr, false}, b + hl.o_ws, pl.total, st, side.ev)
              : CUTBCE_ERR_CUDA;
   if (s != CUTBCE_OK) {
     cudaStreamSynchronize(st);   // no copy from or to the caller's host memory may still run on return
@@ -715,7 +835,8 @@ int cutbce_kernel_launches(const cutbce_problem* prob, int entry) {
   if (check_problem(prob, false) != CUTBCE_OK || entry < 0 || entry > 2) return -1;
   Plan pl;
   make_plan(prob, kWantAll, pl);
-  const Want w = entry == 0 ? Want{true, false, false} : entry == 1 ? Want{false, true, true} : Want{true, true, true};
+  const Want w = entry == 0 ? Want{true, false, false, false}
+                 : entry == 1 ? Want{false, true, true, false} : Want{true, true, true, false};
   return count_launches(pl, w);
 }
 

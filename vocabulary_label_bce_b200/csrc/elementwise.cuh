@@ -112,6 +112,13 @@ __device__ __forceinline__ float nonneg_mask(float t) {
   return r;
 }
 
+// 1 for every normal x > 0, 0 for x <= 0 (and for a subnormal x, flushed to 0).
+__device__ __forceinline__ float positive_mask(float x) {
+  float r;
+  asm("mul.rn.ftz.sat.f32 %0, %1, %2;" : "=f"(r) : "f"(x), "f"(0x1p126f));
+  return r;
+}
+
 // n / w for w = -nw in [1, 2]: linear minimax seed r0 = (24 - 8 w) / 17, then the
 // cubic step applied to the quotient: q = n r0 (1 + e + e^2), e = 1 - w r0, so
 // |q / (n / w) - 1| = |e|^3 <= (1/17)^3 = 2.1e-4.

@@ -13,16 +13,25 @@ namespace cutbce {
 __device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(status, 0, code); }
 
 // ------------------------------------------------------------------ prep: rows
+// A position is valid iff its mask entry is nonzero and its weight (when
+// per-position weights are given) is nonzero: a zero weight is padding.
+__device__ __forceinline__ bool position_valid(const uint8_t* __restrict__ mask, const float* __restrict__ weights,
+                                               int t) {
+  return (mask == nullptr || mask[t] != 0) && (weights == nullptr || weights[t] != 0.f);
+}
+
 // One thread per position t.  A valid row's ids become its positive set P_t
 // (section III-B: sparse [B,N,L] ids, no multi-hot tensor): -1 slots dropped,
-// repeats collapsed (y is 0/1), sorted ascending.  Ids of masked rows are ignored.
-__global__ void k_prep_rows(const int32_t* __restrict__ targets, const uint8_t* __restrict__ mask, int T,
-                            int K, int V, int* __restrict__ ids_out, int* __restrict__ row_cnt,
-                            WsHeader* hdr) {
+// repeats collapsed (y is 0/1), sorted ascending.  Ids of masked rows are
+// ignored.  With a vocabulary shard, ids are global: an id in [-1, V_total) but
+// outside [v_off, v_off + V) belongs to another shard and is dropped, and the
+// kept ids are made shard-local.
+__global__ void k_prep_rows(const int32_t* __restrict__ targets, const uint8_t* __restrict__ mask,
+                            const float* __restrict__ weights, int T, int K, int V, int64_t v_off, int64_t V_total,
+                            int* __restrict__ ids_out, int* __restrict__ row_cnt, WsHeader* hdr) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
-  const bool valid = mask == nullptr || mask[t] != 0;
-  if (!valid) {
+  if (!position_valid(mask, weights, t)) {
     row_cnt[t] = 0;
     return;
   }
@@ -31,12 +40,14 @@ __global__ void k_prep_rows(const int32_t* __restrict__ targets, const uint8_t* 
   bool bad = false;
   const int32_t* row = targets + static_cast<int64_t>(t) * K;
   for (int k = 0; k < K; ++k) {
-    const int id = row[k];
-    if (id == -1) continue;
-    if (id < -1 || id >= V) {
+    const int gid = row[k];
+    if (gid == -1) continue;
+    if (gid < -1 || gid >= V_total) {
       bad = true;
       continue;
     }
+    if (gid < v_off || gid >= v_off + V) continue;     // another shard's item
+    const int id = static_cast<int>(gid - v_off);
     int pos = n;
     while (pos > 0 && buf[pos - 1] > id) --pos;
     if (pos > 0 && buf[pos - 1] == id) continue;
@@ -52,12 +63,14 @@ __global__ void k_prep_rows(const int32_t* __restrict__ targets, const uint8_t* 
 
 // ------------------------------------------------------------------ prep: scan
 // One block.  Exclusive scans over t of valid[t] (compacted row index c) and of
-// |P_t| (pair offsets), then the normalisation s and the gradient scale g*s.
+// |P_t| (pair offsets), then the normalisation s and the gradient scale g*s
+// (V here is the whole vocabulary, for the per-element mean).
 constexpr int kScanThreads = 1024;
 constexpr int kScanItems = 8;
 
 __global__ void __launch_bounds__(kScanThreads) k_prep_scan(const uint8_t* __restrict__ mask,
-                                                            const int* __restrict__ row_cnt, int T, int V,
+                                                            const float* __restrict__ weights,
+                                                            const int* __restrict__ row_cnt, int T, int64_t V,
                                                             int reduction, const float* __restrict__ grad_loss,
                                                             int* __restrict__ cidx, int* __restrict__ orig,
                                                             int* __restrict__ row_ptr, WsHeader* hdr) {
@@ -75,7 +88,7 @@ __global__ void __launch_bounds__(kScanThreads) k_prep_scan(const uint8_t* __res
 #pragma unroll
     for (int i = 0; i < kScanItems; ++i) {
       const int t = base + tid * kScanItems + i;
-      const int v = (t < T && (mask == nullptr || mask[t] != 0)) ? 1 : 0;
+      const int v = (t < T && position_valid(mask, weights, t)) ? 1 : 0;
       const int c = (t < T) ? row_cnt[t] : 0;
       vloc[i] = v;
       cloc[i] = c;
@@ -157,15 +170,17 @@ __global__ void __launch_bounds__(kScanThreads) k_prep_scan(const uint8_t* __res
 // ------------------------------------------------------------------ prep: gather
 // One warp per compacted row c in [0, Tpad).  Copies h_t into the compacted,
 // zero-padded H_c (rows >= n_valid are zero so padded tiles contribute exactly
-// nothing to any gradient), writes the pair lists, and sums the sparse target
-// correction sum_{v in P_t} h_t . e_v of Eq. (2) in fp32 per pair, in a fixed
-// order, into one double per block.
+// nothing to any gradient), writes the pair lists and, with per-position
+// weights, the compacted weights (0 for the padded rows), and sums the sparse
+// target correction sum_{v in P_t} w_t h_t . e_v of Eq. (2) in fp32 per pair, in
+// a fixed order, into one double per block.
 template <typename TIn>
 __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, const TIn* __restrict__ E,
                                                      int D, int DP, int K, int64_t Tpad,
                                                      const int* __restrict__ orig, const int* __restrict__ ids,
                                                      const int* __restrict__ row_cnt,
                                                      const int* __restrict__ row_ptr, const WsHeader* hdr,
+                                                     const float* __restrict__ weights, float* __restrict__ wc,
                                                      TIn* __restrict__ Hc, int* __restrict__ pair_t,
                                                      int* __restrict__ pair_v, double* __restrict__ corr_part) {
   __shared__ double wsum[8];
@@ -175,8 +190,10 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
   double acc = 0.0;
   if (c < Tpad) {
     TIn* dst = Hc + c * DP;
+    if (wc != nullptr && lane == 0) wc[c] = c < nv ? weights[orig[c]] : 0.f;
     if (c < nv) {
       const int t = orig[c];
+      const double wt = weights != nullptr ? static_cast<double>(weights[t]) : 1.0;
       const TIn* src = H + static_cast<int64_t>(t) * D;
       for (int d = lane; d < DP; d += 32) dst[d] = d < D ? src[d] : TIn(0.0f);
       const int p0 = row_ptr[c];
@@ -192,7 +209,7 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
         for (int d = lane; d < D; d += 32) z = fmaf(static_cast<float>(src[d]), static_cast<float>(e[d]), z);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-        acc += static_cast<double>(z);
+        acc += wt * static_cast<double>(z);
       }
     } else {
       for (int d = lane; d < DP; d += 32) dst[d] = TIn(0.0f);
@@ -228,59 +245,109 @@ __device__ double block_sum_fixed(double v, double* red) {
   return r;
 }
 
-__global__ void __launch_bounds__(kFinishThreads) k_finish(
-    int T, int D, int DP, int64_t Tpad, int S, const int* __restrict__ cidx,
-    const float* __restrict__ dh_part, float* __restrict__ dH, const double* __restrict__ loss_part,
-    int n_loss_part, const double* __restrict__ corr_part, int n_corr_part, double* __restrict__ blk_part,
-    double* __restrict__ loss, WsHeader* hdr) {
+struct FinishParams {
+  int T, D, DP, S, V;
+  int64_t Tpad;
+  const int* cidx;            // [T] compacted row of each position, -1 if masked
+  const float* dh_part;       // [S, Tpad, DP] dH partials of the vocabulary splits
+  void* dH;                   // [T, D] output (fp32, or bf16 with dh_bf16), or null
+  int dh_bf16;                // dH is written as bf16 (round to nearest even)
+  int dh_acc;                 // dH += the gradient instead of dH = the gradient
+  const float* weights;       // [T] per-position weights (row t of dH scaled by w_t), or null
+  const double* loss_part;    // dense loss partials
+  int n_loss_part;            // their number, or (with loss_pos_splits > 0) computed from n_valid
+  int loss_pos_splits;        // > 0: the partials are per position-owned work item, splits x ceil(n_valid/128)
+  const double* corr_part;    // sparse correction partials
+  int n_corr_part;
+  double* blk_part;           // [2 * gridDim.x] per-block loss sums
+  double* loss;               // output, or null
+  const int2* met_part;       // [met_slots, Tpad] (count of x > 0, TP) partials, or null
+  int met_slots;
+  int32_t* metrics;           // [T, 4] output TP, FP, FN, TN, or null
+  const int* row_cnt;         // [T] distinct positives of each position
+  WsHeader* hdr;
+};
+
+__global__ void __launch_bounds__(kFinishThreads) k_finish(const FinishParams f) {
   __shared__ double red[kFinishThreads];
   __shared__ int ticket;
-  const float gs = hdr->grad_scale;
-  if (dH != nullptr) {
+  const float gs = f.hdr->grad_scale;
+  const int T = f.T, D = f.D;
+  if (f.dH != nullptr) {
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx < static_cast<int64_t>(T) * D) {
       const int t = static_cast<int>(idx / D);
       const int d = static_cast<int>(idx - static_cast<int64_t>(t) * D);
-      const int c = cidx[t];
+      const int c = f.cidx[t];
       float out = 0.f;
       if (c >= 0) {
         float acc = 0.f;
-        for (int s = 0; s < S; ++s) acc += dh_part[(static_cast<int64_t>(s) * Tpad + c) * DP + d];
-        out = acc * gs;
+        for (int s = 0; s < f.S; ++s) acc += f.dh_part[(static_cast<int64_t>(s) * f.Tpad + c) * f.DP + d];
+        out = __fmul_rn(acc, f.weights != nullptr ? __fmul_rn(gs, f.weights[t]) : gs);
       }
-      dH[idx] = out;
+      // accumulation adds the fp32 gradient as it would be written without it
+      if (f.dh_bf16) {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(f.dH) + idx;
+        if (f.dh_acc) out = __fadd_rn(out, __bfloat162float(*o));
+        *o = __float2bfloat16_rn(out);
+      } else {
+        float* o = static_cast<float*>(f.dH) + idx;
+        if (f.dh_acc) out = __fadd_rn(out, *o);
+        *o = out;
+      }
     }
   }
-  if (loss != nullptr) {
+  if (f.metrics != nullptr) {
+    // Cut Metrics of each position from the integer partials (exact, any order)
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+      const int c = f.cidx[t];
+      int4 out = make_int4(0, 0, 0, 0);
+      if (c >= 0) {
+        int cnt = 0, tp = 0;
+        for (int s = 0; s < f.met_slots; ++s) {
+          const int2 v = f.met_part[static_cast<int64_t>(s) * f.Tpad + c];
+          cnt += v.x;
+          tp += v.y;
+        }
+        const int fn = f.row_cnt[t] - tp;
+        out = make_int4(tp, cnt - tp, fn, f.V - cnt - fn);
+      }
+      reinterpret_cast<int4*>(f.metrics)[t] = out;
+    }
+  }
+  if (f.loss != nullptr) {
     // two levels, both in a fixed order: block b sums slice b of the partials
     // (coalesced, thread-strided, then a fixed tree), the last block to finish
     // sums the block results in block order
     const int nb = static_cast<int>(gridDim.x);
-    const int per_a = (n_loss_part + nb - 1) / nb, per_b = (n_corr_part + nb - 1) / nb;
+    const int n_loss_part = f.loss_pos_splits > 0
+                                ? f.loss_pos_splits * static_cast<int>(ceil_div(f.hdr->n_valid, kTileM)) * kNumEpiWarps
+                                : f.n_loss_part;
+    const int per_a = (n_loss_part + nb - 1) / nb, per_b = (f.n_corr_part + nb - 1) / nb;
     const int a0 = blockIdx.x * per_a, a1 = min(n_loss_part, a0 + per_a);
-    const int b0 = blockIdx.x * per_b, b1 = min(n_corr_part, b0 + per_b);
+    const int b0 = blockIdx.x * per_b, b1 = min(f.n_corr_part, b0 + per_b);
     double a = 0.0, b = 0.0;
-    for (int i = a0 + threadIdx.x; i < a1; i += blockDim.x) a += loss_part[i];
-    for (int i = b0 + threadIdx.x; i < b1; i += blockDim.x) b += corr_part[i];
+    for (int i = a0 + threadIdx.x; i < a1; i += blockDim.x) a += f.loss_part[i];
+    for (int i = b0 + threadIdx.x; i < b1; i += blockDim.x) b += f.corr_part[i];
     a = block_sum_fixed(a, red);
     b = block_sum_fixed(b, red);
     if (threadIdx.x == 0) {
-      blk_part[2 * blockIdx.x] = a;
-      blk_part[2 * blockIdx.x + 1] = b;
+      f.blk_part[2 * blockIdx.x] = a;
+      f.blk_part[2 * blockIdx.x + 1] = b;
       __threadfence();
-      ticket = atomicAdd(&hdr->finish_count, 1);
+      ticket = atomicAdd(&f.hdr->finish_count, 1);
     }
     __syncthreads();
     if (ticket == nb - 1) {
       __threadfence();
       double da = 0.0, db = 0.0;
       for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-        da += *reinterpret_cast<volatile double*>(blk_part + 2 * i);
-        db += *reinterpret_cast<volatile double*>(blk_part + 2 * i + 1);
+        da += *reinterpret_cast<volatile double*>(f.blk_part + 2 * i);
+        db += *reinterpret_cast<volatile double*>(f.blk_part + 2 * i + 1);
       }
       const double dense = block_sum_fixed(da, red);
       const double corr = block_sum_fixed(db, red);
-      if (threadIdx.x == 0) *loss = hdr->n_valid > 0 ? hdr->loss_scale * (dense - corr) : 0.0;
+      if (threadIdx.x == 0) *f.loss = f.hdr->n_valid > 0 ? f.hdr->loss_scale * (dense - corr) : 0.0;
     }
   }
 }
@@ -297,7 +364,8 @@ __device__ __forceinline__ float sigmoid_f32(float z) {
 __global__ void __launch_bounds__(128) k_simt_items(const float* __restrict__ Hc, const float* __restrict__ E,
                                                     int V, int D, const int* __restrict__ row_ptr,
                                                     const int* __restrict__ pair_v, const WsHeader* hdr,
-                                                    float* __restrict__ dE, double* __restrict__ loss_part) {
+                                                    const float* __restrict__ wc, void* __restrict__ dE, int de_bf16,
+                                                    int de_acc, double* __restrict__ loss_part) {
   __shared__ double red[128];
   const int v = blockIdx.x * 128 + threadIdx.x;
   const int nv = hdr->n_valid;
@@ -309,18 +377,32 @@ __global__ void __launch_bounds__(128) k_simt_items(const float* __restrict__ Hc
     const float* e = E + static_cast<int64_t>(v) * D;
     for (int c = 0; c < nv; ++c) {
       const float* h = Hc + static_cast<int64_t>(c) * D;
+      const float w = wc != nullptr ? wc[c] : 1.f;
       float z = 0.f;
       for (int d = 0; d < D; ++d) z = fmaf(h[d], e[d], z);
       float y = 0.f;
       for (int p = row_ptr[c]; p < row_ptr[c + 1]; ++p) y = pair_v[p] == v ? 1.f : y;
-      lsum += static_cast<double>(fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))));
+      lsum += static_cast<double>(w) * static_cast<double>(fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))));
       if (dE != nullptr) {
-        const float g = sigmoid_f32(z) - y;
+        const float g = w * (sigmoid_f32(z) - y);
         for (int d = 0; d < D; ++d) acc[d] = fmaf(g, h[d], acc[d]);
       }
     }
-    if (dE != nullptr)
-      for (int d = 0; d < D; ++d) dE[static_cast<int64_t>(v) * D + d] = acc[d] * gs;
+    if (dE != nullptr) {
+      for (int d = 0; d < D; ++d) {
+        const int64_t k = static_cast<int64_t>(v) * D + d;
+        float out = __fmul_rn(acc[d], gs);
+        if (de_bf16) {
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dE) + k;
+          if (de_acc) out = __fadd_rn(out, __bfloat162float(*o));
+          *o = __float2bfloat16_rn(out);
+        } else {
+          float* o = static_cast<float*>(dE) + k;
+          if (de_acc) out = __fadd_rn(out, *o);
+          *o = out;
+        }
+      }
+    }
   }
   if (loss_part != nullptr) {
     // same layout as the tensor-core path: kNumEpiWarps partials per 128-item tile
@@ -329,11 +411,12 @@ __global__ void __launch_bounds__(128) k_simt_items(const float* __restrict__ Hc
   }
 }
 
-// One thread per compacted row c: dH partial sum_v (s(x)-y) e_v over all items.
+// One thread per compacted row c: dH partial sum_v (s(x)-y) e_v over all items,
+// and/or the row's count of x > 0 and of positives with x > 0 (Cut Metrics).
 __global__ void __launch_bounds__(128) k_simt_rows(const float* __restrict__ Hc, const float* __restrict__ E,
                                                    int V, int D, const int* __restrict__ row_ptr,
                                                    const int* __restrict__ pair_v, const WsHeader* hdr,
-                                                   float* __restrict__ dh_part) {
+                                                   float* __restrict__ dh_part, int2* __restrict__ met_part) {
   const int c = blockIdx.x * 128 + threadIdx.x;
   if (c >= hdr->n_valid) return;
   float acc[kMaxDim];
@@ -341,6 +424,7 @@ __global__ void __launch_bounds__(128) k_simt_rows(const float* __restrict__ Hc,
   const float* h = Hc + static_cast<int64_t>(c) * D;
   int p = row_ptr[c];
   const int pend = row_ptr[c + 1];
+  int cnt = 0, tp = 0;
   for (int v = 0; v < V; ++v) {
     const float* e = E + static_cast<int64_t>(v) * D;
     float z = 0.f;
@@ -350,10 +434,16 @@ __global__ void __launch_bounds__(128) k_simt_rows(const float* __restrict__ Hc,
       y = 1.f;
       ++p;
     }
-    const float g = sigmoid_f32(z) - y;
-    for (int d = 0; d < D; ++d) acc[d] = fmaf(g, e[d], acc[d]);
+    cnt += z > 0.f ? 1 : 0;
+    tp += (z > 0.f && y > 0.f) ? 1 : 0;
+    if (dh_part != nullptr) {
+      const float g = sigmoid_f32(z) - y;
+      for (int d = 0; d < D; ++d) acc[d] = fmaf(g, e[d], acc[d]);
+    }
   }
-  for (int d = 0; d < D; ++d) dh_part[static_cast<int64_t>(c) * D + d] = acc[d];
+  if (dh_part != nullptr)
+    for (int d = 0; d < D; ++d) dh_part[static_cast<int64_t>(c) * D + d] = acc[d];
+  if (met_part != nullptr) met_part[c] = make_int2(cnt, tp);
 }
 
 // Zero a float buffer (used for dE when no position is valid).

@@ -73,9 +73,14 @@ struct TileParams {
   const int* pair_v;           // CSR by position: items of each row, ascending
   const int* tile_pair_off;    // [ceil(V/128) + 1] offsets into tile_pairs, one range per item tile
   const int* tile_pairs;       // pairs grouped by item tile, ascending position: (v mod 128) << 24 | t
-  float* dE;                   // item-owned pass output [V, D] (may be null when no gradient)
-  double* loss_part;           // item-owned pass: one double per (item tile, epilogue warp)
+  float* dE;                   // item-owned pass output [V, D] (fp32, or bf16 with de_bf16; null: no gradient)
+  int de_bf16;                 // dE is written as bf16 (round to nearest even)
+  int de_acc;                  // dE += the gradient instead of dE = the gradient
+  const float* wc;             // [Tpad] per-position weights of the compacted rows (0 past n_valid), or null
+  double* loss_part;           // one double per (work item, epilogue warp): item-owned pass without weights,
+                               // position-owned pass with weights
   float* dh_part;              // position-owned pass output [S, Tpad, DP]
+  int2* met_part;              // position-owned pass with metrics: [S, slabs, Tpad] (count of x > 0, TP)
   int nsplit;                  // position-owned pass: vocabulary splits S
   int tiles_per_split;         // streamed item tiles per split
   int n_item_tiles_bn;         // ceil(V / BN)
@@ -187,7 +192,7 @@ __device__ __forceinline__ uint32_t cursor_take_mask(RowCursor& rc, const int* _
   return mask;
 }
 
-template <int DP, bool kLoss, bool kGrad, bool kDH>
+template <int DP, bool kLoss, bool kGrad, bool kDH, bool kMet = false>
 __global__ void __launch_bounds__(kTileThreads, 1)
     k_tile(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmX, TileParams p) {
   using Cfg = TileCfg<DP, epi_groups<kDH>()>;
@@ -197,8 +202,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   constexpr int NZ = Cfg::NZ;
   constexpr uint32_t S_BYTES = Cfg::S_BYTES, X_BYTES = Cfg::X_BYTES;
   constexpr int ACC_COL = Cfg::ACC_COL;
-  static_assert(!kDH || (kGrad && !kLoss), "the position-owned pass computes dH only");
-  static_assert(kLoss || kGrad, "nothing to do");
+  static_assert(kLoss || kGrad || kMet, "nothing to do");
+  static_assert(!kMet || kDH, "the metrics are counted in the position-owned pass");
   constexpr float kLn2 = kLn2F;
 
   extern __shared__ uint8_t smem_raw[];
@@ -240,10 +245,13 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     // no valid position: dE = 0 and every item's loss is 0
     for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
       if (kLoss && threadIdx.x < kNumEpiWarps) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + threadIdx.x] = 0.0;
-      if (kGrad && p.dE != nullptr) {
+      if (kGrad && p.dE != nullptr && !p.de_acc) {
         const int64_t r0 = static_cast<int64_t>(i) * kTileM;
         const int64_t r1 = min(static_cast<int64_t>(p.V), r0 + kTileM);
-        for (int64_t k = r0 * p.D + threadIdx.x; k < r1 * p.D; k += blockDim.x) p.dE[k] = 0.f;
+        for (int64_t k = r0 * p.D + threadIdx.x; k < r1 * p.D; k += blockDim.x) {
+          if (p.de_bf16) reinterpret_cast<__nv_bfloat16*>(p.dE)[k] = __float2bfloat16_rn(0.f);
+          else p.dE[k] = 0.f;
+        }
       }
     }
     return;
@@ -348,6 +356,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       ItemInfo zit{}, git{};
       if (zi < n_items) zit = git = item_info<DP, kDH>(zi, n_valid, p);
       uint64_t idle_since = 0;
+      uint32_t idle_polls = 0;
       bool ok = true;
       while (ok && (zi < n_items || (kGrad && gi < n_items))) {
         bool progressed = false;
@@ -462,9 +471,13 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           }
         }
         // ---- bounded: give up if nothing became ready within the limit
+#ifndef CUTBCE_MMA_TIMER_EVERY
+#define CUTBCE_MMA_TIMER_EVERY 1
+#endif
         if (progressed) {
           idle_since = 0;
-        } else {
+          idle_polls = 0;
+        } else if (++idle_polls % CUTBCE_MMA_TIMER_EVERY == 0) {
           const uint64_t now = global_timer_ns();
           if (idle_since == 0) idle_since = now;
           int give_up = 0;
@@ -516,6 +529,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
       const int n = it.n_x;
       double item_acc = 0.0;
+      int met_cnt = 0, met_tp = 0;                // position-owned pass: this row's x > 0 count and TP
       // Positives (y = 1).  Position-owned pass: this thread's row (a position)
       // has at most K of them, walked with a forward cursor over its items.
       // Item-owned pass: the item tile's pairs, in ascending position, are
@@ -523,7 +537,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       RowCursor rc{0, 0, 0x7fffffff};
       int seg = 0, seg_end = 0;
       uint32_t win = 0xFFFFFFFFu;                 // item-owned pass: pairs seg .. seg + 31, one per lane
-      if (kGrad) {
+      if (kGrad || kMet) {
         if (kDH) {
           const int r = it.s_row0 + row;
           if (r < n_valid) cursor_init(rc, p.pair_v, __ldg(p.row_ptr + r), __ldg(p.row_ptr + r + 1), it.x_tile0 * BN);
@@ -619,20 +633,39 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_zfree + bz);
           }
-          const uint32_t mask = !kGrad ? 0u : kDH ? cursor_take_mask(rc, p.pair_v, key0 + col0)
-                                                 : (NCH == 1 || ch == 0) ? pmask[0] : pmask[NCH - 1];
-          const bool any_pos = kGrad && __any_sync(0xffffffffu, mask != 0u);
+          const uint32_t mask = !(kGrad || kMet) ? 0u
+                                : kDH ? cursor_take_mask(rc, p.pair_v, key0 + col0)
+                                      : (NCH == 1 || ch == 0) ? pmask[0] : pmask[NCH - 1];
+          const bool any_pos = (kGrad || kMet) && __any_sync(0xffffffffu, mask != 0u);
+          float2 mcnt = f2(0.f, 0.f);             // metrics: x > 0 in this chunk (two lanes of a sum)
+          float mtp = 0.f;                        // metrics: positives with x > 0 in this chunk
           uint32_t pk[CH / 2];
           float2 prod = f2(1.f, 1.f), relu = f2(0.f, 0.f);
           // the chunk's element math; the y = 1 subtraction is compiled into a
           // separate copy taken only by chunks that hold a positive (rare), so
           // the common path has no per-element branch or bit test
-          auto chunk_math = [&](auto with_y) {
+          // column weights (item-owned pass with per-position weights): G = w (sigmoid - y)
+          const float* wcol = (!kDH && kGrad) ? p.wc : nullptr;
+          const int wcol0 = j * BN + col0;        // compacted position of this chunk's first column
+          auto chunk_math = [&](auto with_y, auto with_w) {
 #pragma unroll
             for (int e = 0; e < CH; e += 2) {
               const float2 z = f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
               float2 g = f2(0.f, 0.f);
-              if (kLoss && kGrad) {
+              float2 mpos = f2(0.f, 0.f);
+              if (kMet) {
+                // [x > 0] on the FMA pipe: saturate(x * 2^126) is 1 for every normal x > 0 and
+                // 0 for x <= 0 (a subnormal x is flushed to 0 and counts as not positive)
+                mpos = f2(positive_mask(z.x), positive_mask(z.y));
+                mcnt = __fadd2_rn(mcnt, mpos);
+                if (decltype(with_y)::value) {
+                  if (mask & (1u << e)) mtp += mpos.x;
+                  if (mask & (1u << (e + 1))) mtp += mpos.y;
+                }
+              }
+              if (!kLoss && !kGrad) {
+                // metrics only: no element math beyond the count
+              } else if (kLoss && kGrad) {
                 g = CUTBCE_ITEM_MATH == 0 ? bce_pair_loss_grad(z, prod, relu) : bce_pair_loss_grad_mask(z, prod, relu);
               } else if (kLoss) {
                 bce_pair_loss(z, prod, relu);
@@ -652,12 +685,22 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                   if (mask & (1u << e)) g.x -= 1.f;                // a predicated add, no conversion
                   if (mask & (1u << (e + 1))) g.y -= 1.f;
                 }
+                if (decltype(with_w)::value) g = __fmul2_rn(g, __ldg(reinterpret_cast<const float2*>(wcol + wcol0 + e)));
                 pk[e >> 1] = pack_bf16x2(g.x, g.y);
               }
             }
           };
-          if (any_pos) chunk_math(std::true_type{});
-          else chunk_math(std::false_type{});
+          if (wcol != nullptr) {
+            if (any_pos) chunk_math(std::true_type{}, std::true_type{});
+            else chunk_math(std::false_type{}, std::true_type{});
+          } else {
+            if (any_pos) chunk_math(std::true_type{}, std::false_type{});
+            else chunk_math(std::false_type{}, std::false_type{});
+          }
+          if (kMet) {
+            met_cnt += static_cast<int>(mcnt.x + mcnt.y);     // exact: at most CH
+            met_tp += static_cast<int>(mtp);
+          }
           if (kLoss) {
             // CH / 2 factors per component: the product of the -(1 + u) factors is positive
             tile_l2 += lg2_approx(prod.x * prod.y);
@@ -677,11 +720,18 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           if (lane == 0) mbar_arrive(bar_gready + bz);   // this warp's part of G is in place
         }
         if (kLoss) {
-          if (j == n - 1) {
+          if (!kDH && j == n - 1) {
             // zero rows of H_c past n_valid give z = 0 exactly: each adds log2(2) = 1 to tile_l2
             const int t0 = j * BN;
             const int lo = slab * ZC, hi = lo + ZC;
             const int pad = hi - max(min(n_valid - t0, hi), lo);
+            tile_l2 -= static_cast<float>(pad);
+          }
+          if (kDH && it.x_tile0 + j == p.n_item_tiles_bn - 1) {
+            // item rows past V in the last streamed tile are zero-filled: z = 0, log2(2) = 1 each
+            const int v0 = (it.x_tile0 + j) * BN;
+            const int lo = slab * ZC, hi = lo + ZC;
+            const int pad = hi - max(min(p.V - v0, hi), lo);
             tile_l2 -= static_cast<float>(pad);
           }
           item_acc += static_cast<double>(tile_mx + tile_l2 * kLn2);
@@ -690,10 +740,19 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       if (!ok) break;
       if (kLoss) {
         // one partial per (item tile, epilogue warp): no cross-warp barrier, fixed summation order
-        double val = (it.s_row0 + row < p.V) ? item_acc : 0.0;
+        // item-owned pass: rows past V are padding; position-owned pass: the row's
+        // loss times its weight (0 for the compacted rows past n_valid)
+        double val = kDH ? item_acc * static_cast<double>(__ldg(p.wc + it.s_row0 + row))
+                         : ((it.s_row0 + row < p.V) ? item_acc : 0.0);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
         if (lane == 0) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + ew] = val;
+      }
+      if (kMet) {
+        // one partial per (split, column slab, row), summed in a fixed order by the finish kernel;
+        // every group writes its own slab's counts, so with two groups the slabs of both are summed
+        const int slot = (it.split * Cfg::GROUPS + static_cast<int>(grp)) * Cfg::SLABS + slab;
+        p.met_part[static_cast<int64_t>(slot) * p.Tpad + it.s_row0 + row] = make_int2(met_cnt, met_tp);
       }
       if (kGrad && (cnt + n - 1) % Cfg::GROUPS == grp) {
         // the group that took the item's last tile reads the accumulator out
@@ -708,13 +767,36 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           if (!kDH) {
             const int v = it.s_row0 + row;
             if (v < p.V && p.dE != nullptr) {
-              float* dst = p.dE + static_cast<int64_t>(v) * p.D + col0;
+              const int64_t o = static_cast<int64_t>(v) * p.D + col0;
 #pragma unroll
-              for (int e = 0; e < 16; e += 4)
-                if (col0 + e < p.D)
-                  *reinterpret_cast<float4*>(dst + e) =
-                      make_float4(__uint_as_float(r[e]) * gs, __uint_as_float(r[e + 1]) * gs,
-                                  __uint_as_float(r[e + 2]) * gs, __uint_as_float(r[e + 3]) * gs);
+              for (int e = 0; e < 16; e += 4) {
+                if (col0 + e < p.D) {
+                  // the fp32 gradient, rounded as written without accumulation (no fused multiply-add)
+                  float4 g4 = make_float4(__fmul_rn(__uint_as_float(r[e]), gs), __fmul_rn(__uint_as_float(r[e + 1]), gs),
+                                          __fmul_rn(__uint_as_float(r[e + 2]), gs), __fmul_rn(__uint_as_float(r[e + 3]), gs));
+                  if (p.de_bf16) {
+                    uint2* dst = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dE) + o + e);
+                    if (p.de_acc) {
+                      const uint2 old = *dst;
+                      g4.x = __fadd_rn(g4.x, __uint_as_float(old.x << 16));
+                      g4.y = __fadd_rn(g4.y, __uint_as_float(old.x & 0xFFFF0000u));
+                      g4.z = __fadd_rn(g4.z, __uint_as_float(old.y << 16));
+                      g4.w = __fadd_rn(g4.w, __uint_as_float(old.y & 0xFFFF0000u));
+                    }
+                    *dst = make_uint2(pack_bf16x2(g4.x, g4.y), pack_bf16x2(g4.z, g4.w));
+                  } else {
+                    float4* dst = reinterpret_cast<float4*>(p.dE + o + e);
+                    if (p.de_acc) {
+                      const float4 old = *dst;
+                      g4.x = __fadd_rn(g4.x, old.x);
+                      g4.y = __fadd_rn(g4.y, old.y);
+                      g4.z = __fadd_rn(g4.z, old.z);
+                      g4.w = __fadd_rn(g4.w, old.w);
+                    }
+                    *dst = g4;
+                  }
+                }
+              }
             }
           } else {
             float* dst = p.dh_part + (static_cast<int64_t>(it.split) * p.Tpad + it.s_row0 + row) * DP + col0;
