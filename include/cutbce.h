@@ -345,6 +345,14 @@ cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratc
 /* Human-readable name of a status code (static storage). */
 const char* cutbce_status_string(cutbce_status status);
 
+/* Self-test of the element math: for each of the n device floats x[i], writes
+ * out[i] = 2^x[i] by the FMA-pipe polynomial the gradient-only passes use for
+ * part of their exponentials (valid for x in [-100, 100]), out[n + i] = 2^x[i]
+ * by the SFU (ex2.approx), and out[2n + i], out[3n + i] = the gradient-only
+ * sigmoid of z = x[i] with the exponential from the polynomial and from the
+ * SFU.  out: device float [4n].  Asynchronous on `stream`. */
+cutbce_status cutbce_selftest_exp2(const float* x, float* out, int64_t n, cutbce_stream_t stream);
+
 /* Self-test of the bounded-wait machinery the kernels use: launches one CTA
  * that waits on a shared-memory barrier nothing will ever signal, with a
  * limit of limit_ns nanoseconds.  The wait gives up, writes CUTBCE_ERR_TIMEOUT

@@ -63,3 +63,67 @@ def test_seed_alone_is_within_five_percent():
     r0 = (SEED_NEG - nw.view(np.uint32)).astype(np.uint32).view(np.float32)
     rel = np.abs(1.0 - w.astype(np.float64) * r0.astype(np.float64))
     assert rel.max() <= 0.0506, rel.max()
+
+
+# ---------------------------------------------------------------- FMA-pipe exponential of the gradient-only passes
+# The same float32 operations as exp2_poly3_pair and sigmoid_pair (each fused
+# multiply-add rounded once; the integer exponent insertion as a 32-bit
+# multiply-add), replayed over the clamped input range.
+POLY3 = [np.float32(v) for v in (0.9999280572, 0.6932609677, 0.2426111251, 0.0551716685)]
+SHIFT = np.float32(12582912.0)            # 1.5 * 2^23
+LOG2E = np.float32(1.4426950408889634)
+
+
+def add32(a, b):
+    return (np.asarray(a, np.float32).astype(np.float64) + np.asarray(b, np.float32).astype(np.float64)).astype(np.float32)
+
+
+def exp2_poly3(x):
+    x = np.asarray(x, np.float32)
+    j = add32(x, SHIFT)
+    jr = add32(j, -SHIFT)
+    f = fma32(jr, np.float32(-1.0), x)
+    p = fma32(np.full_like(f, POLY3[3]), f, np.full_like(f, POLY3[2]))
+    p = fma32(p, f, np.full_like(f, POLY3[1]))
+    p = fma32(p, f, np.full_like(f, POLY3[0]))
+    bits = (j.view(np.uint32).astype(np.uint64) * (1 << 23) + p.view(np.uint32).astype(np.uint64)) & 0xFFFFFFFF
+    return bits.astype(np.uint32).view(np.float32)
+
+
+def sat(v):
+    return np.clip(v, np.float32(0.0), np.float32(1.0)).astype(np.float32)
+
+
+def sigmoid_pair(z, poly):
+    z = np.asarray(z, np.float32)
+    a = sat(fma32(z, np.float32(-LOG2E / np.float32(200.0)), np.float32(0.5)))
+    x = fma32(a, np.float32(200.0), np.float32(-100.0))
+    v = exp2_poly3(x) if poly else np.exp2(x.astype(np.float64)).astype(np.float32)
+    nw = fma32(v, np.float32(-1.0), np.float32(-1.0))
+    return rcp_cubic(-nw)
+
+
+def test_exp2_poly3_bound():
+    x = np.linspace(-100.0, 100.0, 2000001).astype(np.float32)
+    got = exp2_poly3(x).astype(np.float64)
+    rel = np.abs(got / np.exp2(x.astype(np.float64)) - 1.0)
+    assert np.all(np.isfinite(got))
+    assert rel.max() <= 7.6e-5, rel.max()
+    # the polynomial's own fit, without the range reduction, at its extremes
+    f = np.linspace(-0.5, 0.5, 100001).astype(np.float32)
+    assert np.abs(exp2_poly3(f).astype(np.float64) / np.exp2(f.astype(np.float64)) - 1).max() <= 7.6e-5
+
+
+def test_gradient_only_sigmoid_bound():
+    z = np.concatenate([np.linspace(-69.0, 69.0, 400001), np.linspace(-8.0, 8.0, 200001)]).astype(np.float32)
+    ref = 1.0 / (1.0 + np.exp(-z.astype(np.float64)))
+    for poly in (False, True):
+        got = sigmoid_pair(z, poly).astype(np.float64)
+        rel = np.abs(got / ref - 1.0)
+        # clamp 4e-6 relative in 2^x (at most that in sigmoid) + 2^x (7.5e-5 with the polynomial,
+        # the SFU's own error in the kernel) + reciprocal 1.3e-4
+        assert rel.max() <= (2.1e-4 if poly else 1.4e-4), (poly, rel.max())
+    # beyond the clamp the result stays positive and tiny instead of underflowing to garbage
+    far = sigmoid_pair(np.array([-80.0, -500.0, -3e38], np.float32), True)
+    assert np.all(far > 0) and np.all(far < 1e-29)
+    assert np.all(sigmoid_pair(np.array([80.0, 3e38], np.float32), True) > np.float32(0.9998))

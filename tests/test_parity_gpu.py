@@ -220,3 +220,23 @@ def test_canary_guards_untouched(outputs):
            "dH": dH.cpu().numpy().astype(np.float64) if dH is not None else None,
            "dE": dE.cpu().numpy().astype(np.float64) if dE is not None else None}
     check_against_oracle(p, got, "mean")
+
+
+def test_fma_pipe_exponential_on_the_device():
+    # the device polynomial equals its float32 host replay bit for bit, and both
+    # exponential paths stay within their bounds of 2^x
+    from test_elementwise_bounds import exp2_poly3, sigmoid_pair
+    x = np.linspace(-100.0, 100.0, 1 << 20).astype(np.float32)
+    out = B.cutbce_selftest_exp2(torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    poly, sfu, sig_poly, sig_sfu = (out[k].cpu().numpy() for k in range(4))
+    assert np.array_equal(poly.view(np.uint32), exp2_poly3(x).view(np.uint32))
+    ref = np.exp2(x.astype(np.float64))
+    assert np.max(np.abs(poly / ref - 1.0)) <= 7.6e-5
+    assert np.max(np.abs(sfu / ref - 1.0)) <= 2.0 ** -20
+    z = np.linspace(-60.0, 60.0, 1 << 18).astype(np.float32)
+    out = B.cutbce_selftest_exp2(torch.from_numpy(z).cuda())
+    sref = 1.0 / (1.0 + np.exp(-z.astype(np.float64)))
+    assert np.max(np.abs(out[2].cpu().numpy() / sref - 1.0)) <= 2.1e-4
+    assert np.max(np.abs(out[3].cpu().numpy() / sref - 1.0)) <= 1.4e-4
+    assert np.array_equal(out[2].cpu().numpy().view(np.uint32), sigmoid_pair(z, True).view(np.uint32))

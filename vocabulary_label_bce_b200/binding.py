@@ -23,7 +23,7 @@ __all__ = [
     "cutbce_backward", "cutbce_forward_backward",
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
-    "cutbce_selftest_wait_timeout", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
+    "cutbce_selftest_wait_timeout", "cutbce_selftest_exp2", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
     "KERNEL_KINDS", "cutbce_probe_scratch_bytes", "cutbce_probe_pipe_rate", "PROBES", "cutbce_probe_mma",
 ]
 
@@ -97,6 +97,7 @@ _SIGS = {
     "cutbce_kernel_launches": (ctypes.c_int, [_P, ctypes.c_int]),
     "cutbce_status_string": (ctypes.c_char_p, [_i32]),
     "cutbce_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
+    "cutbce_selftest_exp2": (_i32, [_vp, _vp, _i64, _vp]),
     "cutbce_profile_enable": (_i32, [ctypes.c_int]),
     "cutbce_profile_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64), ctypes.c_int]),
     "cutbce_probe_scratch_bytes": (_sz, []),
@@ -269,6 +270,16 @@ def cutbce_status_string(status: int) -> str:
 def cutbce_selftest_wait_timeout(limit_ns: int, status_dev: torch.Tensor, stream=None) -> None:
     _check(load_library().cutbce_selftest_wait_timeout(int(limit_ns), status_dev.data_ptr(), _stream(stream)),
            "cutbce_selftest_wait_timeout")
+
+
+def cutbce_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """[4, n] device tensor: FMA-pipe 2^x, SFU 2^x, gradient-only sigmoid(x) by each (see include/cutbce.h)."""
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 tensor")
+    out = torch.empty((4, x.numel()), dtype=torch.float32, device=x.device)
+    _check(load_library().cutbce_selftest_exp2(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)),
+           "cutbce_selftest_exp2")
+    return out
 
 
 def cutbce_profile_enable(enable: bool) -> None:

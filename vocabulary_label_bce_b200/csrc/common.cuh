@@ -28,14 +28,8 @@ constexpr int kNumEpiWarps = 16;      // groups x (4 TMEM lane quarters x column
 // Epilogue groups taking tiles in turn: two for the item-owned pass (one
 // group's tile handshakes overlap the other's math), one for the
 // position-owned pass (all 16 warps on every tile).
-#ifndef CUTBCE_POS_GROUPS
-#define CUTBCE_POS_GROUPS 1
-#endif
-#ifndef CUTBCE_ITEM_GROUPS
-#define CUTBCE_ITEM_GROUPS 2
-#endif
 template <bool kDH>
-__host__ __device__ constexpr int epi_groups() { return kDH ? CUTBCE_POS_GROUPS : CUTBCE_ITEM_GROUPS; }
+__host__ __device__ constexpr int epi_groups() { return kDH ? 1 : 2; }
 
 // First 256 bytes of the workspace.
 struct WsHeader {

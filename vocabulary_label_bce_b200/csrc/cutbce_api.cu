@@ -982,6 +982,13 @@ const char* cutbce_status_string(cutbce_status s) {
   return "unknown status";
 }
 
+cutbce_status cutbce_selftest_exp2(const float* x, float* out, int64_t n, cutbce_stream_t stream) {
+  if (x == nullptr || out == nullptr || n <= 0 || n > (int64_t(1) << 30)) return CUTBCE_ERR_INVALID_ARG;
+  k_selftest_exp2<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, out, n);
+  return cudaGetLastError() == cudaSuccess ? CUTBCE_OK : CUTBCE_ERR_CUDA;
+}
+
 cutbce_status cutbce_selftest_wait_timeout(int64_t limit_ns, int32_t* status_dev, cutbce_stream_t stream) {
   if (status_dev == nullptr || limit_ns <= 0 || limit_ns > 10000000000LL) return CUTBCE_ERR_INVALID_ARG;
   k_selftest_wait<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, status_dev);

@@ -23,6 +23,9 @@
 // Both seeds are formed from -w, which the FMA pipe produces in the same
 // instruction as 1 + u (bits(-w) = bits(w) + 2^31 for the integer seed).
 //
+// Gradient-only passes move a share of their exponentials to the FMA pipe as
+// well (exp2_poly3_pair below).
+//
 // Packed fp32x2 instructions (two lanes of work per instruction) halve the
 // issue slots of the FMA-pipe part; the SFU and the selects stay scalar.
 #pragma once
@@ -81,71 +84,12 @@ __device__ __forceinline__ void bce_pair_loss(float2 z, float2& prod, float2& re
   relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
 }
 
-// Gradient only (the position-owned pass, and the item pass without the
-// loss): sigmoid(z) = 1 / (1 + 2^{-z log2 e}) over the whole range, the
-// exponent clamped at 100 (below z = -69.3 the result is 2^-100 instead of
-// a smaller positive number).  Seed and cubic step: |rel err| <= 1.3e-4 plus
-// rounding, well inside the bf16 rounding of G that follows (up to 2^-9).
-__device__ __forceinline__ float2 sigmoid_pair(float2 z) {
-  const float2 tz = __fmul2_rn(z, f2(-kLog2eF, -kLog2eF));
-  const float2 u = f2(ex2_approx(fminf(tz.x, 100.f)), ex2_approx(fminf(tz.y, 100.f)));
-  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + u)
-  return rcp2_cubic(nw);
-}
-
-// ---------------------------------------------------------------- variants under measurement
-#ifndef CUTBCE_ITEM_MATH
-#define CUTBCE_ITEM_MATH 0
-#endif
-#ifndef CUTBCE_POS_MATH
-#define CUTBCE_POS_MATH 0
-#endif
-#ifndef CUTBCE_POS_POLY_PAIRS
-#define CUTBCE_POS_POLY_PAIRS 0
-#endif
-
-// 1 for t >= 0, 0 for t < 0, on the FMA pipe: saturate(t * 2^100 + 1).  Only for
-// |t| < 2^-100 is the result strictly between 0 and 1.
-__device__ __forceinline__ float nonneg_mask(float t) {
-  float r;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(t), "f"(0x1p100f), "f"(1.0f));
-  return r;
-}
-
-// 1 for every normal x > 0, 0 for x <= 0 (and for a subnormal x, flushed to 0).
+// 1 for every normal x > 0, 0 for x <= 0 (and for a subnormal x, flushed to 0):
+// the Cut Metrics decision, on the FMA pipe.
 __device__ __forceinline__ float positive_mask(float x) {
   float r;
   asm("mul.rn.ftz.sat.f32 %0, %1, %2;" : "=f"(r) : "f"(x), "f"(0x1p126f));
   return r;
-}
-
-// n / w for w = -nw in [1, 2]: linear minimax seed r0 = (24 - 8 w) / 17, then the
-// cubic step applied to the quotient: q = n r0 (1 + e + e^2), e = 1 - w r0, so
-// |q / (n / w) - 1| = |e|^3 <= (1/17)^3 = 2.1e-4.
-__device__ __forceinline__ float2 quot2_unit_interval(float2 n, float2 nw) {
-  const float2 r = __ffma2_rn(nw, f2(8.f / 17.f, 8.f / 17.f), f2(24.f / 17.f, 24.f / 17.f));
-  const float2 e = __ffma2_rn(nw, r, f2(1.f, 1.f));
-  const float2 t = __ffma2_rn(e, e, e);
-  const float2 q = __fmul2_rn(n, r);
-  return __ffma2_rn(q, t, q);
-}
-
-// Item-owned pass, select-free: the sign of z enters through the FMA-pipe mask
-// s = [z >= 0], which also forms max(z, 0) = z s in one packed FMA.
-__device__ __forceinline__ float2 bce_pair_loss_grad_mask(float2 z, float2& prod, float2& relu) {
-  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
-  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));   // e^{-|z|}
-  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));           // -(1 + u)
-  prod = __fmul2_rn(prod, nw);
-  const float2 s = f2(nonneg_mask(tz.x), nonneg_mask(tz.y));
-  relu = __ffma2_rn(z, s, relu);
-#if CUTBCE_ITEM_MATH == 2
-  const float2 n = f2(fmaxf(u.x, s.x), fmaxf(u.y, s.y));                     // 1 (z >= 0) or u
-#else
-  const float2 omu = __ffma2_rn(u, f2(-1.f, -1.f), f2(1.f, 1.f));            // 1 - u
-  const float2 n = __ffma2_rn(s, omu, u);                                    // 1 (z >= 0) or u
-#endif
-  return quot2_unit_interval(n, nw);
 }
 
 // 2^x for x in [-100, 100] on the FMA pipe: x = j + f with j = rint(x) taken from
@@ -153,7 +97,8 @@ __device__ __forceinline__ float2 bce_pair_loss_grad_mask(float2 z, float2& prod
 // polynomial fitted by a Remez exchange for minimum relative error on
 // [-1/2, 1/2] (max relative error 7.5e-5, float32 Horner included); the
 // exponent j is added to the result's exponent field with one integer
-// multiply-add (bits(j_shifted) * 2^23 keeps j's low 9 bits, two's complement).
+// multiply-add (bits(x + 1.5 * 2^23) * 2^23 keeps j's low 9 bits, two's
+// complement, and the polynomial's exponent is -1 or 0).
 __device__ __forceinline__ float2 exp2_poly3_pair(float2 x) {
   constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
   const float2 j = __fadd2_rn(x, f2(kShift, kShift));
@@ -168,12 +113,23 @@ __device__ __forceinline__ float2 exp2_poly3_pair(float2 x) {
   return f2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
-// Gradient only, saturating clamp on the FMA pipe: x = clamp(-z log2 e, -100, 100)
-// formed as 200 * saturate(-z log2 e / 200 + 1/2) - 100 (error <= 200 * 2^-25 in x,
-// 4e-6 relative in 2^x), then sigmoid = 1 / (1 + 2^x) with the exponent-flip
-// seed and the cubic step.  kPoly: 2^x on the FMA pipe instead of the SFU.
+// Pairs of every 16 (one 32-logit chunk) whose exponential the gradient-only
+// passes evaluate on the FMA pipe instead of the SFU.  The SFU retires 16
+// exponentials per clock per SM and the polynomial costs about four more issue
+// slots than the SFU instruction, so only a small share moves (the best of
+// 0, 1, 2, 3 and 4 of 16 measured on the position-owned pass).
+constexpr int kPolyPairsPerChunk = 2;
+
+// Gradient only (the position-owned pass, and the item pass without the loss):
+// sigmoid(z) = 1 / (1 + 2^x), x = -z log2 e clamped to [-100, 100] as
+// 200 * saturate(-z log2 e / 200 + 1/2) - 100 on the FMA pipe (error <= 200 *
+// 2^-25 in x, 4e-6 relative in 2^x); below z = -69.3 the result is 2^-100
+// instead of a smaller positive number.  2^x from the SFU, or (kPoly) from the
+// FMA-pipe polynomial; then the exponent-flip seed and the cubic step
+// (|rel err| <= 1.3e-4).  Total relative error <= 2.1e-4 plus rounding, well
+// inside the bf16 rounding of G that follows (up to 2^-9).
 template <bool kPoly>
-__device__ __forceinline__ float2 sigmoid_pair_sat(float2 z) {
+__device__ __forceinline__ float2 sigmoid_pair(float2 z) {
   float ax, ay;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ax) : "f"(z.x), "f"(-kLog2eF / 200.f), "f"(0.5f));
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ay) : "f"(z.y), "f"(-kLog2eF / 200.f), "f"(0.5f));
@@ -181,15 +137,6 @@ __device__ __forceinline__ float2 sigmoid_pair_sat(float2 z) {
   const float2 v = kPoly ? exp2_poly3_pair(x) : f2(ex2_approx(x.x), ex2_approx(x.y));
   const float2 nw = __ffma2_rn(v, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + v)
   return rcp2_cubic(nw);
-}
-
-// Gradient only, symmetric form: u = 2^{-|z| log2 e}, n = [z >= 0] or u, q = n / (1 + u).
-__device__ __forceinline__ float2 sigmoid_pair_sym(float2 z) {
-  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
-  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));
-  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));
-  const float2 n = f2(fmaxf(u.x, nonneg_mask(tz.x)), fmaxf(u.y, nonneg_mask(tz.y)));
-  return quot2_unit_interval(n, nw);
 }
 
 }  // namespace cutbce

@@ -356,7 +356,6 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       ItemInfo zit{}, git{};
       if (zi < n_items) zit = git = item_info<DP, kDH>(zi, n_valid, p);
       uint64_t idle_since = 0;
-      uint32_t idle_polls = 0;
       bool ok = true;
       while (ok && (zi < n_items || (kGrad && gi < n_items))) {
         bool progressed = false;
@@ -471,13 +470,9 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           }
         }
         // ---- bounded: give up if nothing became ready within the limit
-#ifndef CUTBCE_MMA_TIMER_EVERY
-#define CUTBCE_MMA_TIMER_EVERY 1
-#endif
         if (progressed) {
           idle_since = 0;
-          idle_polls = 0;
-        } else if (++idle_polls % CUTBCE_MMA_TIMER_EVERY == 0) {
+        } else {
           const uint64_t now = global_timer_ns();
           if (idle_since == 0) idle_since = now;
           int give_up = 0;
@@ -666,19 +661,13 @@ __global__ void __launch_bounds__(kTileThreads, 1)
               if (!kLoss && !kGrad) {
                 // metrics only: no element math beyond the count
               } else if (kLoss && kGrad) {
-                g = CUTBCE_ITEM_MATH == 0 ? bce_pair_loss_grad(z, prod, relu) : bce_pair_loss_grad_mask(z, prod, relu);
+                g = bce_pair_loss_grad(z, prod, relu);
               } else if (kLoss) {
                 bce_pair_loss(z, prod, relu);
+              } else if (((e >> 1) * kPolyPairsPerChunk) % 16 < kPolyPairsPerChunk) {
+                g = sigmoid_pair<true>(z);          // exponential on the FMA pipe (a few pairs, spread evenly)
               } else {
-#if CUTBCE_POS_MATH == 0
-                g = sigmoid_pair(z);
-#elif CUTBCE_POS_MATH == 1
-                // CUTBCE_POS_POLY_PAIRS of the 16 pairs of a chunk, spread evenly, on the FMA pipe
-                if (((e >> 1) * CUTBCE_POS_POLY_PAIRS) % 16 < CUTBCE_POS_POLY_PAIRS) g = sigmoid_pair_sat<true>(z);
-                else g = sigmoid_pair_sat<false>(z);
-#else
-                g = sigmoid_pair_sym(z);
-#endif
+                g = sigmoid_pair<false>(z);         // exponential on the SFU
               }
               if (kGrad) {
                 if (decltype(with_y)::value) {                     // y = 1 at the masked columns
@@ -821,6 +810,19 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
+}
+
+// Element-math self test: for each x, the FMA-pipe 2^x, the SFU 2^x and the
+// gradient-only sigmoid of z = x (both exponential paths).  Used only by
+// cutbce_selftest_exp2.
+__global__ void k_selftest_exp2(const float* __restrict__ x, float* __restrict__ out, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float v = x[i];
+  out[i] = exp2_poly3_pair(f2(v, v)).x;
+  out[n + i] = ex2_approx(v);
+  out[2 * n + i] = sigmoid_pair<true>(f2(v, v)).x;
+  out[3 * n + i] = sigmoid_pair<false>(f2(v, v)).x;
 }
 
 // A deliberately unsignalled barrier: the bounded wait must give up, record the
