@@ -341,3 +341,42 @@ def metrics_from_counts(counts: np.ndarray, beta: float = 1.0) -> dict:
     fbeta = (1.0 + b2) * precision * recall / denom if denom > 0 else 0.0
     return {"accuracy": (tp + tn) / total if total > 0 else 0.0, "precision": precision, "recall": recall,
             "fbeta": fbeta}
+
+
+# ---------------------------------------------------------------- full-vocabulary top-k and Hit@k (section III-E)
+# Evaluation: a query (the hidden state of a sequence's last non-pad position)
+# is scored against every item, x_v = q . e_v; the k highest scores rank the
+# items; a query is a hit if at least one of its held-out target ids is among
+# them (Hit@8 in the pages: k = 8, 8 held-out items).  Reading where the pages
+# are silent: items are ranked by descending score, equal scores by ascending
+# id; -1 marks an empty target slot; a query with no target is not a hit.
+
+def topk(Q: np.ndarray, E: np.ndarray, k: int, chunk: int = 65536):
+    """(ids int64 [B, k], scores float64 [B, k]): the k best items of each query."""
+    Q64 = np.asarray(Q, dtype=np.float64)
+    B, V = Q64.shape[0], E.shape[0]
+    k = min(k, V)
+    best_s = np.full((B, 0), -np.inf)
+    best_i = np.zeros((B, 0), dtype=np.int64)
+    for c0 in range(0, V, chunk):
+        c1 = min(V, c0 + chunk)
+        S = Q64 @ np.asarray(E[c0:c1], dtype=np.float64).T
+        cand_s = np.concatenate([best_s, S], axis=1)
+        cand_i = np.concatenate([best_i, np.broadcast_to(np.arange(c0, c1), S.shape)], axis=1)
+        kk = min(k, cand_s.shape[1])                             # the first chunks may hold fewer than k
+        keep_s = np.empty((B, kk))
+        keep_i = np.empty((B, kk), dtype=np.int64)
+        for b in range(B):
+            order = np.lexsort((cand_i[b], -cand_s[b]))[:kk]     # score descending, then id ascending
+            keep_s[b] = cand_s[b, order]
+            keep_i[b] = cand_i[b, order]
+        best_s, best_i = keep_s, keep_i
+    return best_i, best_s
+
+
+def hit_at_k(topk_ids: np.ndarray, targets: np.ndarray) -> np.ndarray:
+    """int64 [B]: 1 if a target id (>= 0) of the query is among its top-k ids."""
+    ids = np.asarray(topk_ids)
+    tg = np.asarray(targets)
+    return np.array([int(np.any(np.isin(tg[b][tg[b] >= 0], ids[b]))) for b in range(ids.shape[0])],
+                    dtype=np.int64)
