@@ -256,6 +256,30 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
                                            void* dev_buf, size_t dev_bytes,
                                            cutbce_stream_t stream);
 
+/* Full-vocabulary ranking for evaluation (section III-E: the hidden state of a
+ * sequence's last non-pad position is scored against every item; Hit@8 asks
+ * whether one of the held-out items is among the 8 best).
+ *
+ * Q: [B, D] bf16 queries, E: [V, D] bf16 items (device, row-major, 16-byte
+ * aligned; D a multiple of 8, at most 256), 1 <= k <= 16.  Writes, for each
+ * query b, the k best items by the score x_bv = q_b . e_v (fp32 accumulation of
+ * the bf16 products on the tensor cores) in descending score, equal scores in
+ * ascending id: ids int32 [B, k] (-1 when V < k), scores float [B, k].  No
+ * [B, V] score array is written anywhere: every score tile lives in tensor
+ * memory until per-thread running top-k lists have taken it in.  ws: device
+ * workspace of cutbce_topk_workspace_size bytes, 256-byte aligned, whose first
+ * bytes hold the status word (cutbce_read_status).  dtype must be CUTBCE_BF16.
+ * Asynchronous on `stream`. */
+cutbce_status cutbce_topk_workspace_size(int64_t B, int64_t V, int64_t D, int k, size_t* bytes);
+cutbce_status cutbce_topk(const void* Q, int64_t B, const void* E, int64_t V, int64_t D, int32_t dtype, int k,
+                          int32_t* ids, float* scores, void* ws, size_t ws_bytes, cutbce_stream_t stream);
+
+/* Hit@k of ranked ids (e.g. from cutbce_topk): hits[b] = 1 if one of the target
+ * ids targets[b, 0..L) (-1 = empty slot) is among ids[b, 0..k), else 0.  All
+ * device arrays (ids int32 [B, k], targets int32 [B, L], hits int32 [B]). */
+cutbce_status cutbce_hit_at_k(const int32_t* ids, int64_t B, int k, const int32_t* targets, int64_t L, int32_t* hits,
+                              cutbce_stream_t stream);
+
 /* Synchronises `stream` and returns the device status word of the last call
  * that used this workspace (CUTBCE_OK, TARGET_RANGE or TIMEOUT). */
 cutbce_status cutbce_read_status(const void* ws, cutbce_stream_t stream);

@@ -23,7 +23,8 @@ __all__ = [
     "cutbce_backward", "cutbce_forward_backward",
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
-    "cutbce_selftest_wait_timeout", "cutbce_selftest_exp2", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
+    "cutbce_selftest_wait_timeout", "cutbce_selftest_exp2", "cutbce_topk_workspace_size", "cutbce_topk",
+    "cutbce_hit_at_k", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
     "KERNEL_KINDS", "cutbce_probe_scratch_bytes", "cutbce_probe_pipe_rate", "PROBES", "cutbce_probe_mma",
 ]
 
@@ -98,6 +99,9 @@ _SIGS = {
     "cutbce_status_string": (ctypes.c_char_p, [_i32]),
     "cutbce_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
     "cutbce_selftest_exp2": (_i32, [_vp, _vp, _i64, _vp]),
+    "cutbce_topk_workspace_size": (_i32, [_i64, _i64, _i64, ctypes.c_int, ctypes.POINTER(_sz)]),
+    "cutbce_topk": (_i32, [_vp, _i64, _vp, _i64, _i64, _i32, ctypes.c_int, _vp, _vp, _vp, _sz, _vp]),
+    "cutbce_hit_at_k": (_i32, [_vp, _i64, ctypes.c_int, _vp, _i64, _vp, _vp]),
     "cutbce_profile_enable": (_i32, [ctypes.c_int]),
     "cutbce_profile_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64), ctypes.c_int]),
     "cutbce_probe_scratch_bytes": (_sz, []),
@@ -280,6 +284,37 @@ def cutbce_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
     _check(load_library().cutbce_selftest_exp2(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)),
            "cutbce_selftest_exp2")
     return out
+
+
+def cutbce_topk_workspace_size(B: int, V: int, D: int, k: int) -> int:
+    n = _sz(0)
+    _check(load_library().cutbce_topk_workspace_size(int(B), int(V), int(D), int(k), ctypes.byref(n)),
+           "cutbce_topk_workspace_size")
+    return int(n.value)
+
+
+def cutbce_topk(Q: torch.Tensor, E: torch.Tensor, k: int, ws: Optional[torch.Tensor] = None, stream=None):
+    """(ids int32 [B, k], scores float32 [B, k]) of the k best items of every query row of Q (bf16 [B, D])."""
+    if Q.dtype != torch.bfloat16 or E.dtype != torch.bfloat16 or not (Q.is_contiguous() and E.is_contiguous()):
+        raise ValueError("Q and E must be contiguous bf16 tensors")
+    B, D = Q.shape
+    V = E.shape[0]
+    if ws is None:
+        ws = torch.empty(cutbce_topk_workspace_size(B, V, D, k), dtype=torch.uint8, device=Q.device)
+    ids = torch.empty((B, k), dtype=torch.int32, device=Q.device)
+    scores = torch.empty((B, k), dtype=torch.float32, device=Q.device)
+    _check(load_library().cutbce_topk(Q.data_ptr(), B, E.data_ptr(), V, D, BF16, int(k), ids.data_ptr(),
+                                      scores.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)), "cutbce_topk")
+    return ids, scores
+
+
+def cutbce_hit_at_k(ids: torch.Tensor, targets: torch.Tensor, stream=None) -> torch.Tensor:
+    """int32 [B]: 1 where one of the query's target ids (-1 = empty) is among its ranked ids."""
+    B, k = ids.shape
+    hits = torch.empty(B, dtype=torch.int32, device=ids.device)
+    _check(load_library().cutbce_hit_at_k(ids.data_ptr(), B, int(k), targets.data_ptr(), targets.shape[1],
+                                          hits.data_ptr(), _stream(stream)), "cutbce_hit_at_k")
+    return hits
 
 
 def cutbce_profile_enable(enable: bool) -> None:

@@ -15,7 +15,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcutbce.so")
 SOURCES = ["cutbce_api.cu"]
 DEPS = ["cutbce_api.cu", "common.cuh", "prep_finish.cuh", "pair_sort.cuh", "tile_engine.cuh", "ptx_sm100.cuh", "probes.cuh",
-        "elementwise.cuh"]
+        "elementwise.cuh", "topk.cuh"]
 
 
 def nvcc_path() -> str:

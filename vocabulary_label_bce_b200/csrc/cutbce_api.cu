@@ -20,6 +20,7 @@
 #include "pair_sort.cuh"
 #include "tile_engine.cuh"
 #include "probes.cuh"
+#include "topk.cuh"
 
 namespace {
 using namespace cutbce;
@@ -337,6 +338,73 @@ cudaError_t launch_tile_dp(int DP, int grid, const CUtensorMap& s, const CUtenso
     case 256: return launch_tile<256, kLoss, kGrad, kDH, kMet>(grid, s, x, tp, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// ---------------------------------------------------------------- top-k dispatch
+template <int DP, int KMAX>
+cudaError_t launch_topk(int grid, const CUtensorMap& q, const CUtensorMap& e, const TopkParams& tp,
+                        cudaStream_t st) {
+  auto kern = k_topk<DP, KMAX>;
+  constexpr uint32_t smem = TopkCfg<DP>::SMEM_BYTES;
+  static std::atomic<uint64_t> configured{0};   // the attribute belongs to the current device
+  int dev = 0;
+  cudaError_t e2 = cudaGetDevice(&dev);
+  if (e2 != cudaSuccess) return e2;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = uint64_t(1) << dev;
+  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
+    e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e2 != cudaSuccess) return e2;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  kern<<<grid, kTileThreads, smem, st>>>(q, e, tp);
+  return cudaGetLastError();
+}
+
+template <int KMAX>
+cudaError_t launch_topk_dp(int DP, int grid, const CUtensorMap& q, const CUtensorMap& e, const TopkParams& tp,
+                           cudaStream_t st) {
+  switch (DP) {
+    case 64: return launch_topk<64, KMAX>(grid, q, e, tp, st);
+    case 128: return launch_topk<128, KMAX>(grid, q, e, tp, st);
+    case 192: return launch_topk<192, KMAX>(grid, q, e, tp, st);
+    case 256: return launch_topk<256, KMAX>(grid, q, e, tp, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+struct TopkPlan {
+  int DP, BN, KMAX, n_qt, n_vtiles, S, tps;
+  size_t o_hdr, o_s, o_i, total;
+};
+
+cutbce_status topk_plan(int64_t B, int64_t V, int64_t D, int k, int sms, TopkPlan& tp) {
+  if (B <= 0 || V <= 0 || D <= 0 || k <= 0) return CUTBCE_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > kMaxDim || k > 16 || V >= (int64_t(1) << 31) || B >= (int64_t(1) << 24))
+    return CUTBCE_ERR_UNSUPPORTED;
+  tp.DP = static_cast<int>(round_up(D, 64));
+  tp.BN = tp.DP <= 128 ? 128 : 64;
+  tp.KMAX = k <= 8 ? 8 : 16;
+  tp.n_qt = static_cast<int>(ceil_div(B, kTileM));
+  tp.n_vtiles = static_cast<int>(ceil_div(V, tp.BN));
+  // about one work item per SM of a 148-SM part, every split non-empty; depends
+  // only on the sizes, so the merge order never depends on the device
+  (void)sms;
+  const int64_t s0 = std::max<int64_t>(1, std::min<int64_t>(tp.n_vtiles, ceil_div(148, tp.n_qt)));
+  tp.tps = static_cast<int>(ceil_div(tp.n_vtiles, s0));
+  tp.S = static_cast<int>(ceil_div(tp.n_vtiles, tp.tps));
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  const size_t n = static_cast<size_t>(tp.n_qt) * tp.S * 4 * kTileM * tp.KMAX;
+  tp.o_hdr = take(256);
+  tp.o_s = take(4 * n);
+  tp.o_i = take(4 * n);
+  tp.total = o;
+  return CUTBCE_OK;
 }
 
 int count_launches(const Plan& pl, Want w) {
@@ -800,6 +868,67 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   if (dE != nullptr) give_side_stream(side);
   if (!ok || !sync_ok) return CUTBCE_ERR_CUDA;
   return static_cast<cutbce_status>(dev_status);
+}
+
+cutbce_status cutbce_topk_workspace_size(int64_t B, int64_t V, int64_t D, int k, size_t* bytes) {
+  if (bytes == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  TopkPlan tp;
+  const cutbce_status s = topk_plan(B, V, D, k, 148, tp);
+  if (s != CUTBCE_OK) return s;
+  *bytes = tp.total;
+  return CUTBCE_OK;
+}
+
+cutbce_status cutbce_topk(const void* Q, int64_t B, const void* E, int64_t V, int64_t D, int32_t dtype, int k,
+                          int32_t* ids, float* scores, void* ws, size_t ws_bytes, cutbce_stream_t stream) {
+  if (Q == nullptr || E == nullptr || ids == nullptr || scores == nullptr || ws == nullptr) return CUTBCE_ERR_INVALID_ARG;
+  if (dtype != CUTBCE_BF16) return CUTBCE_ERR_UNSUPPORTED;
+  if (((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(E)) & 15) != 0 ||
+      (reinterpret_cast<uintptr_t>(ws) & 255) != 0)
+    return CUTBCE_ERR_INVALID_ARG;
+  DeviceFacts dev;
+  cutbce_status s = device_facts(dev);
+  if (s != CUTBCE_OK) return s;
+  TopkPlan pl;
+  if ((s = topk_plan(B, V, D, k, dev.sms, pl)) != CUTBCE_OK) return s;
+  if (ws_bytes < pl.total) return CUTBCE_ERR_WORKSPACE;
+  if (!(dev.major == 10 && dev.minor == 0)) return CUTBCE_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap mq, me;
+  if (!make_map(&mq, Q, D, B, D, kTileM) || !make_map(&me, E, D, V, D, pl.BN)) return CUTBCE_ERR_CUDA;
+  TopkParams tp{};
+  tp.B = static_cast<int>(B);
+  tp.V = static_cast<int>(V);
+  tp.n_qt = pl.n_qt;
+  tp.nsplit = pl.S;
+  tp.tiles_per_split = pl.tps;
+  tp.n_vtiles = pl.n_vtiles;
+  tp.cand_s = at<float>(ws, pl.o_s);
+  tp.cand_i = at<int>(ws, pl.o_i);
+  tp.hdr = at<WsHeader>(ws, pl.o_hdr);
+  tp.timeout_ns = kDefaultTimeoutNs;
+  if (cudaMemsetAsync(tp.hdr, 0, 256, st) != cudaSuccess) return CUTBCE_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(dev.sms),
+                                                       static_cast<int64_t>(pl.n_qt) * pl.S, kMaxCtas}));
+  cudaError_t e = pl.KMAX == 8 ? launch_topk_dp<8>(pl.DP, grid, mq, me, tp, st)
+                               : launch_topk_dp<16>(pl.DP, grid, mq, me, tp, st);
+  if (e != cudaSuccess) return CUTBCE_ERR_CUDA;
+  const unsigned mgrid = static_cast<unsigned>(ceil_div(B * 32, 256));
+  if (pl.KMAX == 8)
+    k_topk_merge<8><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+  else
+    k_topk_merge<16><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+  return cudaGetLastError() == cudaSuccess ? CUTBCE_OK : CUTBCE_ERR_CUDA;
+}
+
+cutbce_status cutbce_hit_at_k(const int32_t* ids, int64_t B, int k, const int32_t* targets, int64_t L, int32_t* hits,
+                              cutbce_stream_t stream) {
+  if (ids == nullptr || targets == nullptr || hits == nullptr || B <= 0 || k <= 0 || L <= 0)
+    return CUTBCE_ERR_INVALID_ARG;
+  if (B >= (int64_t(1) << 31) || L >= (int64_t(1) << 20) || k > 16) return CUTBCE_ERR_UNSUPPORTED;
+  k_hit_at_k<<<static_cast<unsigned>(ceil_div(B, 256)), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      ids, static_cast<int>(B), k, targets, static_cast<int>(L), hits);
+  return cudaGetLastError() == cudaSuccess ? CUTBCE_OK : CUTBCE_ERR_CUDA;
 }
 
 cutbce_status cutbce_read_status(const void* ws, cutbce_stream_t stream) {
