@@ -50,6 +50,7 @@ def parse_args():
     ap.add_argument("--workload", default="sasrec_876k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the side measurements (metrics, top-8)")
     ap.add_argument("--cpu-sample-items", type=int, default=32768)
     ap.add_argument("--calls-only", type=int, default=0,
                     help="run this many untimed fused calls on --workload and exit (a target for ncu)")
@@ -377,6 +378,9 @@ def run_ours(args):
                "entry": "cutbce_forward_backward_host (pinned host H, E, targets, mask in; loss, dH, dE out)"}
         del buf
 
+    extras = measure_extras(B, p, prob, H, E, tg, loss, dH, dE, ws, flush, stream, dev) \
+        if (world == 1 and not args.no_extras) else None
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_items = min(p.V, args.cpu_sample_items)
@@ -410,12 +414,66 @@ def run_ours(args):
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "extras": extras,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _time_calls(fn, flush, stream, n=5):
+    """Mean CUDA-event time (ms) of n calls on `stream`, L2 flushed before each."""
+    import torch
+    fn()
+    ts = []
+    for _ in range(n):
+        flush.zero_()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn()
+        e.record(stream)
+        e.synchronize()
+        ts.append(s.elapsed_time(e))
+    return statistics.mean(ts)
+
+
+def measure_extras(B, p, prob, H, E, tg, loss, dH, dE, ws, flush, stream, dev):
+    """Side measurements after the timed region (not part of the step): the fused
+    step with Cut Metrics on against the plain step, and full-vocabulary top-8
+    ranking (one query per sequence: its last valid position; and 8,192 queries)."""
+    import torch
+    plain = _time_calls(lambda: B.cutbce_forward_backward(prob, None, loss, dH, dE, ws, stream), flush, stream)
+    met = torch.empty((p.T, 4), dtype=torch.int32, device=dev)
+    opts = B.make_options(metrics=met)
+    bits = B.OUT_LOSS | B.OUT_DH | B.OUT_DE | B.OUT_METRICS
+    wsm = torch.empty(B.cutbce_workspace_size_ex(prob, opts, bits), dtype=torch.uint8, device=dev)
+    with_met = _time_calls(lambda: B.cutbce_forward_backward_ex(prob, opts, None, loss, dH, dE, wsm, stream),
+                           flush, stream)
+    if B.cutbce_read_status(wsm, stream) != 0:
+        raise SystemExit("device status after the metrics call")
+    del wsm
+    out = {"metrics_overhead": {"step_ms": plain, "step_with_metrics_ms": with_met,
+                                "overhead_ms": with_met - plain,
+                                "what": "cutbce_forward_backward_ex with per-position TP/FP/FN/TN"}}
+    mask = np.asarray(p.mask).reshape(p.B, p.N)
+    last = np.array([np.nonzero(mask[b])[0][-1] if mask[b].any() else 0 for b in range(p.B)])
+    Hq = H.view(p.B, p.N, p.D)
+    rows = {"one_per_sequence": Hq[torch.arange(p.B, device=dev), torch.from_numpy(last).to(dev)].contiguous(),
+            "8192_queries": H[torch.from_numpy(np.nonzero(p.mask)[0][:8192]).to(dev)].contiguous()}
+    out["topk"] = {}
+    for name, Q in rows.items():
+        k = 8
+        wst = torch.empty(B.cutbce_topk_workspace_size(Q.shape[0], p.V, p.D, k), dtype=torch.uint8, device=dev)
+        ms = _time_calls(lambda: B.cutbce_topk(Q, E, k, wst, stream), flush, stream)
+        if B.cutbce_read_status(wst, stream) != 0:
+            raise SystemExit("device status after the top-k call")
+        out["topk"][name] = {"queries": int(Q.shape[0]), "V": p.V, "k": k, "ms": ms,
+                             "queries_per_s": Q.shape[0] / (ms * 1e-3),
+                             "tflops": 2.0 * Q.shape[0] * p.V * p.D / (ms * 1e-3) / 1e12}
+    return out
 
 
 def run_calls_only(args):

@@ -359,23 +359,32 @@ cutbce_status cutbce_probe_pipe_rate(int op, void* scratch, size_t scratch_bytes
 
 /* Tensor-core probe: on every SM one thread issues `iters` bf16 tcgen05.mma
  * instructions of shape 128 x n x 16 (n = 64, 128 or 256; fp32 accumulator in
- * tensor memory; A from shared memory, or from tensor memory if bit 0 of
- * a_in_tmem is set; B K-major, or MN-major if bit 1 is set) and waits for them.  Writes the median over SMs of the cycles per instruction
- * spent issuing and until completion (the dense ideal on B200 is n/2 cycles).
+ * tensor memory) and waits for them.  flags: bit 0, A from tensor memory
+ * (else shared memory); bit 1, B MN-major (else K-major); bit 2, SM pairs:
+ * 2-CTA clusters whose even CTA issues tcgen05.mma.cta_group::2 of shape
+ * 256 x n x 16 (each CTA holds 128 rows of A and half of B; B K-major only).
+ * Writes the median over issuing CTAs of the cycles per instruction spent
+ * issuing and until completion (the dense ideal on B200 is n/2 cycles per
+ * 128 x n x 16 on one SM, the same per 256 x n x 16 on a pair).
  * Synchronises `stream`. */
-cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratch, size_t scratch_bytes,
+cutbce_status cutbce_probe_mma(int n, int flags, int64_t iters, void* scratch, size_t scratch_bytes,
                                double* issue_cycles_per_mma, double* cycles_per_mma, cutbce_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* cutbce_status_string(cutbce_status status);
 
-/* Self-test of the element math: for each of the n device floats x[i], writes
- * out[i] = 2^x[i] by the FMA-pipe polynomial the gradient-only passes use for
- * part of their exponentials (valid for x in [-100, 100]), out[n + i] = 2^x[i]
- * by the SFU (ex2.approx), and out[2n + i], out[3n + i] = the gradient-only
- * sigmoid of z = x[i] with the exponential from the polynomial and from the
- * SFU.  out: device float [4n].  Asynchronous on `stream`. */
-cutbce_status cutbce_selftest_exp2(const float* x, float* out, int64_t n, cutbce_stream_t stream);
+/* Self-test of the element math the tile kernels run ("Cut Binary Cross
+ * Entropy" section III-A Eq. (2) and section III-B Eq. (4)): for each of the n
+ * device floats x[i], writes
+ *   out[i]      = 2^x[i] by the FMA-pipe polynomial (valid for x in [-100, 100]);
+ *   out[n + i]  = 2^x[i] by the SFU (ex2.approx);
+ *   out[2n + i] = sigmoid(x[i]) as the gradient-only passes form it on the FMA
+ *                 pipe alone (that polynomial, a seed and a cubic reciprocal step);
+ *   out[3n + i] = sigmoid(x[i]) from the SFU's tanh, (1 + tanh(x/2)) / 2;
+ *   out[4n + i] = w = 1 + |tanh(x[i]/2)| = 2 sigmoid(|x[i]|), the factor whose
+ *                 log gives the loss in the passes that form loss and gradient.
+ * out: device float [5n].  Asynchronous on `stream`. */
+cutbce_status cutbce_selftest_element_math(const float* x, float* out, int64_t n, cutbce_stream_t stream);
 
 /* Self-test of the bounded-wait machinery the kernels use: launches one CTA
  * that waits on a shared-memory barrier nothing will ever signal, with a

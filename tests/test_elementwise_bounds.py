@@ -1,14 +1,14 @@
-"""Host-side check of the reciprocals the tile engine uses for the sigmoid.
+"""Host-side replay of the FMA-pipe element math of the tile engine.
 
-The kernels compute 1/w on the FMA pipe instead of the SFU: a seed, then one
-cubically convergent step r1 = r0 (1 + e + e^2), e = 1 - w r0.
-  * item pass, w in (1, 2]: linear minimax seed r0 = (24 - 8 w) / 17, one
-    fused multiply-add on -w; bound (1/17)^3 = 2.1e-4;
-  * gradient-only passes, w up to 2^100: exponent-flip seed
-    r0 = bits^-1(C - bits(w)), C = 0x7EF31000 (formed from -w, whose bits are
-    bits(w) + 2^31); bound 1.3e-4.
-This test replays the same float32 operations (each fused multiply-add
-rounded once, as on the GPU) over the ranges the kernels use.
+The gradient-only passes evaluate one pair of logits in 16 wholly on the FMA
+pipe: 2^x by a degree-3 polynomial with integer exponent insertion, then 1/w
+by the exponent-flip seed r0 = bits^-1(C - bits(w)), C = 0x7EF31000 (formed
+from -w, whose bits are bits(w) + 2^31), and one cubically convergent step
+r1 = r0 (1 + e + e^2), e = 1 - w r0, which leaves |e|^3 <= 1.3e-4.
+These tests replay the same float32 operations (each fused multiply-add
+rounded once, as on the GPU) over the ranges the kernels use; the GPU test of
+the element-math self test checks the device against this replay bit for bit.
+The SFU paths (ex2, tanh) are checked on the device against their bounds.
 """
 import numpy as np
 
@@ -29,21 +29,9 @@ def rcp_cubic(w):
     return fma32(r, t, r)
 
 
-def rcp_linear_seed(w):
-    w = np.asarray(w, np.float32)
-    nw = -w
-    r = fma32(nw, np.float32(8.0 / 17.0), np.float32(24.0 / 17.0))
-    e = fma32(nw, r, np.float32(1.0))
-    t = fma32(e, e, e)
-    return fma32(r, t, r)
-
-
-def test_reciprocal_bound_item_range():
-    # item pass: w = 1 + e^{-|z|} in (1, 2]
+def test_reciprocal_bound_unit_range():
+    # w in (1, 2]
     w = np.linspace(1.0, 2.0, 400001, dtype=np.float32)[1:]
-    rel = np.abs(1.0 - w.astype(np.float64) * rcp_linear_seed(w).astype(np.float64))
-    assert rel.max() <= (1.0 / 17.0) ** 3 + 1e-6, rel.max()
-    # and the exponent-flip variant on the same range
     rel = np.abs(1.0 - w.astype(np.float64) * rcp_cubic(w).astype(np.float64))
     assert rel.max() <= 1.3e-4 + 1e-6, rel.max()
 
@@ -65,8 +53,8 @@ def test_seed_alone_is_within_five_percent():
     assert rel.max() <= 0.0506, rel.max()
 
 
-# ---------------------------------------------------------------- FMA-pipe exponential of the gradient-only passes
-# The same float32 operations as exp2_poly3_pair and sigmoid_pair (each fused
+# ---------------------------------------------------------------- FMA-pipe sigmoid of the gradient-only passes
+# The same float32 operations as exp2_poly3_pair and sigmoid_pair_fma (each fused
 # multiply-add rounded once; the integer exponent insertion as a 32-bit
 # multiply-add), replayed over the clamped input range.
 POLY3 = [np.float32(v) for v in (0.9999280572, 0.6932609677, 0.2426111251, 0.0551716685)]
@@ -94,11 +82,11 @@ def sat(v):
     return np.clip(v, np.float32(0.0), np.float32(1.0)).astype(np.float32)
 
 
-def sigmoid_pair(z, poly):
+def sigmoid_fma(z):
     z = np.asarray(z, np.float32)
     a = sat(fma32(z, np.float32(-LOG2E / np.float32(200.0)), np.float32(0.5)))
     x = fma32(a, np.float32(200.0), np.float32(-100.0))
-    v = exp2_poly3(x) if poly else np.exp2(x.astype(np.float64)).astype(np.float32)
+    v = exp2_poly3(x)
     nw = fma32(v, np.float32(-1.0), np.float32(-1.0))
     return rcp_cubic(-nw)
 
@@ -117,13 +105,11 @@ def test_exp2_poly3_bound():
 def test_gradient_only_sigmoid_bound():
     z = np.concatenate([np.linspace(-69.0, 69.0, 400001), np.linspace(-8.0, 8.0, 200001)]).astype(np.float32)
     ref = 1.0 / (1.0 + np.exp(-z.astype(np.float64)))
-    for poly in (False, True):
-        got = sigmoid_pair(z, poly).astype(np.float64)
-        rel = np.abs(got / ref - 1.0)
-        # clamp 4e-6 relative in 2^x (at most that in sigmoid) + 2^x (7.5e-5 with the polynomial,
-        # the SFU's own error in the kernel) + reciprocal 1.3e-4
-        assert rel.max() <= (2.1e-4 if poly else 1.4e-4), (poly, rel.max())
+    got = sigmoid_fma(z).astype(np.float64)
+    rel = np.abs(got / ref - 1.0)
+    # clamp 4e-6 relative in 2^x (at most that in sigmoid) + polynomial 7.5e-5 + reciprocal 1.3e-4
+    assert rel.max() <= 2.1e-4, rel.max()
     # beyond the clamp the result stays positive and tiny instead of underflowing to garbage
-    far = sigmoid_pair(np.array([-80.0, -500.0, -3e38], np.float32), True)
+    far = sigmoid_fma(np.array([-80.0, -500.0, -3e38], np.float32))
     assert np.all(far > 0) and np.all(far < 1e-29)
-    assert np.all(sigmoid_pair(np.array([80.0, 3e38], np.float32), True) > np.float32(0.9998))
+    assert np.all(sigmoid_fma(np.array([80.0, 3e38], np.float32)) > np.float32(0.9998))

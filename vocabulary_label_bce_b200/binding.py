@@ -23,7 +23,7 @@ __all__ = [
     "cutbce_backward", "cutbce_forward_backward",
     "cutbce_host_buffer_size", "cutbce_forward_backward_host", "cutbce_read_status",
     "cutbce_read_counts", "cutbce_kernel_launches", "cutbce_status_string",
-    "cutbce_selftest_wait_timeout", "cutbce_selftest_exp2", "cutbce_topk_workspace_size", "cutbce_topk",
+    "cutbce_selftest_wait_timeout", "cutbce_selftest_element_math", "cutbce_topk_workspace_size", "cutbce_topk",
     "cutbce_hit_at_k", "cutbce_profile_enable", "cutbce_profile_read", "REDUCTIONS",
     "KERNEL_KINDS", "cutbce_probe_scratch_bytes", "cutbce_probe_pipe_rate", "PROBES", "cutbce_probe_mma",
 ]
@@ -98,7 +98,7 @@ _SIGS = {
     "cutbce_kernel_launches": (ctypes.c_int, [_P, ctypes.c_int]),
     "cutbce_status_string": (ctypes.c_char_p, [_i32]),
     "cutbce_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
-    "cutbce_selftest_exp2": (_i32, [_vp, _vp, _i64, _vp]),
+    "cutbce_selftest_element_math": (_i32, [_vp, _vp, _i64, _vp]),
     "cutbce_topk_workspace_size": (_i32, [_i64, _i64, _i64, ctypes.c_int, ctypes.POINTER(_sz)]),
     "cutbce_topk": (_i32, [_vp, _i64, _vp, _i64, _i64, _i32, ctypes.c_int, _vp, _vp, _vp, _sz, _vp]),
     "cutbce_hit_at_k": (_i32, [_vp, _i64, ctypes.c_int, _vp, _i64, _vp, _vp]),
@@ -276,13 +276,14 @@ def cutbce_selftest_wait_timeout(limit_ns: int, status_dev: torch.Tensor, stream
            "cutbce_selftest_wait_timeout")
 
 
-def cutbce_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
-    """[4, n] device tensor: FMA-pipe 2^x, SFU 2^x, gradient-only sigmoid(x) by each (see include/cutbce.h)."""
+def cutbce_selftest_element_math(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """[5, n] device tensor: FMA-pipe 2^x, SFU 2^x, FMA-pipe sigmoid(x), sigmoid(x) from
+    tanh, and w = 1 + |tanh(x/2)| (see include/cutbce.h)."""
     if x.dtype != torch.float32 or not x.is_contiguous():
         raise ValueError("x must be a contiguous float32 tensor")
-    out = torch.empty((4, x.numel()), dtype=torch.float32, device=x.device)
-    _check(load_library().cutbce_selftest_exp2(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)),
-           "cutbce_selftest_exp2")
+    out = torch.empty((5, x.numel()), dtype=torch.float32, device=x.device)
+    _check(load_library().cutbce_selftest_element_math(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)),
+           "cutbce_selftest_element_math")
     return out
 
 
@@ -346,12 +347,13 @@ def cutbce_probe_pipe_rate(op: str | int, scratch: Optional[torch.Tensor] = None
 
 
 def cutbce_probe_mma(n: int, a_in_tmem: bool, iters: int = 4096, scratch: Optional[torch.Tensor] = None,
-                     stream=None, b_mn_major: bool = False) -> tuple[float, float]:
-    """(issue cycles, total cycles) per 128 x n x 16 bf16 tcgen05.mma, median over SMs."""
+                     stream=None, b_mn_major: bool = False, sm_pair: bool = False) -> tuple[float, float]:
+    """(issue cycles, total cycles) per 128 x n x 16 bf16 tcgen05.mma (256 x n x 16
+    over an SM pair if sm_pair), median over the issuing CTAs."""
     if scratch is None:
         scratch = torch.empty(cutbce_probe_scratch_bytes(), dtype=torch.uint8, device="cuda")
     a, b = ctypes.c_double(0.0), ctypes.c_double(0.0)
-    flags = (1 if a_in_tmem else 0) | (2 if b_mn_major else 0)
+    flags = (1 if a_in_tmem else 0) | (2 if b_mn_major else 0) | (4 if sm_pair else 0)
     _check(load_library().cutbce_probe_mma(int(n), flags, int(iters), scratch.data_ptr(),
                                            scratch.numel(), ctypes.byref(a), ctypes.byref(b), _stream(stream)),
            "cutbce_probe_mma")

@@ -1047,7 +1047,7 @@ cutbce_status cutbce_probe_pipe_rate(int op, void* scratch, size_t scratch_bytes
   return CUTBCE_OK;
 }
 
-cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratch, size_t scratch_bytes,
+cutbce_status cutbce_probe_mma(int n, int flags, int64_t iters, void* scratch, size_t scratch_bytes,
                                double* issue_cycles_per_mma, double* cycles_per_mma, cutbce_stream_t stream) {
   if ((n != 64 && n != 128 && n != 256) || iters <= 0 || iters > (1 << 24) || scratch == nullptr ||
       scratch_bytes < cutbce_probe_scratch_bytes() || issue_cycles_per_mma == nullptr || cycles_per_mma == nullptr)
@@ -1056,7 +1056,7 @@ cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratc
   cutbce_status s = device_facts(dev);
   if (s != CUTBCE_OK) return s;
   if (!(dev.major == 10 && dev.minor == 0)) return CUTBCE_ERR_UNSUPPORTED;
-  const int grid = std::min(dev.sms, kMaxCtas);
+  const int grid = std::min(dev.sms, kMaxCtas) & ~1;   // even: whole 2-CTA clusters for the pair probe
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto* out = static_cast<unsigned long long*>(scratch);
   const int smem = 1024 + 16384 + n * 128 + 16 * 2048;
@@ -1069,9 +1069,15 @@ cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratc
       e = cudaGetLastError();
     }
   };
-  const bool bmn = (a_in_tmem & 2) != 0;
-  const bool at = (a_in_tmem & 1) != 0;
-  if (n == 64) {
+  const bool bmn = (flags & 2) != 0;
+  const bool at = (flags & 1) != 0;
+  const bool pair = (flags & 4) != 0;
+  if (pair) {
+    if (bmn) return CUTBCE_ERR_INVALID_ARG;
+    if (n == 64) at ? launch(k_probe_mma_pair<64, true>) : launch(k_probe_mma_pair<64, false>);
+    else if (n == 128) at ? launch(k_probe_mma_pair<128, true>) : launch(k_probe_mma_pair<128, false>);
+    else at ? launch(k_probe_mma_pair<256, true>) : launch(k_probe_mma_pair<256, false>);
+  } else if (n == 64) {
     if (bmn) at ? launch(k_probe_mma<64, true, true>) : launch(k_probe_mma<64, false, true>);
     else at ? launch(k_probe_mma<64, true, false>) : launch(k_probe_mma<64, false, false>);
   } else if (n == 128) {
@@ -1086,15 +1092,16 @@ cutbce_status cutbce_probe_mma(int n, int a_in_tmem, int64_t iters, void* scratc
   if (cudaMemcpyAsync(h.data(), out, 16 * grid, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return CUTBCE_ERR_CUDA;
-  std::vector<unsigned long long> issue(grid), total(grid);
-  for (int b = 0; b < grid; ++b) {
-    issue[b] = h[2 * b];
-    total[b] = h[2 * b + 1];
+  // with SM pairs only the even CTA of each cluster issues and records
+  std::vector<unsigned long long> issue, total;
+  for (int b = 0; b < grid; b += pair ? 2 : 1) {
+    issue.push_back(h[2 * b]);
+    total.push_back(h[2 * b + 1]);
   }
   std::sort(issue.begin(), issue.end());
   std::sort(total.begin(), total.end());
-  *issue_cycles_per_mma = static_cast<double>(issue[grid / 2]) / static_cast<double>(iters);
-  *cycles_per_mma = static_cast<double>(total[grid / 2]) / static_cast<double>(iters);
+  *issue_cycles_per_mma = static_cast<double>(issue[issue.size() / 2]) / static_cast<double>(iters);
+  *cycles_per_mma = static_cast<double>(total[total.size() / 2]) / static_cast<double>(iters);
   return CUTBCE_OK;
 }
 
@@ -1111,9 +1118,9 @@ const char* cutbce_status_string(cutbce_status s) {
   return "unknown status";
 }
 
-cutbce_status cutbce_selftest_exp2(const float* x, float* out, int64_t n, cutbce_stream_t stream) {
+cutbce_status cutbce_selftest_element_math(const float* x, float* out, int64_t n, cutbce_stream_t stream) {
   if (x == nullptr || out == nullptr || n <= 0 || n > (int64_t(1) << 30)) return CUTBCE_ERR_INVALID_ARG;
-  k_selftest_exp2<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  k_selftest_element_math<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       x, out, n);
   return cudaGetLastError() == cudaSuccess ? CUTBCE_OK : CUTBCE_ERR_CUDA;
 }

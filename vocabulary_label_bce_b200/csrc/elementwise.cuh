@@ -1,33 +1,29 @@
 // Per-logit BCE math of the tile engine, two logits at a time.
 //
 // For a logit z (section III-A, Eq. (2) of "Cut Binary Cross Entropy"):
-//   u = e^{-|z|} in (0, 1],   w = 1 + u in (1, 2]
-//   l(z, 0) = max(z, 0) + log(1 + e^{-|z|}) = max(z, 0) + ln 2 * log2(w)
-//   sigmoid(z) = 1 / w  (z >= 0),   u / w  (z < 0)      (Eq. (4): G = sigmoid(Z) - Y)
+//   l(z, 0) = max(z, 0) + log(1 + e^{-|z|})
+//   sigmoid(z) = 1 / (1 + e^{-z})      (Eq. (4): G = sigmoid(Z) - Y)
 //
 // Pipe budget on B200 (measured with the library's pipe probes): the SFU
-// (ex2, rcp, lg2, tanh) retires 16 results per clock per SM, the FMA pipe 128,
-// so one SFU operation costs as much as eight FMAs.  Each logit therefore gets
-// exactly one SFU operation (the exponential); the reciprocal runs on the FMA
-// pipe, and the logarithm is taken once per 32 logits of a row as the log2 of
-// the product of their w (each factor is in (1, 2], so 32 of them stay finite).
+// (ex2, rcp, tanh, lg2) retires 16 results per clock per SM, the FMA pipe 128,
+// and the SM issues one warp instruction per clock per sub-partition, so a
+// packed fp32x2 FMA-pipe instruction does two lanes of work in one issue slot.
+// The passes are bound by issue slots and the SFU, so each logit gets exactly
+// one SFU operation and as few issued instructions as the accuracy allows:
 //
-// Reciprocal, on the FMA pipe: a seed, then the cubically convergent step
-// r1 = r0 (1 + e + e^2) with e = 1 - w r0, which leaves |1 - w r1| = |e|^3.
-//  * item pass, w in (1, 2]: linear minimax seed (24 - 8 w) / 17, |e| <= 1/17,
-//    so |1 - w r1| <= 2.1e-4;
-//  * gradient-only passes, w in (1, 2^100]: exponent-flip seed
-//    r0 = bits^-1(C - bits(w)) (the integer subtraction negates the exponent
-//    and roughly reflects the mantissa; with C = 0x7EF31000, |e| <= 0.0506 for
-//    every normal w), so |1 - w r1| <= 1.3e-4.
-// Both seeds are formed from -w, which the FMA pipe produces in the same
-// instruction as 1 + u (bits(-w) = bits(w) + 2^31 for the integer seed).
+//  * passes with the loss (with or without the gradient): one tanh per logit.
+//    With t = tanh(z/2): sigmoid(z) = (1 + t)/2, and w = 1 + |t| = 2 sigmoid(|z|),
+//    which is in [1, 2], so l(z, 0) = max(z, 0) + ln 2 - ln w.  The log is
+//    taken once per 32 logits of a row, as log2 of the product of their w.
+//  * gradient only: sigmoid(z) = (1 + tanh(z/2))/2 from one tanh, except for
+//    one pair in 16, whose sigmoid runs wholly on the FMA pipe (an FMA-pipe
+//    2^x and a reciprocal by seed and cubic step) to take load off the SFU.
 //
-// Gradient-only passes move a share of their exponentials to the FMA pipe as
-// well (exp2_poly3_pair below).
-//
-// Packed fp32x2 instructions (two lanes of work per instruction) halve the
-// issue slots of the FMA-pipe part; the SFU and the selects stay scalar.
+// tanh.approx.f32 is measured on B200 by the library's element-math self test
+// (cutbce_selftest_element_math) over [-40, 40]: sigmoid from it is within
+// 4.0e-6 of the exact value, ln w within 4.4e-6, and the mean error of ln w
+// over z ~ N(0, 1) is 4e-8 of the mean element loss; the bf16 rounding of G
+// that follows is up to 2^-9 relative.
 #pragma once
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -41,7 +37,12 @@ constexpr uint32_t kRcpSeedNeg = 0x7EF31000u + 0x80000000u;   // C + 2^31: seed 
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
-// 1 / w from nw = -w (w normal and positive): seed plus cubic step, |rel err| <= 1.3e-4.
+// 1 / w from nw = -w (w normal and positive) on the FMA pipe: the exponent-flip
+// seed r0 = bits^-1(C - bits(w)), C = 0x7EF31000 (the integer subtraction
+// negates the exponent and roughly reflects the mantissa: |1 - w r0| <= 0.0506
+// for every normal w), formed from -w since bits(-w) = bits(w) + 2^31; then the
+// cubically convergent step r1 = r0 (1 + e + e^2), e = 1 - w r0, which leaves
+// |1 - w r1| = |e|^3 <= 1.3e-4.
 __device__ __forceinline__ float2 rcp2_cubic(float2 nw) {
   float2 r = f2(__uint_as_float(kRcpSeedNeg - __float_as_uint(nw.x)),
                 __uint_as_float(kRcpSeedNeg - __float_as_uint(nw.y)));
@@ -50,37 +51,24 @@ __device__ __forceinline__ float2 rcp2_cubic(float2 nw) {
   return __ffma2_rn(r, t, r);                          // r0 (1 + e + e^2)
 }
 
-// 1 / w for w in [1, 2] from nw = -w: linear minimax seed r0 = (24 - 8 w) / 17
-// (|rel err| <= 1/17), one FFMA2 instead of two integer subtractions, then the
-// cubic step: |rel err| <= (1/17)^3 = 2.1e-4.
-__device__ __forceinline__ float2 rcp2_unit_interval(float2 nw) {
-  float2 r = __ffma2_rn(nw, f2(8.f / 17.f, 8.f / 17.f), f2(24.f / 17.f, 24.f / 17.f));
-  const float2 e = __ffma2_rn(nw, r, f2(1.f, 1.f));    // 1 - w r0
-  const float2 t = __ffma2_rn(e, e, e);                // e + e^2
-  return __ffma2_rn(r, t, r);                          // r0 (1 + e + e^2)
-}
-
-// Item-owned pass, loss and gradient: returns sigmoid(z) for both logits and
-// folds their loss terms into the running products `prod` (of w, sign-free
-// over an even count of factors per component) and the running sum `relu`
-// of max(z, 0).  z log2 e is formed for both logits in one packed multiply;
-// the exponential takes -|.| of it as operand modifiers.
+// Passes with the loss and the gradient (the item-owned pass, and the
+// position-owned pass when it takes the weighted loss): returns sigmoid(z) for
+// both logits and folds their loss terms into the running product `prod` of
+// w = 1 + |tanh(z/2)| and the running sum `relu` of max(z, 0).
 __device__ __forceinline__ float2 bce_pair_loss_grad(float2 z, float2& prod, float2& relu) {
-  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
-  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));   // e^{-|z|}
-  const float2 nw = __ffma2_rn(u, f2(-1.f, -1.f), f2(-1.f, -1.f));           // -(1 + u)
-  prod = __fmul2_rn(prod, nw);
+  const float2 h = __fmul2_rn(z, f2(0.5f, 0.5f));
+  const float2 t = f2(tanh_approx(h.x), tanh_approx(h.y));
+  prod = __fmul2_rn(prod, f2(1.f + fabsf(t.x), 1.f + fabsf(t.y)));
   relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
-  const float2 r = rcp2_unit_interval(nw);
-  const float2 ur = __fmul2_rn(u, r);
-  return f2(z.x >= 0.f ? r.x : ur.x, z.y >= 0.f ? r.y : ur.y);
+  return __ffma2_rn(t, f2(0.5f, 0.5f), f2(0.5f, 0.5f));
 }
 
-// Item-owned pass, loss only.
+// Loss only (the forward): the same terms as bce_pair_loss_grad, so that the
+// forward and the fused call give the same loss bit for bit.
 __device__ __forceinline__ void bce_pair_loss(float2 z, float2& prod, float2& relu) {
-  const float2 tz = __fmul2_rn(z, f2(kLog2eF, kLog2eF));
-  const float2 u = f2(ex2_approx(-fabsf(tz.x)), ex2_approx(-fabsf(tz.y)));
-  prod = __fmul2_rn(prod, __fadd2_rn(u, f2(1.f, 1.f)));
+  const float2 h = __fmul2_rn(z, f2(0.5f, 0.5f));
+  const float2 t = f2(tanh_approx(h.x), tanh_approx(h.y));
+  prod = __fmul2_rn(prod, f2(1.f + fabsf(t.x), 1.f + fabsf(t.y)));
   relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
 }
 
@@ -113,30 +101,34 @@ __device__ __forceinline__ float2 exp2_poly3_pair(float2 x) {
   return f2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
-// Pairs of every 16 (one 32-logit chunk) whose exponential the gradient-only
-// passes evaluate on the FMA pipe instead of the SFU.  The SFU retires 16
-// exponentials per clock per SM and the polynomial costs about four more issue
-// slots than the SFU instruction, so only a small share moves (the best of
-// 0, 1, 2, 3 and 4 of 16 measured on the position-owned pass).
-constexpr int kPolyPairsPerChunk = 2;
+// Pairs of every 16 (one 32-logit chunk) whose sigmoid the gradient-only
+// passes evaluate wholly on the FMA pipe instead of from the SFU's tanh.  The
+// FMA-pipe path costs about ten more issue slots a pair, so only a small share
+// moves (the best of 0 to 3 of 16, measured on the position-owned pass).
+constexpr int kPolyPairsPerChunk = 1;
 
-// Gradient only (the position-owned pass, and the item pass without the loss):
+// Gradient only, on the FMA pipe alone:
 // sigmoid(z) = 1 / (1 + 2^x), x = -z log2 e clamped to [-100, 100] as
-// 200 * saturate(-z log2 e / 200 + 1/2) - 100 on the FMA pipe (error <= 200 *
-// 2^-25 in x, 4e-6 relative in 2^x); below z = -69.3 the result is 2^-100
-// instead of a smaller positive number.  2^x from the SFU, or (kPoly) from the
-// FMA-pipe polynomial; then the exponent-flip seed and the cubic step
-// (|rel err| <= 1.3e-4).  Total relative error <= 2.1e-4 plus rounding, well
-// inside the bf16 rounding of G that follows (up to 2^-9).
-template <bool kPoly>
-__device__ __forceinline__ float2 sigmoid_pair(float2 z) {
+// 200 * saturate(-z log2 e / 200 + 1/2) - 100 (error <= 200 * 2^-25 in x,
+// 4e-6 relative in 2^x); below z = -69.3 the result is 2^-100 instead of a
+// smaller positive number.  2^x from the FMA-pipe polynomial (7.5e-5), then the
+// exponent-flip seed and the cubic step (|rel err| <= 1.3e-4).  Total relative
+// error <= 2.1e-4 plus rounding, inside the bf16 rounding of G that follows.
+__device__ __forceinline__ float2 sigmoid_pair_fma(float2 z) {
   float ax, ay;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ax) : "f"(z.x), "f"(-kLog2eF / 200.f), "f"(0.5f));
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ay) : "f"(z.y), "f"(-kLog2eF / 200.f), "f"(0.5f));
   const float2 x = __ffma2_rn(f2(ax, ay), f2(200.f, 200.f), f2(-100.f, -100.f));
-  const float2 v = kPoly ? exp2_poly3_pair(x) : f2(ex2_approx(x.x), ex2_approx(x.y));
+  const float2 v = exp2_poly3_pair(x);
   const float2 nw = __ffma2_rn(v, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + v)
   return rcp2_cubic(nw);
+}
+
+// Gradient only, one SFU operation and two packed FMA-pipe instructions per pair:
+// sigmoid(z) = (1 + tanh(z / 2)) / 2.
+__device__ __forceinline__ float2 sigmoid_pair_tanh(float2 z) {
+  const float2 h = __fmul2_rn(z, f2(0.5f, 0.5f));
+  return __ffma2_rn(f2(tanh_approx(h.x), tanh_approx(h.y)), f2(0.5f, 0.5f), f2(0.5f, 0.5f));
 }
 
 }  // namespace cutbce

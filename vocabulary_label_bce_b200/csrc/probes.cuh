@@ -205,4 +205,71 @@ __global__ void __launch_bounds__(128, 1) k_probe_mma(int iters, unsigned long l
   }
 }
 
+// The same probe on an SM pair: 2-CTA clusters, and the even CTA of each issues
+// `iters` tcgen05.mma.cta_group::2 of shape 256 x N x 16 (each CTA holds 128
+// rows of A, in shared or tensor memory, and its half of B; zero operands).
+// Both CTAs allocate the pair's tensor memory; neither frees it before the
+// issuing CTA has seen the commit and both have passed a cluster barrier.
+template <int N, bool kATmem>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1) k_probe_mma_pair(int iters, unsigned long long* out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                    // 128 x 64 bf16, 128-byte swizzle (16 KB)
+  uint8_t* sB = smem + 16384;            // N x 64 bf16, K-major, 128-byte swizzle
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  for (int i = threadIdx.x; i < (16384 + N * 128) / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  const uint32_t rank = cluster_ctarank();
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  fence_proxy_async_smem();
+  if ((threadIdx.x >> 5) == 0) tmem_alloc_pair(&tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tslot;
+  if (kATmem) {
+    uint32_t z[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) z[k] = 0;
+    tmem_st16(tbase + ((static_cast<uint32_t>(threadIdx.x >> 5) * 32) << 16) + 256, z);
+    tmem_st_wait();
+  }
+  // both CTAs' operands are in place before the even CTA issues
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  if (rank == 0 && threadIdx.x == 0) {
+    const uint32_t idesc = idesc_bf16_f32(256, N, false, false);
+    const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+    const long long t0 = clock64();
+    for (int i = 0; i < iters; ++i) {
+      const int ks = i & 3;
+      const uint64_t bd = smem_desc_sw128(b_base + ks * 32, 16, 1024);
+      if (kATmem) {
+        umma_bf16_pair_tmem_a(tbase, tbase + 256, bd, idesc, i > 0 ? 1u : 0u);
+      } else {
+        const uint64_t ad = smem_desc_sw128(a_base + ks * 32, 16, 1024);
+        umma_bf16_pair(tbase, ad, bd, idesc, i > 0 ? 1u : 0u);
+      }
+    }
+    const long long t1 = clock64();
+    umma_commit_pair(&bar);
+    wait_bar_drain(&bar, 0, 2000000000LL);
+    const long long t2 = clock64();
+    out[2 * blockIdx.x] = static_cast<unsigned long long>(t1 - t0);
+    out[2 * blockIdx.x + 1] = static_cast<unsigned long long>(t2 - t0);
+  }
+  // the pair's MMAs are complete before either CTA frees its tensor memory
+  tc_fence_before();
+  cluster_sync_all();
+  if ((threadIdx.x >> 5) == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tbase, 512);
+  }
+}
+
 }  // namespace cutbce

@@ -665,9 +665,9 @@ __global__ void __launch_bounds__(kTileThreads, 1)
               } else if (kLoss) {
                 bce_pair_loss(z, prod, relu);
               } else if (((e >> 1) * kPolyPairsPerChunk) % 16 < kPolyPairsPerChunk) {
-                g = sigmoid_pair<true>(z);          // exponential on the FMA pipe (a few pairs, spread evenly)
+                g = sigmoid_pair_fma(z);            // wholly on the FMA pipe (a few pairs, spread evenly)
               } else {
-                g = sigmoid_pair<false>(z);         // exponential on the SFU
+                g = sigmoid_pair_tanh(z);           // one tanh per logit on the SFU
               }
               if (kGrad) {
                 if (decltype(with_y)::value) {                     // y = 1 at the masked columns
@@ -691,8 +691,9 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             met_tp += static_cast<int>(mtp);
           }
           if (kLoss) {
-            // CH / 2 factors per component: the product of the -(1 + u) factors is positive
-            tile_l2 += lg2_approx(prod.x * prod.y);
+            // CH / 2 factors in [1, 2] per component: the product stays finite;
+            // tile_l2 collects log2(1 + e^{-|z|}) = 1 - log2 w of each element (w = 2 sigmoid(|z|))
+            tile_l2 += static_cast<float>(CH) - lg2_approx(prod.x * prod.y);
             tile_mx += relu.x + relu.y;
           }
           // G over the first half of this warp's own (already loaded) logit columns
@@ -812,17 +813,21 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   }
 }
 
-// Element-math self test: for each x, the FMA-pipe 2^x, the SFU 2^x and the
-// gradient-only sigmoid of z = x (both exponential paths).  Used only by
-// cutbce_selftest_exp2.
-__global__ void k_selftest_exp2(const float* __restrict__ x, float* __restrict__ out, int64_t n) {
+// Element-math self test, for each x: [0] the FMA-pipe 2^x, [1] the SFU 2^x,
+// [2] the gradient-only sigmoid of z = x on the FMA pipe, [3] the sigmoid from
+// tanh, [4] w = 1 + |tanh(x/2)| as the loss-and-gradient passes form it.  Used
+// only by cutbce_selftest_element_math.
+__global__ void k_selftest_element_math(const float* __restrict__ x, float* __restrict__ out, int64_t n) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const float v = x[i];
   out[i] = exp2_poly3_pair(f2(v, v)).x;
   out[n + i] = ex2_approx(v);
-  out[2 * n + i] = sigmoid_pair<true>(f2(v, v)).x;
-  out[3 * n + i] = sigmoid_pair<false>(f2(v, v)).x;
+  out[2 * n + i] = sigmoid_pair_fma(f2(v, v)).x;
+  out[3 * n + i] = sigmoid_pair_tanh(f2(v, v)).x;
+  float2 prod = f2(1.f, 1.f), relu = f2(0.f, 0.f);
+  bce_pair_loss_grad(f2(v, v), prod, relu);
+  out[4 * n + i] = prod.x;
 }
 
 // A deliberately unsignalled barrier: the bounded wait must give up, record the
