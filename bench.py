@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the side measurements (metrics, top-8)")
+    ap.add_argument("--topk-queries", type=int, default=0,
+                    help="with --calls-only: top-8 ranking calls for this many queries instead of the fused step")
     ap.add_argument("--cpu-sample-items", type=int, default=32768)
     ap.add_argument("--calls-only", type=int, default=0,
                     help="run this many untimed fused calls on --workload and exit (a target for ncu)")
@@ -492,8 +494,15 @@ def run_calls_only(args):
     loss = torch.empty((), dtype=torch.float64, device=dev)
     dH = torch.empty((p.T, p.D), dtype=torch.float32, device=dev)
     dE = torch.empty((p.V, p.D), dtype=torch.float32, device=dev)
-    for _ in range(args.calls_only):
-        B.cutbce_forward_backward(prob, None, loss, dH, dE, ws)
+    if args.topk_queries > 0:
+        # top-8 ranking of the first topk_queries valid rows of H against the whole vocabulary
+        Q = H[torch.from_numpy(np.nonzero(p.mask)[0][:args.topk_queries]).to(dev)].contiguous()
+        ws = torch.empty(B.cutbce_topk_workspace_size(Q.shape[0], p.V, p.D, 8), dtype=torch.uint8, device=dev)
+        for _ in range(args.calls_only):
+            B.cutbce_topk(Q, E, 8, ws)
+    else:
+        for _ in range(args.calls_only):
+            B.cutbce_forward_backward(prob, None, loss, dH, dE, ws)
     torch.cuda.synchronize(dev)
     status = B.cutbce_read_status(ws)
     if status != 0:

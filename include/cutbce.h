@@ -306,7 +306,9 @@ enum {
   CUTBCE_KERNEL_POSITION_PASS = 5,  /* tensor-core pass owning position tiles: dH partials */
   CUTBCE_KERNEL_FINISH = 6,         /* fixed-order dH reduction and the loss */
   CUTBCE_KERNEL_PAIR_SORT = 7,      /* pairs grouped by item tile, ascending position: sort keys and all radix passes */
-  CUTBCE_NUM_KERNEL_KINDS = 8
+  CUTBCE_KERNEL_TOPK = 8,           /* cutbce_topk: tensor-core scores and per-thread candidate lists */
+  CUTBCE_KERNEL_TOPK_MERGE = 9,     /* cutbce_topk: fixed-order merge of the candidate lists */
+  CUTBCE_NUM_KERNEL_KINDS = 10
 };
 
 /* Per-kernel device timing for benchmarks.  While enabled (process-wide),

@@ -910,14 +910,21 @@ cutbce_status cutbce_topk(const void* Q, int64_t B, const void* E, int64_t V, in
   if (cudaMemsetAsync(tp.hdr, 0, 256, st) != cudaSuccess) return CUTBCE_ERR_CUDA;
   const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(dev.sms),
                                                        static_cast<int64_t>(pl.n_qt) * pl.S, kMaxCtas}));
-  cudaError_t e = pl.KMAX == 8 ? launch_topk_dp<8>(pl.DP, grid, mq, me, tp, st)
-                               : launch_topk_dp<16>(pl.DP, grid, mq, me, tp, st);
+  cudaError_t e;
+  {
+    LaunchScope ls(CUTBCE_KERNEL_TOPK, st);
+    e = pl.KMAX == 8 ? launch_topk_dp<8>(pl.DP, grid, mq, me, tp, st)
+                     : launch_topk_dp<16>(pl.DP, grid, mq, me, tp, st);
+  }
   if (e != cudaSuccess) return CUTBCE_ERR_CUDA;
   const unsigned mgrid = static_cast<unsigned>(ceil_div(B * 32, 256));
-  if (pl.KMAX == 8)
-    k_topk_merge<8><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
-  else
-    k_topk_merge<16><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+  {
+    LaunchScope ls(CUTBCE_KERNEL_TOPK_MERGE, st);
+    if (pl.KMAX == 8)
+      k_topk_merge<8><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+    else
+      k_topk_merge<16><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+  }
   return cudaGetLastError() == cudaSuccess ? CUTBCE_OK : CUTBCE_ERR_CUDA;
 }
 

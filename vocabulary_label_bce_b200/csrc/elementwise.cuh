@@ -9,10 +9,12 @@
 // and the SM issues one warp instruction per clock per sub-partition, so a
 // packed fp32x2 FMA-pipe instruction does two lanes of work in one issue slot.
 // The passes are bound by issue slots and the SFU, so each logit gets exactly
-// one SFU operation and as few issued instructions as the accuracy allows:
+// one SFU operation and as few issued instructions as the accuracy allows.
+// The tensor-core tiles hold zh = z / 2 (the compacted H is stored halved,
+// exactly), which is the argument of the tanh below; the functions here take zh.
 //
 //  * passes with the loss (with or without the gradient): one tanh per logit.
-//    With t = tanh(z/2): sigmoid(z) = (1 + t)/2, and w = 1 + |t| = 2 sigmoid(|z|),
+//    With t = tanh(zh): sigmoid(z) = (1 + t)/2, and w = 1 + |t| = 2 sigmoid(|z|),
 //    which is in [1, 2], so l(z, 0) = max(z, 0) + ln 2 - ln w.  The log is
 //    taken once per 32 logits of a row, as log2 of the product of their w.
 //  * gradient only: sigmoid(z) = (1 + tanh(z/2))/2 from one tanh, except for
@@ -53,23 +55,22 @@ __device__ __forceinline__ float2 rcp2_cubic(float2 nw) {
 
 // Passes with the loss and the gradient (the item-owned pass, and the
 // position-owned pass when it takes the weighted loss): returns sigmoid(z) for
-// both logits and folds their loss terms into the running product `prod` of
-// w = 1 + |tanh(z/2)| and the running sum `relu` of max(z, 0).
-__device__ __forceinline__ float2 bce_pair_loss_grad(float2 z, float2& prod, float2& relu) {
-  const float2 h = __fmul2_rn(z, f2(0.5f, 0.5f));
-  const float2 t = f2(tanh_approx(h.x), tanh_approx(h.y));
+// both logits (zh = z / 2) and folds their loss terms into the running product
+// `prod` of w = 1 + |tanh(zh)| and the running sum `relu` of max(zh, 0) (half of
+// the sum of max(z, 0), which the caller doubles).
+__device__ __forceinline__ float2 bce_pair_loss_grad(float2 zh, float2& prod, float2& relu) {
+  const float2 t = f2(tanh_approx(zh.x), tanh_approx(zh.y));
   prod = __fmul2_rn(prod, f2(1.f + fabsf(t.x), 1.f + fabsf(t.y)));
-  relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
+  relu = __fadd2_rn(relu, f2(fmaxf(zh.x, 0.f), fmaxf(zh.y, 0.f)));
   return __ffma2_rn(t, f2(0.5f, 0.5f), f2(0.5f, 0.5f));
 }
 
 // Loss only (the forward): the same terms as bce_pair_loss_grad, so that the
 // forward and the fused call give the same loss bit for bit.
-__device__ __forceinline__ void bce_pair_loss(float2 z, float2& prod, float2& relu) {
-  const float2 h = __fmul2_rn(z, f2(0.5f, 0.5f));
-  const float2 t = f2(tanh_approx(h.x), tanh_approx(h.y));
+__device__ __forceinline__ void bce_pair_loss(float2 zh, float2& prod, float2& relu) {
+  const float2 t = f2(tanh_approx(zh.x), tanh_approx(zh.y));
   prod = __fmul2_rn(prod, f2(1.f + fabsf(t.x), 1.f + fabsf(t.y)));
-  relu = __fadd2_rn(relu, f2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
+  relu = __fadd2_rn(relu, f2(fmaxf(zh.x, 0.f), fmaxf(zh.y, 0.f)));
 }
 
 // 1 for every normal x > 0, 0 for x <= 0 (and for a subnormal x, flushed to 0):
@@ -107,28 +108,28 @@ __device__ __forceinline__ float2 exp2_poly3_pair(float2 x) {
 // moves (the best of 0 to 3 of 16, measured on the position-owned pass).
 constexpr int kPolyPairsPerChunk = 1;
 
-// Gradient only, on the FMA pipe alone:
+// Gradient only, on the FMA pipe alone, from zh = z / 2:
 // sigmoid(z) = 1 / (1 + 2^x), x = -z log2 e clamped to [-100, 100] as
-// 200 * saturate(-z log2 e / 200 + 1/2) - 100 (error <= 200 * 2^-25 in x,
+// 200 * saturate(-zh (2 log2 e) / 200 + 1/2) - 100 (the same bits as with z and
+// log2 e / 200: both factors are scaled by exact powers of two; error <= 200 * 2^-25 in x,
 // 4e-6 relative in 2^x); below z = -69.3 the result is 2^-100 instead of a
 // smaller positive number.  2^x from the FMA-pipe polynomial (7.5e-5), then the
 // exponent-flip seed and the cubic step (|rel err| <= 1.3e-4).  Total relative
 // error <= 2.1e-4 plus rounding, inside the bf16 rounding of G that follows.
-__device__ __forceinline__ float2 sigmoid_pair_fma(float2 z) {
+__device__ __forceinline__ float2 sigmoid_pair_fma(float2 zh) {
   float ax, ay;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ax) : "f"(z.x), "f"(-kLog2eF / 200.f), "f"(0.5f));
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ay) : "f"(z.y), "f"(-kLog2eF / 200.f), "f"(0.5f));
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ax) : "f"(zh.x), "f"(-kLog2eF / 100.f), "f"(0.5f));
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(ay) : "f"(zh.y), "f"(-kLog2eF / 100.f), "f"(0.5f));
   const float2 x = __ffma2_rn(f2(ax, ay), f2(200.f, 200.f), f2(-100.f, -100.f));
   const float2 v = exp2_poly3_pair(x);
   const float2 nw = __ffma2_rn(v, f2(-1.f, -1.f), f2(-1.f, -1.f));   // -(1 + v)
   return rcp2_cubic(nw);
 }
 
-// Gradient only, one SFU operation and two packed FMA-pipe instructions per pair:
-// sigmoid(z) = (1 + tanh(z / 2)) / 2.
-__device__ __forceinline__ float2 sigmoid_pair_tanh(float2 z) {
-  const float2 h = __fmul2_rn(z, f2(0.5f, 0.5f));
-  return __ffma2_rn(f2(tanh_approx(h.x), tanh_approx(h.y)), f2(0.5f, 0.5f), f2(0.5f, 0.5f));
+// Gradient only, one SFU operation and one packed FMA-pipe instruction per pair:
+// sigmoid(z) = (1 + tanh(zh)) / 2, zh = z / 2.
+__device__ __forceinline__ float2 sigmoid_pair_tanh(float2 zh) {
+  return __ffma2_rn(f2(tanh_approx(zh.x), tanh_approx(zh.y)), f2(0.5f, 0.5f), f2(0.5f, 0.5f));
 }
 
 }  // namespace cutbce

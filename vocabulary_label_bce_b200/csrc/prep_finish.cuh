@@ -170,10 +170,16 @@ __global__ void __launch_bounds__(kScanThreads) k_prep_scan(const uint8_t* __res
 // ------------------------------------------------------------------ prep: gather
 // One warp per compacted row c in [0, Tpad).  Copies h_t into the compacted,
 // zero-padded H_c (rows >= n_valid are zero so padded tiles contribute exactly
-// nothing to any gradient), writes the pair lists and, with per-position
+// nothing to any gradient; with bf16 inputs the row is stored halved, h_t / 2,
+// which is exact, so that the tensor-core tiles hold z / 2: the argument of the
+// tanh the element math takes), writes the pair lists and, with per-position
 // weights, the compacted weights (0 for the padded rows), and sums the sparse
 // target correction sum_{v in P_t} w_t h_t . e_v of Eq. (2) in fp32 per pair, in
 // a fixed order, into one double per block.
+// bf16 H_c (the tensor-core path) holds h / 2; fp32 H_c (the SIMT path) holds h.
+template <typename TIn>
+constexpr bool kHalveHc = sizeof(TIn) == 2;
+
 template <typename TIn>
 __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, const TIn* __restrict__ E,
                                                      int D, int DP, int K, int64_t Tpad,
@@ -195,7 +201,8 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
       const int t = orig[c];
       const double wt = weights != nullptr ? static_cast<double>(weights[t]) : 1.0;
       const TIn* src = H + static_cast<int64_t>(t) * D;
-      for (int d = lane; d < DP; d += 32) dst[d] = d < D ? src[d] : TIn(0.0f);
+      for (int d = lane; d < DP; d += 32)
+        dst[d] = d < D ? (kHalveHc<TIn> ? TIn(0.5f * static_cast<float>(src[d])) : src[d]) : TIn(0.0f);
       const int p0 = row_ptr[c];
       const int n = row_cnt[t];
       for (int k = 0; k < n; ++k) {

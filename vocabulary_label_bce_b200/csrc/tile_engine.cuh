@@ -31,6 +31,11 @@
 // uses no Y at all (Eq. (2): l(x,y) = l(x,0) - y x); the -y x part is the
 // sparse correction summed in the prep kernel.
 //
+// The compacted H is stored halved (exact in bf16), so the tiles hold z / 2,
+// the argument of the element math's tanh; the item-owned accumulator then
+// holds G^T (H / 2) and is scaled by twice the gradient scale (exact), and the
+// sum of max(z / 2, 0) is doubled.
+//
 // Warp roles (576 threads, one CTA per SM):
 //   warp 0      TMA producer (stationary tile, ring of NX streamed tiles)
 //   warp 1      TMEM allocator and MMA issuer: an event loop over the logit
@@ -513,7 +518,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     const int slab = (ew >> 2) % Cfg::SLABS;       // column slab within the group
     const int row = q * 32 + lane;                // stationary row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    const float gs = hdr->grad_scale;
+    // the item-owned accumulator holds G^T (H / 2): its scale is doubled (exact)
+    const float gs = hdr->grad_scale * (kDH ? 1.f : 2.f);
     uint32_t* wmask = sMask + ew * 32 * Cfg::MASK_WORDS;   // this warp's positives scratch
 #pragma unroll
     for (int k = 0; k < Cfg::MASK_WORDS; ++k) wmask[lane * Cfg::MASK_WORDS + k] = 0u;
@@ -645,12 +651,12 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           auto chunk_math = [&](auto with_y, auto with_w) {
 #pragma unroll
             for (int e = 0; e < CH; e += 2) {
-              const float2 z = f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+              const float2 z = f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));   // z / 2 (H_c holds H / 2)
               float2 g = f2(0.f, 0.f);
               float2 mpos = f2(0.f, 0.f);
               if (kMet) {
-                // [x > 0] on the FMA pipe: saturate(x * 2^126) is 1 for every normal x > 0 and
-                // 0 for x <= 0 (a subnormal x is flushed to 0 and counts as not positive)
+                // [x > 0] on the FMA pipe, from x / 2: saturate(x / 2 * 2^126) is 1 for every
+                // normal x / 2 > 0 and 0 for x <= 0 (a subnormal is flushed to 0: not positive)
                 mpos = f2(positive_mask(z.x), positive_mask(z.y));
                 mcnt = __fadd2_rn(mcnt, mpos);
                 if (decltype(with_y)::value) {
@@ -724,7 +730,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             const int pad = hi - max(min(p.V - v0, hi), lo);
             tile_l2 -= static_cast<float>(pad);
           }
-          item_acc += static_cast<double>(tile_mx + tile_l2 * kLn2);
+          item_acc += static_cast<double>(2.f * tile_mx + tile_l2 * kLn2);   // tile_mx sums max(z / 2, 0)
         }
       }
       if (!ok) break;
@@ -823,10 +829,11 @@ __global__ void k_selftest_element_math(const float* __restrict__ x, float* __re
   const float v = x[i];
   out[i] = exp2_poly3_pair(f2(v, v)).x;
   out[n + i] = ex2_approx(v);
-  out[2 * n + i] = sigmoid_pair_fma(f2(v, v)).x;
-  out[3 * n + i] = sigmoid_pair_tanh(f2(v, v)).x;
+  const float vh = 0.5f * v;                     // the tiles hold z / 2
+  out[2 * n + i] = sigmoid_pair_fma(f2(vh, vh)).x;
+  out[3 * n + i] = sigmoid_pair_tanh(f2(vh, vh)).x;
   float2 prod = f2(1.f, 1.f), relu = f2(0.f, 0.f);
-  bce_pair_loss_grad(f2(v, v), prod, relu);
+  bce_pair_loss_grad(f2(vh, vh), prod, relu);
   out[4 * n + i] = prod.x;
 }
 

@@ -60,6 +60,12 @@ struct TopkParams {
 
 // Insert (s, v) into a list sorted by descending score whose last entry is
 // beaten (s > ls[K-1]); equal scores keep the earlier entry first.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 template <int K>
 __device__ __forceinline__ void topk_insert(float (&ls)[K], int (&li)[K], float s, int v) {
 #pragma unroll
@@ -250,10 +256,24 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         if (lane == 0) mbar_arrive(bar_zfree + zb);
         const int v0 = (t0 + j) * BN + slab * ZC;
         const int valid_cols = min(ZC, p.V - v0);     // item rows past V are zero-filled: excluded
+        if (valid_cols < ZC) {
 #pragma unroll
-        for (int e = 0; e < ZC; ++e) {
-          const float s = __uint_as_float(r[e]);
-          if (s > ls[KMAX - 1] && e < valid_cols) topk_insert<KMAX>(ls, li, s, v0 + e);
+          for (int e = 0; e < ZC; ++e)
+            if (e >= valid_cols) r[e] = __float_as_uint(-INFINITY);
+        }
+        // the tile's best score first (three-input max): once the lists have
+        // filled, almost no tile holds a score that beats this thread's k-th,
+        // and the tile then costs ZC / 2 max operations and one branch
+        float m = __uint_as_float(r[0]);
+#pragma unroll
+        for (int e = 1; e + 1 < ZC; e += 2) m = fmax3(m, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+        if (ZC % 2 == 0) m = fmaxf(m, __uint_as_float(r[ZC - 1]));
+        if (m > ls[KMAX - 1]) {
+#pragma unroll
+          for (int e = 0; e < ZC; ++e) {
+            const float s = __uint_as_float(r[e]);
+            if (s > ls[KMAX - 1]) topk_insert<KMAX>(ls, li, s, v0 + e);
+          }
         }
       }
       if (!ok) break;
