@@ -1,6 +1,6 @@
 """Host-side replay of the FMA-pipe element math of the tile engine.
 
-The gradient-only passes evaluate one pair of logits in 16 wholly on the FMA
+The gradient-only passes evaluate two pairs of logits in 16 wholly on the FMA
 pipe: 2^x by a degree-3 polynomial with integer exponent insertion, then 1/w
 by the exponent-flip seed r0 = bits^-1(C - bits(w)), C = 0x7EF31000 (formed
 from -w, whose bits are bits(w) + 2^31), and one cubically convergent step

@@ -239,7 +239,7 @@ def test_element_math_on_the_device():
     out = B.cutbce_selftest_element_math(torch.from_numpy(z).cuda()).cpu().numpy()
     z64 = z.astype(np.float64)
     sref = 1.0 / (1.0 + np.exp(-z64))
-    # sigmoid wholly on the FMA pipe (one pair in 16 of the gradient-only passes)
+    # sigmoid wholly on the FMA pipe (two pairs in 16 of the gradient-only passes)
     assert np.max(np.abs(out[2] / sref - 1.0)) <= 2.1e-4
     assert np.array_equal(out[2].view(np.uint32), sigmoid_fma(z).view(np.uint32))
     # sigmoid from tanh: absolute error (4.0e-6 measured), relative where sigmoid >= 1/16

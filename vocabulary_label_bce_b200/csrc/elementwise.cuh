@@ -18,7 +18,7 @@
 //    which is in [1, 2], so l(z, 0) = max(z, 0) + ln 2 - ln w.  The log is
 //    taken once per 32 logits of a row, as log2 of the product of their w.
 //  * gradient only: sigmoid(z) = (1 + tanh(z/2))/2 from one tanh, except for
-//    one pair in 16, whose sigmoid runs wholly on the FMA pipe (an FMA-pipe
+//    two pairs in 16, whose sigmoid runs wholly on the FMA pipe (an FMA-pipe
 //    2^x and a reciprocal by seed and cubic step) to take load off the SFU.
 //
 // tanh.approx.f32 is measured on B200 by the library's element-math self test
@@ -106,7 +106,7 @@ __device__ __forceinline__ float2 exp2_poly3_pair(float2 x) {
 // passes evaluate wholly on the FMA pipe instead of from the SFU's tanh.  The
 // FMA-pipe path costs about ten more issue slots a pair, so only a small share
 // moves (the best of 0 to 3 of 16, measured on the position-owned pass).
-constexpr int kPolyPairsPerChunk = 1;
+constexpr int kPolyPairsPerChunk = 2;
 
 // Gradient only, on the FMA pipe alone, from zh = z / 2:
 // sigmoid(z) = 1 / (1 + 2^x), x = -z log2 e clamped to [-100, 100] as
