@@ -308,7 +308,8 @@ enum {
   CUTBCE_KERNEL_PAIR_SORT = 7,      /* pairs grouped by item tile, ascending position: sort keys and all radix passes */
   CUTBCE_KERNEL_TOPK = 8,           /* cutbce_topk: tensor-core scores and per-thread candidate lists */
   CUTBCE_KERNEL_TOPK_MERGE = 9,     /* cutbce_topk: fixed-order merge of the candidate lists */
-  CUTBCE_NUM_KERNEL_KINDS = 10
+  CUTBCE_KERNEL_COL_SUMS = 10,      /* column sums of E and of the compacted H: the loss's linear half */
+  CUTBCE_NUM_KERNEL_KINDS = 11
 };
 
 /* Per-kernel device timing for benchmarks.  While enabled (process-wide),

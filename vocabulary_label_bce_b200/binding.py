@@ -112,7 +112,7 @@ _SIGS = {
 PROBES = ["ffma", "ffma2", "ex2", "rcp", "tanh", "lg2", "cvt_bf16x2", "fmax", "add2", "iadd", "prmt",
           "ex2_f16x2", "ex2_bf16x2", "tanh_f16x2", "hfma2", "cvt_f16x2", "ffma_sat", "select", "lop", "fmul2"]
 KERNEL_KINDS = ["prep_rows", "prep_scan", "prep_gather", "csc_offsets", "item_pass", "position_pass", "finish",
-                "pair_sort", "topk", "topk_merge"]
+                "pair_sort", "topk", "topk_merge", "col_sums"]
 
 
 def load_library() -> ctypes.CDLL:

@@ -41,7 +41,11 @@ struct WsHeader {
   float grad_scale;    // g * s
   int wait_block;      // CTA of that wait
   int finish_count;    // blocks of the finish kernel done with their loss slice
+  int role_wait_tag[7];  // [role - 1]: where role 1 (producer), 2 (MMA), 4 (epilogue) stood when its CTA gave up
+  int colsum_count;    // blocks of the column-sum kernel done
+  double lin;          // (sum_c w_c H_c[c]) . (sum_v e_v): the linear half of the dense loss
 };
+static_assert(sizeof(WsHeader) <= 256, "the workspace header is 256 bytes");
 
 // Geometry of the tcgen05 tile engine for one padded feature width DP and G
 // epilogue groups.

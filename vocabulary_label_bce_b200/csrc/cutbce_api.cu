@@ -93,8 +93,9 @@ struct Plan {
   int radix_passes, radix_blocks;
   size_t elem;
   size_t o_hdr, o_cidx, o_orig, o_rowcnt, o_rowptr, o_ids, o_pair_t, o_pair_v, o_srt[4], o_ghist, o_cscoff, o_hc,
-      o_lpart, o_cpart, o_dhpart, o_fpart, o_metpart, o_wc, total;
+      o_lpart, o_cpart, o_dhpart, o_fpart, o_metpart, o_wc, o_csum, total;
   int met_slots;
+  int csum_nbE, csum_nbH;   // column-sum blocks (loss on the tensor-core path), 0 otherwise
 };
 
 cutbce_status check_problem(const cutbce_problem* p, bool need_data) {
@@ -184,6 +185,10 @@ void make_plan(const cutbce_problem* p, Want w, Plan& pl, bool weighted = false)
   pl.o_dhpart = w.dH ? take(4 * static_cast<size_t>(pl.S) * pl.Tpad * pl.DP) : 0;
   pl.met_slots = bf16 ? pl.S * kMetSlotsPerSplit : 1;
   pl.o_metpart = w.met ? take(8 * static_cast<size_t>(pl.met_slots) * pl.Tpad) : 0;
+  // the linear half of the dense loss (tensor-core path): column sums of E and of H_c
+  pl.csum_nbE = (bf16 && w.loss) ? kColSumBlocksE : 0;
+  pl.csum_nbH = (bf16 && w.loss) ? static_cast<int>(std::min<int64_t>(kColSumBlocksHMax, ceil_div(pl.Tpad, 256))) : 0;
+  pl.o_csum = (bf16 && w.loss) ? take(8 * static_cast<size_t>(pl.csum_nbE + pl.csum_nbH) * p->D) : 0;
   pl.total = o;
 }
 
@@ -411,6 +416,7 @@ int count_launches(const Plan& pl, Want w) {
   const bool bf16 = pl.dtype == CUTBCE_BF16;
   int n = 3;                                            // rows, scan, gather
   if (bf16 && w.dE) n += 1 + 3 * pl.radix_passes + 1;   // sort keys, radix passes, item-tile offsets
+  if (bf16 && w.loss) n += 1;                           // column sums
   if (w.loss || w.dE) n += 1;                           // item-owned pass
   if (w.dH || w.met) n += 1;                            // position-owned pass (dH and/or metrics)
   if (w.loss || w.dH || w.met) n += 1;                  // finish
@@ -489,6 +495,14 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   // With per-position weights the tensor-core path sums the loss in the
   // position-owned pass (one weight per row there); the item-owned pass then
   // computes dE only.  The fp32 path sums it per item with the column weights.
+  if (bf16 && w.loss) {
+    LaunchScope ls(CUTBCE_KERNEL_COL_SUMS, st);
+    k_col_sums<<<static_cast<unsigned>(pl.csum_nbE + pl.csum_nbH), kColSumThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(p->E), V, at<__nv_bfloat16>(ws, pl.o_hc), wc, pl.Tpad, D, pl.DP,
+        pl.csum_nbE, pl.csum_nbH, at<double>(ws, pl.o_csum), hdr);
+    CUTBCE_CK(cudaGetLastError());
+  }
+
   const bool loss_in_pos = bf16 && weighted && w.loss;
   const bool item_loss = w.loss && !loss_in_pos;
   const bool item_pass = item_loss || w.dE;
@@ -624,6 +638,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     fp.met_slots = pl.met_slots;
     fp.metrics = w.met ? o.metrics : nullptr;
     fp.row_cnt = rowcnt;
+    fp.use_lin = (bf16 && w.loss) ? 1 : 0;
     fp.hdr = hdr;
     LaunchScope ls(CUTBCE_KERNEL_FINISH, st);
     k_finish<<<grid, kFinishThreads, 0, st>>>(fp);

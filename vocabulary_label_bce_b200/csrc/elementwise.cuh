@@ -16,7 +16,9 @@
 //  * passes with the loss (with or without the gradient): one tanh per logit.
 //    With t = tanh(zh): sigmoid(z) = (1 + t)/2, and w = 1 + |t| = 2 sigmoid(|z|),
 //    which is in [1, 2], so l(z, 0) = max(z, 0) + ln 2 - ln w.  The log is
-//    taken once per 32 logits of a row, as log2 of the product of their w.
+//    taken once per 32 logits of a row, as log2 of the product of their w, and
+//    max(z, 0) = z / 2 + |z| / 2: the tiles sum |z| / 2, the linear z / 2 is
+//    summed over the whole problem as one dot product of column sums.
 //  * gradient only: sigmoid(z) = (1 + tanh(z/2))/2 from one tanh, except for
 //    two pairs in 16, whose sigmoid runs wholly on the FMA pipe (an FMA-pipe
 //    2^x and a reciprocal by seed and cubic step) to take load off the SFU.
@@ -56,21 +58,24 @@ __device__ __forceinline__ float2 rcp2_cubic(float2 nw) {
 // Passes with the loss and the gradient (the item-owned pass, and the
 // position-owned pass when it takes the weighted loss): returns sigmoid(z) for
 // both logits (zh = z / 2) and folds their loss terms into the running product
-// `prod` of w = 1 + |tanh(zh)| and the running sum `relu` of max(zh, 0) (half of
-// the sum of max(z, 0), which the caller doubles).
-__device__ __forceinline__ float2 bce_pair_loss_grad(float2 zh, float2& prod, float2& relu) {
+// `prod` of w = 1 + |tanh(zh)| and the running sum `absz` of |zh| = |z| / 2 (the
+// other half of max(z, 0) = z / 2 + |z| / 2 is linear in z and summed once,
+// from column sums, by the finish).
+__device__ __forceinline__ float2 bce_pair_loss_grad(float2 zh, float2& prod, float2& absz) {
   const float2 t = f2(tanh_approx(zh.x), tanh_approx(zh.y));
   prod = __fmul2_rn(prod, f2(1.f + fabsf(t.x), 1.f + fabsf(t.y)));
-  relu = __fadd2_rn(relu, f2(fmaxf(zh.x, 0.f), fmaxf(zh.y, 0.f)));
+  absz.x += fabsf(zh.x);
+  absz.y += fabsf(zh.y);
   return __ffma2_rn(t, f2(0.5f, 0.5f), f2(0.5f, 0.5f));
 }
 
 // Loss only (the forward): the same terms as bce_pair_loss_grad, so that the
 // forward and the fused call give the same loss bit for bit.
-__device__ __forceinline__ void bce_pair_loss(float2 zh, float2& prod, float2& relu) {
+__device__ __forceinline__ void bce_pair_loss(float2 zh, float2& prod, float2& absz) {
   const float2 t = f2(tanh_approx(zh.x), tanh_approx(zh.y));
   prod = __fmul2_rn(prod, f2(1.f + fabsf(t.x), 1.f + fabsf(t.y)));
-  relu = __fadd2_rn(relu, f2(fmaxf(zh.x, 0.f), fmaxf(zh.y, 0.f)));
+  absz.x += fabsf(zh.x);
+  absz.y += fabsf(zh.y);
 }
 
 // 1 for every normal x > 0, 0 for x <= 0 (and for a subnormal x, flushed to 0):

@@ -231,6 +231,107 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
   }
 }
 
+// ------------------------------------------------------------------ prep: column sums
+// The linear half of the dense loss.  With max(z, 0) = z / 2 + |z| / 2,
+//   sum_{t valid} w_t sum_{v < V} max(z_tv, 0)
+//     = 1/2 (sum_t w_t h_t) . (sum_v e_v)  +  sum_{t, v} w_t |z_tv| / 2,
+// so the tile kernels accumulate only |z / 2| (their tiles hold z / 2), and the
+// first term is one dot product of two column sums.  Blocks [0, nbE) sum fixed
+// slices of the rows of E, blocks [nbE, nbE + nbH) fixed slices of the
+// compacted H (which holds h / 2, rows past n_valid zero) times the compacted
+// weights; each block writes one fp64 partial per column, and the last block
+// to finish (a ticket in the header, which each call clears) sums the partials
+// in a fixed order and writes the dot product to the header.  Eight bf16
+// columns per 16-byte load; D is a multiple of 8.
+constexpr int kColSumThreads = 256;
+constexpr int kColSumBlocksE = 444;
+constexpr int kColSumBlocksHMax = 64;
+
+__global__ void __launch_bounds__(kColSumThreads) k_col_sums(const __nv_bfloat16* __restrict__ E, int64_t V,
+                                                              const __nv_bfloat16* __restrict__ Hc,
+                                                              const float* __restrict__ wc, int64_t Tpad, int D,
+                                                              int DP, int nbE, int nbH, double* __restrict__ part,
+                                                              WsHeader* hdr) {
+  __shared__ double red[kColSumThreads * 8];
+  __shared__ int ticket;
+  const int b = blockIdx.x;
+  const bool isE = b < nbE;
+  const int64_t rows = isE ? V : Tpad;
+  const int64_t stride = isE ? D : DP;
+  const __nv_bfloat16* src = isE ? E : Hc;
+  const int nb = isE ? nbE : nbH;
+  const int bb = isE ? b : b - nbE;
+  const int64_t per = (rows + nb - 1) / nb;
+  const int64_t r0 = static_cast<int64_t>(bb) * per, r1 = min(rows, r0 + per);
+  const int tpr = D / 8;                       // threads per row, 8 columns each
+  const int rpp = kColSumThreads / tpr;        // rows per pass
+  const int cg = threadIdx.x % tpr, rs = threadIdx.x / tpr;
+  double acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.0;
+  if (rs < rpp) {
+#pragma unroll 4
+    for (int64_t r = r0 + rs; r < r1; r += rpp) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + r * stride) + cg);
+      const double w = (!isE && wc != nullptr) ? static_cast<double>(__ldg(wc + r)) : 1.0;
+      const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[2 * k] += w * static_cast<double>(__uint_as_float(u[k] << 16));
+        acc[2 * k + 1] += w * static_cast<double>(__uint_as_float(u[k] & 0xFFFF0000u));
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) red[k * kColSumThreads + threadIdx.x] = rs < rpp ? acc[k] : 0.0;
+  __syncthreads();
+  // column d = 8 cg + k: the rpp row groups in order
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    const int g = d / 8, k = d % 8;
+    double sum = 0.0;
+    for (int q = 0; q < rpp; ++q) sum += red[k * kColSumThreads + q * tpr + g];
+    part[static_cast<int64_t>(b) * D + d] = sum;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) ticket = atomicAdd(&hdr->colsum_count, 1);
+  __syncthreads();
+  if (ticket != static_cast<int>(gridDim.x) - 1) return;
+  __threadfence();
+  // the last block: thread (d, j) sums every np-th partial from j on, the np
+  // sums of a column are then added in order (np = 256 / D threads per column)
+  const int np = kColSumThreads / D;
+  const int d = threadIdx.x % D, j = threadIdx.x / D;
+  double se = 0.0, sh = 0.0;
+  if (j < np) {
+#pragma unroll 8
+    for (int i = j; i < nbE; i += np) se += __ldcg(part + static_cast<int64_t>(i) * D + d);
+#pragma unroll 8
+    for (int i = j; i < nbH; i += np) sh += __ldcg(part + static_cast<int64_t>(nbE + i) * D + d);
+  }
+  red[threadIdx.x] = j < np ? se : 0.0;
+  red[kColSumThreads + threadIdx.x] = j < np ? sh : 0.0;
+  __syncthreads();
+  double prod = 0.0;
+  if (threadIdx.x < D) {
+    double e = 0.0, h = 0.0;
+    for (int q = 0; q < np; ++q) {
+      e += red[q * D + threadIdx.x];
+      h += red[kColSumThreads + q * D + threadIdx.x];
+    }
+    prod = e * h;
+  }
+  __syncthreads();
+  // fixed tree over the columns
+  red[threadIdx.x] = prod;
+  __syncthreads();
+  for (int st = kColSumThreads / 2; st > 0; st >>= 1) {
+    if (threadIdx.x < st) red[threadIdx.x] += red[threadIdx.x + st];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) hdr->lin = red[0];
+}
+
 // ------------------------------------------------------------------ finish
 // dH[t, d] = g*s * sum_{split} partial[split][c(t)][d] in split order (0 for
 // masked rows).  The loss = s * (dense - correction) is summed in two levels:
@@ -272,6 +373,7 @@ struct FinishParams {
   int met_slots;
   int32_t* metrics;           // [T, 4] output TP, FP, FN, TN, or null
   const int* row_cnt;         // [T] distinct positives of each position
+  int use_lin;                // add the linear half of the dense loss (hdr->lin, from k_col_sums)
   WsHeader* hdr;
 };
 
@@ -354,7 +456,9 @@ __global__ void __launch_bounds__(kFinishThreads) k_finish(const FinishParams f)
       }
       const double dense = block_sum_fixed(da, red);
       const double corr = block_sum_fixed(db, red);
-      if (threadIdx.x == 0) *f.loss = f.hdr->n_valid > 0 ? f.hdr->loss_scale * (dense - corr) : 0.0;
+      // the linear half of the dense term: (sum_c wc_c H_c[c]) . (sum_v e_v), H_c holding h / 2
+      const double lin = f.use_lin ? *reinterpret_cast<volatile double*>(&f.hdr->lin) : 0.0;
+      if (threadIdx.x == 0) *f.loss = f.hdr->n_valid > 0 ? f.hdr->loss_scale * (dense + lin - corr) : 0.0;
     }
   }
 }

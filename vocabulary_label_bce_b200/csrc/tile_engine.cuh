@@ -33,8 +33,9 @@
 //
 // The compacted H is stored halved (exact in bf16), so the tiles hold z / 2,
 // the argument of the element math's tanh; the item-owned accumulator then
-// holds G^T (H / 2) and is scaled by twice the gradient scale (exact), and the
-// sum of max(z / 2, 0) is doubled.
+// holds G^T (H / 2) and is scaled by twice the gradient scale (exact).  The
+// loss tiles sum |z| / 2; the linear half of max(z, 0) = z / 2 + |z| / 2 is one
+// dot product of column sums, added by the finish kernel.
 //
 // Warp roles (576 threads, one CTA per SM):
 //   warp 0      TMA producer (stationary tile, ring of NX streamed tiles)
@@ -114,7 +115,8 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const W
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*w.abort_flag) {
       // record where each role stood when the CTA gave up (first record per role wins)
-      if (tag != 0) atomicCAS(reinterpret_cast<int*>(w.hdr) + 8 + ((tag >> 28) & 7), 0, tag);
+      const int role = (tag >> 28) & 7;
+      if (tag != 0 && role >= 1) atomicCAS(&w.hdr->role_wait_tag[role - 1], 0, tag);
       return false;
     }
     if (static_cast<long long>(global_timer_ns() - t0) > w.limit) {
@@ -641,7 +643,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           float2 mcnt = f2(0.f, 0.f);             // metrics: x > 0 in this chunk (two lanes of a sum)
           float mtp = 0.f;                        // metrics: positives with x > 0 in this chunk
           uint32_t pk[CH / 2];
-          float2 prod = f2(1.f, 1.f), relu = f2(0.f, 0.f);
+          float2 prod = f2(1.f, 1.f), absz = f2(0.f, 0.f);
           // the chunk's element math; the y = 1 subtraction is compiled into a
           // separate copy taken only by chunks that hold a positive (rare), so
           // the common path has no per-element branch or bit test
@@ -667,9 +669,9 @@ __global__ void __launch_bounds__(kTileThreads, 1)
               if (!kLoss && !kGrad) {
                 // metrics only: no element math beyond the count
               } else if (kLoss && kGrad) {
-                g = bce_pair_loss_grad(z, prod, relu);
+                g = bce_pair_loss_grad(z, prod, absz);
               } else if (kLoss) {
-                bce_pair_loss(z, prod, relu);
+                bce_pair_loss(z, prod, absz);
               } else if (((e >> 1) * kPolyPairsPerChunk) % 16 < kPolyPairsPerChunk) {
                 g = sigmoid_pair_fma(z);            // wholly on the FMA pipe (a few pairs, spread evenly)
               } else {
@@ -700,7 +702,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             // CH / 2 factors in [1, 2] per component: the product stays finite;
             // tile_l2 collects log2(1 + e^{-|z|}) = 1 - log2 w of each element (w = 2 sigmoid(|z|))
             tile_l2 += static_cast<float>(CH) - lg2_approx(prod.x * prod.y);
-            tile_mx += relu.x + relu.y;
+            tile_mx += absz.x + absz.y;
           }
           // G over the first half of this warp's own (already loaded) logit columns
           if (kGrad) {
@@ -730,7 +732,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             const int pad = hi - max(min(p.V - v0, hi), lo);
             tile_l2 -= static_cast<float>(pad);
           }
-          item_acc += static_cast<double>(2.f * tile_mx + tile_l2 * kLn2);   // tile_mx sums max(z / 2, 0)
+          item_acc += static_cast<double>(tile_mx + tile_l2 * kLn2);   // tile_mx sums |z| / 2
         }
       }
       if (!ok) break;
@@ -832,8 +834,8 @@ __global__ void k_selftest_element_math(const float* __restrict__ x, float* __re
   const float vh = 0.5f * v;                     // the tiles hold z / 2
   out[2 * n + i] = sigmoid_pair_fma(f2(vh, vh)).x;
   out[3 * n + i] = sigmoid_pair_tanh(f2(vh, vh)).x;
-  float2 prod = f2(1.f, 1.f), relu = f2(0.f, 0.f);
-  bce_pair_loss_grad(f2(vh, vh), prod, relu);
+  float2 prod = f2(1.f, 1.f), absz = f2(0.f, 0.f);
+  bce_pair_loss_grad(f2(vh, vh), prod, absz);
   out[4 * n + i] = prod.x;
 }
 
