@@ -35,7 +35,12 @@
  *    never allocates or frees device memory and keeps no state between calls
  *    apart from cached device attributes and the static scratch array of
  *    cutbce_forward_fixed_scratch.
- *  - All compute calls are asynchronous on `stream`.  Errors a host can see
+ *  - All compute calls are asynchronous on `stream`.  A call that computes the
+ *    loss runs the column sums of E on a second stream of the library's own
+ *    (created once per device, pooled), forked from `stream` and joined back
+ *    to it by events, so the work is ordered on `stream` as usual (and is
+ *    captured into a CUDA graph with it); cutbce_forward_fixed_scratch uses
+ *    `stream` alone.  Errors a host can see
  *    (NULL pointers, sizes <= 0, unsupported D or dtype, a workspace that is
  *    too small, a device that is not sm_100) are returned before anything is
  *    launched.  Data-dependent errors (an id out of range, a bounded wait in a
@@ -139,7 +144,8 @@ cutbce_status cutbce_forward(const cutbce_problem* prob, void* ws, size_t ws_byt
  * Limit: problems with cutbce_workspace_size_for(prob, CUTBCE_OUT_LOSS) >
  * CUTBCE_FIXED_SCRATCH_BYTES are rejected with CUTBCE_ERR_WORKSPACE before
  * anything is launched.  That loss-only workspace is about
- * 16 T K + 2 T D' + 16 * 8 * ceil(V / 128) bytes (D' = D rounded up to 64), so
+ * 16 T K + 2 T D' + 16 * 8 * ceil(V / 128) + 8 D (444 + ceil(T / 256)) bytes
+ * (D' = D rounded up to 64; at most 64 in the last ceiling), so
  * for example T = 12,800 positions with K = 16 slots, D = 64 and V = 876,000
  * items (about 6 MB) fits.
  * Setup: the first call on each device, with that device current, looks up

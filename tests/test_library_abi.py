@@ -108,10 +108,10 @@ def test_workspace_size_per_outputs():
 
 def test_launch_accounting():
     p = _prob()
-    # rows, scan, gather, column sums, sort keys, 2 radix passes x 3 (6844 item tiles:
-    # 13-bit keys), item-tile offsets, item pass, dH pass, finish
-    assert B.cutbce_kernel_launches(p, 2) == 15
-    assert B.cutbce_kernel_launches(p, 0) == 6          # rows, scan, gather, column sums, item pass, finish
+    # rows, scan, gather, column sums of E and of H_c, sort keys, 2 radix passes x 3
+    # (6844 item tiles: 13-bit keys), item-tile offsets, item pass, dH pass, finish
+    assert B.cutbce_kernel_launches(p, 2) == 16
+    assert B.cutbce_kernel_launches(p, 0) == 7          # rows, scan, gather, 2 column sums, item pass, finish
     assert B.cutbce_kernel_launches(p, 1) == 14         # backward: no loss, so no column sums
     assert B.cutbce_kernel_launches(p, 3) == -1
 

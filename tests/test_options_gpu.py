@@ -77,6 +77,22 @@ def test_weights_match_oracle(shape, reduction):
     assert rel_fro(got["dE"].cpu().numpy(), ref.dE) <= GRAD_RTOL
 
 
+def test_weights_with_one_signed_logits():
+    # weighted loss (taken in the position-owned pass) whose linear half, from the
+    # weighted column sums, is most of the loss
+    p = W.draw(T=257, V=1500, D=128, K=6, dtype="bf16", seed=33, ids="zipf", mask="random", mask_frac=0.1)
+    p.E_bits &= np.uint16(0x7FFF)
+    p.E[:] = np.abs(p.E)
+    p.H_bits &= np.uint16(0x7FFF)
+    p.H[:] = np.abs(p.H)
+    w = weights_for(p, 4)
+    got = call(p, to_device(p), "sum", weights=w)
+    ref = O.forward_backward(p.H, p.E, p.targets, p.mask, reduction=RED["sum"], weights=w.astype(np.float64))
+    assert abs(got["loss"] - ref.loss) <= LOSS_RTOL * abs(ref.loss), (got["loss"], ref.loss)
+    assert rel_fro(got["dH"].cpu().numpy(), ref.dH) <= GRAD_RTOL
+    assert rel_fro(got["dE"].cpu().numpy(), ref.dE) <= GRAD_RTOL
+
+
 @pytest.mark.parametrize("want", [("loss",), ("loss", "metrics"), ("dE",), ("dH",), ("loss", "dE")])
 def test_weights_partial_outputs(want):
     p = W.draw(T=333, V=1500, D=64, K=4, dtype="bf16", seed=32, ids="zipf", mask="random", mask_frac=0.2)

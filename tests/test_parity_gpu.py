@@ -129,6 +129,23 @@ def test_zero_activations_closed_form():
     check_against_oracle(p, got, "sum")
 
 
+@pytest.mark.parametrize("signs", ["all_positive", "positive_items"])
+def test_linear_half_of_the_loss(signs):
+    # the tile kernels sum |z| / 2 and the finish adds the linear half z / 2 from
+    # column sums; with every logit positive (or every row of logits one-signed)
+    # the linear half is most of the loss, so its precision is exposed
+    p = W.draw(T=300, V=2047, D=64, K=5, dtype="bf16", seed=12, ids="zipf", mask="random", mask_frac=0.1)
+    p.E_bits &= np.uint16(0x7FFF)
+    p.E[:] = np.abs(p.E)
+    if signs == "all_positive":
+        p.H_bits &= np.uint16(0x7FFF)
+        p.H[:] = np.abs(p.H)
+    for red in ("sum", "mean"):
+        got = run_gpu(p, red)
+        _, rep = check_against_oracle(p, got, red)
+        print(signs, red, rep)
+
+
 def test_paper_stress_distribution():
     # A, E ~ N(0, I), D=128, L=8 uniform ids (mini-benchmark inputs): saturated logits
     p = W.draw(T=256, V=2000, D=128, K=8, dtype="bf16", seed=11, e_std=1.0, ids="uniform", mask="none")

@@ -53,6 +53,7 @@ struct Opts {
   const float* weights = nullptr;
   bool grad_bf16 = false, acc_dH = false, acc_dE = false;
   int64_t v_off = 0, V_total = 0;   // V_total resolved: the problem's V when not sharded
+  bool one_stream = false;           // everything on the caller's stream (no pooled second stream)
 };
 
 cutbce_status resolve_opts(const cutbce_problem* p, const cutbce_options* o, Opts& out) {
@@ -412,11 +413,65 @@ cutbce_status topk_plan(int64_t B, int64_t V, int64_t D, int k, int sms, TopkPla
   return CUTBCE_OK;
 }
 
+// Second streams: the host-buffer entry copies dE out on one, ordered after the
+// item-owned pass by an event, and a call that computes the loss runs the
+// column sums of E on one, concurrently with the prep kernels.  Streams and
+// events are created once per device and pooled: each call takes what it uses
+// for its duration, so concurrent calls never share an event.
+struct SideStream {
+  int dev;
+  cudaStream_t s;
+  cudaEvent_t ev, ev2;
+};
+std::mutex g_side_mu;
+std::vector<SideStream> g_side_free;
+
+cutbce_status take_side_stream(SideStream& out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CUTBCE_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    for (size_t i = 0; i < g_side_free.size(); ++i) {
+      if (g_side_free[i].dev == dev) {
+        out = g_side_free[i];
+        g_side_free.erase(g_side_free.begin() + static_cast<std::ptrdiff_t>(i));
+        return CUTBCE_OK;
+      }
+    }
+  }
+  out.dev = dev;
+  if (cudaStreamCreateWithFlags(&out.s, cudaStreamNonBlocking) != cudaSuccess) return CUTBCE_ERR_CUDA;
+  if (cudaEventCreateWithFlags(&out.ev, cudaEventDisableTiming) != cudaSuccess) {
+    cudaStreamDestroy(out.s);
+    return CUTBCE_ERR_CUDA;
+  }
+  if (cudaEventCreateWithFlags(&out.ev2, cudaEventDisableTiming) != cudaSuccess) {
+    cudaEventDestroy(out.ev);
+    cudaStreamDestroy(out.s);
+    return CUTBCE_ERR_CUDA;
+  }
+  return CUTBCE_OK;
+}
+
+void give_side_stream(const SideStream& s) {
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  g_side_free.push_back(s);
+}
+
+// Gives a taken side stream back when the call returns, on every path.
+struct SideStreamLease {
+  SideStream s{};
+  bool held = false;
+  ~SideStreamLease() {
+    if (held) give_side_stream(s);
+  }
+};
+
 int count_launches(const Plan& pl, Want w) {
   const bool bf16 = pl.dtype == CUTBCE_BF16;
   int n = 3;                                            // rows, scan, gather
   if (bf16 && w.dE) n += 1 + 3 * pl.radix_passes + 1;   // sort keys, radix passes, item-tile offsets
-  if (bf16 && w.loss) n += 1;                           // column sums
+  if (bf16 && w.loss) n += 2;                           // column sums of E (second stream) and of H_c
   if (w.loss || w.dE) n += 1;                           // item-owned pass
   if (w.dH || w.met) n += 1;                            // position-owned pass (dH and/or metrics)
   if (w.loss || w.dH || w.met) n += 1;                  // finish
@@ -465,6 +520,26 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     if ((x) != cudaSuccess) return CUTBCE_ERR_CUDA; \
   } while (0)
 
+  // the column sums of E depend on E alone: a second stream computes them while
+  // the prep kernels run, and the column-sum kernel of H_c waits for it
+  // (the fixed-scratch entry keeps to one stream: it runs them in order)
+  SideStreamLease side;
+  if (bf16 && w.loss) {
+    cudaStream_t cs = st;
+    if (!o.one_stream) {
+      if ((s = take_side_stream(side.s)) != CUTBCE_OK) return s;
+      side.held = true;
+      CUTBCE_CK(cudaEventRecord(side.s.ev, st));
+      CUTBCE_CK(cudaStreamWaitEvent(side.s.s, side.s.ev, 0));
+      cs = side.s.s;
+    }
+    LaunchScope ls(CUTBCE_KERNEL_COL_SUMS, cs);
+    k_col_sums<<<static_cast<unsigned>(pl.csum_nbE), kColSumThreads, 0, cs>>>(
+        static_cast<const __nv_bfloat16*>(p->E), V, nullptr, nullptr, pl.Tpad, D, pl.DP, pl.csum_nbE, pl.csum_nbH,
+        at<double>(ws, pl.o_csum), hdr, 0, 0);
+    CUTBCE_CK(cudaGetLastError());
+    if (side.held) CUTBCE_CK(cudaEventRecord(side.s.ev2, side.s.s));
+  }
   CUTBCE_CK(cudaMemsetAsync(hdr, 0, 256, st));
   {
   LaunchScope ls(CUTBCE_KERNEL_PREP_ROWS, st);
@@ -496,10 +571,11 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   // position-owned pass (one weight per row there); the item-owned pass then
   // computes dE only.  The fp32 path sums it per item with the column weights.
   if (bf16 && w.loss) {
+    if (side.held) CUTBCE_CK(cudaStreamWaitEvent(st, side.s.ev2, 0));
     LaunchScope ls(CUTBCE_KERNEL_COL_SUMS, st);
-    k_col_sums<<<static_cast<unsigned>(pl.csum_nbE + pl.csum_nbH), kColSumThreads, 0, st>>>(
+    k_col_sums<<<static_cast<unsigned>(pl.csum_nbH), kColSumThreads, 0, st>>>(
         static_cast<const __nv_bfloat16*>(p->E), V, at<__nv_bfloat16>(ws, pl.o_hc), wc, pl.Tpad, D, pl.DP,
-        pl.csum_nbE, pl.csum_nbH, at<double>(ws, pl.o_csum), hdr);
+        pl.csum_nbE, pl.csum_nbH, at<double>(ws, pl.o_csum), hdr, pl.csum_nbE, 1);
     CUTBCE_CK(cudaGetLastError());
   }
 
@@ -673,45 +749,6 @@ void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
 }
 
 // ---------------------------------------------------------------- host-entry side streams
-// The host-buffer entry copies dE out on a second stream, ordered after the
-// item-owned pass by an event.  Streams and events are created once per device
-// and pooled: each call takes one pair for its duration, so concurrent calls
-// never share an event.
-struct SideStream {
-  int dev;
-  cudaStream_t s;
-  cudaEvent_t ev;
-};
-std::mutex g_side_mu;
-std::vector<SideStream> g_side_free;
-
-cutbce_status take_side_stream(SideStream& out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return CUTBCE_ERR_CUDA;
-  {
-    std::lock_guard<std::mutex> lk(g_side_mu);
-    for (size_t i = 0; i < g_side_free.size(); ++i) {
-      if (g_side_free[i].dev == dev) {
-        out = g_side_free[i];
-        g_side_free.erase(g_side_free.begin() + static_cast<std::ptrdiff_t>(i));
-        return CUTBCE_OK;
-      }
-    }
-  }
-  out.dev = dev;
-  if (cudaStreamCreateWithFlags(&out.s, cudaStreamNonBlocking) != cudaSuccess) return CUTBCE_ERR_CUDA;
-  if (cudaEventCreateWithFlags(&out.ev, cudaEventDisableTiming) != cudaSuccess) {
-    cudaStreamDestroy(out.s);
-    return CUTBCE_ERR_CUDA;
-  }
-  return CUTBCE_OK;
-}
-
-void give_side_stream(const SideStream& s) {
-  std::lock_guard<std::mutex> lk(g_side_mu);
-  g_side_free.push_back(s);
-}
-
 // ---------------------------------------------------------------- fixed scratch
 // Scratch of cutbce_forward_fixed_scratch: a static device array of the
 // library's own module, so that entry needs no caller workspace and allocates
@@ -773,8 +810,10 @@ cutbce_status cutbce_forward_fixed_scratch(const cutbce_problem* prob, double* l
   if (pl.total > kFixedScratchBytes) return CUTBCE_ERR_WORKSPACE;   // the problem needs more than the fixed array
   void* ws = nullptr;
   if ((s = fixed_scratch_ptr(&ws)) != CUTBCE_OK) return s;
+  Opts o{};
+  o.one_stream = true;                                              // creates no stream or event either
   return run(prob, nullptr, loss, nullptr, nullptr, Want{true, false, false, false}, ws, kFixedScratchBytes,
-             reinterpret_cast<cudaStream_t>(stream));
+             reinterpret_cast<cudaStream_t>(stream), nullptr, o);
 }
 
 cutbce_status cutbce_backward(const cutbce_problem* prob, const float* grad_loss, float* dH, float* dE, void* ws,

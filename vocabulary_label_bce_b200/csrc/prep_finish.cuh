@@ -239,10 +239,11 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
 // first term is one dot product of two column sums.  Blocks [0, nbE) sum fixed
 // slices of the rows of E, blocks [nbE, nbE + nbH) fixed slices of the
 // compacted H (which holds h / 2, rows past n_valid zero) times the compacted
-// weights; each block writes one fp64 partial per column, and the last block
-// to finish (a ticket in the header, which each call clears) sums the partials
-// in a fixed order and writes the dot product to the header.  Eight bf16
-// columns per 16-byte load; D is a multiple of 8.
+// weights; each block writes one fp64 partial per column.  A launch covers the
+// logical blocks [first_block, first_block + gridDim.x); with `final`, the last
+// of its blocks to finish (a ticket in the header, which each call clears) sums
+// all nbE + nbH partials in a fixed order and writes the dot product to the
+// header.  Eight bf16 columns per 16-byte load; D is a multiple of 8.
 constexpr int kColSumThreads = 256;
 constexpr int kColSumBlocksE = 444;
 constexpr int kColSumBlocksHMax = 64;
@@ -251,10 +252,10 @@ __global__ void __launch_bounds__(kColSumThreads) k_col_sums(const __nv_bfloat16
                                                               const __nv_bfloat16* __restrict__ Hc,
                                                               const float* __restrict__ wc, int64_t Tpad, int D,
                                                               int DP, int nbE, int nbH, double* __restrict__ part,
-                                                              WsHeader* hdr) {
+                                                              WsHeader* hdr, int first_block, int final) {
   __shared__ double red[kColSumThreads * 8];
   __shared__ int ticket;
-  const int b = blockIdx.x;
+  const int b = static_cast<int>(blockIdx.x) + first_block;
   const bool isE = b < nbE;
   const int64_t rows = isE ? V : Tpad;
   const int64_t stride = isE ? D : DP;
@@ -292,6 +293,7 @@ __global__ void __launch_bounds__(kColSumThreads) k_col_sums(const __nv_bfloat16
     for (int q = 0; q < rpp; ++q) sum += red[k * kColSumThreads + q * tpr + g];
     part[static_cast<int64_t>(b) * D + d] = sum;
   }
+  if (!final) return;
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) ticket = atomicAdd(&hdr->colsum_count, 1);
