@@ -249,14 +249,20 @@ cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes)
  * asynchronous), grad_loss is a host value, and loss / dH / dE are host
  * outputs (dH, dE may be NULL).  dev_buf (>= cutbce_host_buffer_size bytes,
  * 256-byte aligned, caller-owned device memory) holds the device copies and the
- * workspace.  The call copies the inputs in, runs cutbce_forward_backward,
- * copies the results out and synchronises `stream`; on return the host outputs
- * are valid and the returned status includes the device status word.  dE is
- * final once the item-owned pass ends, so its copy to the host runs on a second
- * stream while the dH pass still runs on `stream`; both streams are
- * synchronised before the call returns.  That second stream and its event are
- * created by the first such calls on a device and kept in a per-device pool for
- * the rest of the process (one pair per call in flight). */
+ * workspace.  The call copies the inputs in, runs the fused computation,
+ * copies the results out and synchronises; on return the host outputs are
+ * valid and the returned status includes the device status word.
+ * Overlap: with a bf16 item table of more than 32 MiB, the call works in up to
+ * four vocabulary shards of whole 128-item tiles (the shard options of
+ * cutbce_forward_backward_ex): shard s + 1 of E is copied in on a second stream
+ * while shard s is computed on `stream`, and each shard's dE rows are copied
+ * out on a third stream as soon as its item-owned pass ends, while its dH pass
+ * and the next shard run.  The shards' losses are added on the host and their
+ * dH on the device, in shard order, so the results are deterministic and equal
+ * those of cutbce_forward_backward to rounding (bit for bit with one shard).
+ * The streams and events come from a per-device pool, created by the first
+ * such calls and kept for the rest of the process; every stream the call used
+ * is synchronised before it returns. */
 cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float grad_loss,
                                            double* loss, float* dH, float* dE,
                                            void* dev_buf, size_t dev_bytes,

@@ -726,8 +726,33 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
 
 // Host-buffer entry: layout of the caller's device buffer.
 struct HostLayout {
-  size_t o_H, o_E, o_tg, o_mask, o_loss, o_grad, o_dH, o_dE, o_ws, total;
+  size_t o_H, o_E, o_tg, o_mask, o_loss, o_status, o_grad, o_dH, o_dE, o_ws, total;
 };
+
+// The host-buffer entry runs a large item table in up to kMaxHostShards
+// vocabulary shards of whole 128-item tiles, so that copying shard s + 1 in and
+// shard s - 1's dE out overlap the computation of shard s.
+constexpr int kMaxHostShards = 4;
+constexpr int64_t kHostShardBytes = int64_t(32) << 20;
+
+int host_shards(const cutbce_problem* p) {
+  if (p->dtype != CUTBCE_BF16) return 1;
+  int64_t n = ceil_div(2 * p->V * p->D, kHostShardBytes);
+  n = std::min<int64_t>({n, static_cast<int64_t>(kMaxHostShards), ceil_div(p->V, kTileM)});
+  return static_cast<int>(std::max<int64_t>(1, n));
+}
+
+// Items [v0, v1) of shard k of n, in whole tiles.  The first and the last shard
+// are the smaller ones: the first one's copy in and the last one's copy out are
+// the only copies nothing overlaps.  Cumulative shares in 1/20 of the tiles.
+void host_shard_bounds(int64_t V, int n, int k, int64_t& v0, int64_t& v1) {
+  static const int kCum[kMaxHostShards + 1][kMaxHostShards + 1] = {
+      {0, 0, 0, 0, 0}, {0, 20, 0, 0, 0}, {0, 10, 20, 0, 0}, {0, 5, 15, 20, 0}, {0, 3, 10, 17, 20}};
+  const int64_t tiles = ceil_div(V, kTileM);
+  const int64_t t0 = tiles * kCum[n][k] / 20, t1 = tiles * kCum[n][k + 1] / 20;
+  v0 = std::min(V, t0 * kTileM);
+  v1 = std::min(V, t1 * kTileM);
+}
 
 void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
   size_t o = 0;
@@ -740,7 +765,8 @@ void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
   hl.o_E = take(pl.elem * p->V * p->D);
   hl.o_tg = take(4 * p->T * p->K);
   hl.o_mask = take(p->T);
-  hl.o_loss = take(8);
+  hl.o_loss = take(8 * kMaxHostShards);       // one loss per shard, summed on the host in shard order
+  hl.o_status = take(4 * kMaxHostShards);     // the status word of each shard's call
   hl.o_grad = take(4);
   hl.o_dH = take(4 * p->T * p->D);
   hl.o_dE = take(4 * p->V * p->D);
@@ -748,7 +774,6 @@ void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
   hl.total = o;
 }
 
-// ---------------------------------------------------------------- host-entry side streams
 // ---------------------------------------------------------------- fixed scratch
 // Scratch of cutbce_forward_fixed_scratch: a static device array of the
 // library's own module, so that entry needs no caller workspace and allocates
@@ -878,50 +903,87 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   HostLayout hl;
   host_layout(prob, pl, hl);
   if (dev_bytes < hl.total) return CUTBCE_ERR_WORKSPACE;
-  // dE is final once the item-owned pass ends: its copy to the host runs on a
-  // second stream while the position-owned pass and the finish run on `st`.
-  // The stream and its event come from a per-device pool (created on first use).
-  SideStream side{};
-  if (dE != nullptr && (s = take_side_stream(side)) != CUTBCE_OK) return s;
+  const int nsh = host_shards(prob);
+  // Streams (per-device pool, created on first use): E's shards are copied in on
+  // `cin`, the computation runs on `st`, and each shard's dE is copied out on
+  // `cout` as soon as its item-owned pass ends (dE is final then), while the
+  // dH pass and the next shard run on `st`.
+  SideStreamLease cin, cout;
+  if (nsh > 1) {
+    if ((s = take_side_stream(cin.s)) != CUTBCE_OK) return s;
+    cin.held = true;
+  }
+  if (dE != nullptr) {
+    if ((s = take_side_stream(cout.s)) != CUTBCE_OK) return s;
+    cout.held = true;
+  }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t in = nsh > 1 ? cin.s.s : st;
   uint8_t* b = static_cast<uint8_t*>(dev_buf);
-  const size_t szH = pl.elem * prob->T * prob->D, szE = pl.elem * prob->V * prob->D;
-  bool copied = cudaMemcpyAsync(b + hl.o_H, prob->H, szH, cudaMemcpyHostToDevice, st) == cudaSuccess &&
-                cudaMemcpyAsync(b + hl.o_E, prob->E, szE, cudaMemcpyHostToDevice, st) == cudaSuccess &&
-                cudaMemcpyAsync(b + hl.o_tg, prob->targets, 4 * prob->T * prob->K, cudaMemcpyHostToDevice, st) ==
-                    cudaSuccess &&
-                (prob->mask == nullptr ||
-                 cudaMemcpyAsync(b + hl.o_mask, prob->mask, prob->T, cudaMemcpyHostToDevice, st) == cudaSuccess) &&
-                cudaMemcpyAsync(b + hl.o_grad, &grad_loss, 4, cudaMemcpyHostToDevice, st) == cudaSuccess;
+  const size_t rowE = pl.elem * prob->D;
+  bool ok = cudaMemcpyAsync(b + hl.o_H, prob->H, pl.elem * prob->T * prob->D, cudaMemcpyHostToDevice, st) ==
+                cudaSuccess &&
+            cudaMemcpyAsync(b + hl.o_tg, prob->targets, 4 * prob->T * prob->K, cudaMemcpyHostToDevice, st) ==
+                cudaSuccess &&
+            (prob->mask == nullptr ||
+             cudaMemcpyAsync(b + hl.o_mask, prob->mask, prob->T, cudaMemcpyHostToDevice, st) == cudaSuccess) &&
+            cudaMemcpyAsync(b + hl.o_grad, &grad_loss, 4, cudaMemcpyHostToDevice, st) == cudaSuccess;
   cutbce_problem dp = *prob;
   dp.H = b + hl.o_H;
-  dp.E = b + hl.o_E;
   dp.targets = reinterpret_cast<const int32_t*>(b + hl.o_tg);
   dp.mask = prob->mask != nullptr ? reinterpret_cast<const uint8_t*>(b + hl.o_mask) : nullptr;
   float* ddH = dH ? reinterpret_cast<float*>(b + hl.o_dH) : nullptr;
   float* ddE = dE ? reinterpret_cast<float*>(b + hl.o_dE) : nullptr;
-  s = copied ? run(&dp, reinterpret_cast<const float*>(b + hl.o_grad), reinterpret_cast<double*>(b + hl.o_loss),
-                   ddH, ddE, Want{true, dE != nullptr, dH != nullptr, false}, b + hl.o_ws, pl.total, st, side.ev)
-             : CUTBCE_ERR_CUDA;
-  if (s != CUTBCE_OK) {
-    cudaStreamSynchronize(st);   // no copy from or to the caller's host memory may still run on return
-    if (dE != nullptr) give_side_stream(side);
-    return s;
+  double* dloss = reinterpret_cast<double*>(b + hl.o_loss);
+  int32_t* dstatus = reinterpret_cast<int32_t*>(b + hl.o_status);
+  for (int k = 0; k < nsh && ok && s == CUTBCE_OK; ++k) {
+    int64_t v0 = 0, v1 = prob->V;
+    if (nsh > 1) host_shard_bounds(prob->V, nsh, k, v0, v1);   // never empty: nsh > 1 needs V D > 16 Mi
+    if (v1 <= v0) {
+      s = CUTBCE_ERR_INVALID_ARG;
+      break;
+    }
+    ok = cudaMemcpyAsync(b + hl.o_E + v0 * rowE, static_cast<const uint8_t*>(prob->E) + v0 * rowE,
+                         (v1 - v0) * rowE, cudaMemcpyHostToDevice, in) == cudaSuccess;
+    if (ok && nsh > 1)
+      ok = cudaEventRecord(cin.s.ev, in) == cudaSuccess && cudaStreamWaitEvent(st, cin.s.ev, 0) == cudaSuccess;
+    if (!ok) break;
+    cutbce_problem sp = dp;
+    sp.E = b + hl.o_E + v0 * rowE;
+    sp.V = v1 - v0;
+    Opts o{};
+    o.v_off = v0;
+    o.V_total = prob->V;
+    o.acc_dH = k > 0;                        // the shards' dH add up, in shard order
+    s = run(&sp, reinterpret_cast<const float*>(b + hl.o_grad), dloss + k, ddH,
+            ddE ? ddE + v0 * prob->D : nullptr, Want{true, dE != nullptr, dH != nullptr, false}, b + hl.o_ws,
+            pl.total, st, dE != nullptr ? cout.s.ev : nullptr, o);
+    if (s != CUTBCE_OK) break;
+    ok = cudaMemcpyAsync(dstatus + k, b + hl.o_ws + pl.o_hdr, 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    if (ok && dE != nullptr)
+      ok = cudaStreamWaitEvent(cout.s.s, cout.s.ev, 0) == cudaSuccess &&
+           cudaMemcpyAsync(dE + v0 * prob->D, ddE + v0 * prob->D, 4 * (v1 - v0) * prob->D, cudaMemcpyDeviceToHost,
+                           cout.s.s) == cudaSuccess;
   }
-  int dev_status = 0;
-  bool ok = true;
-  if (dE != nullptr)
-    ok = cudaStreamWaitEvent(side.s, side.ev, 0) == cudaSuccess &&
-         cudaMemcpyAsync(dE, ddE, 4 * prob->V * prob->D, cudaMemcpyDeviceToHost, side.s) == cudaSuccess;
-  ok = ok && cudaMemcpyAsync(loss, b + hl.o_loss, 8, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
-       (!dH || cudaMemcpyAsync(dH, ddH, 4 * prob->T * prob->D, cudaMemcpyDeviceToHost, st) == cudaSuccess) &&
-       cudaMemcpyAsync(&dev_status, b + hl.o_ws + pl.o_hdr, 4, cudaMemcpyDeviceToHost, st) == cudaSuccess;
-  // both streams are drained before returning, also after an error
-  const bool sync_ok = cudaStreamSynchronize(st) == cudaSuccess &&
-                       (dE == nullptr || cudaStreamSynchronize(side.s) == cudaSuccess);
-  if (dE != nullptr) give_side_stream(side);
+  double losses[kMaxHostShards] = {};
+  int32_t statuses[kMaxHostShards] = {};
+  if (ok && s == CUTBCE_OK)
+    ok = cudaMemcpyAsync(losses, dloss, 8 * nsh, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
+         (!dH || cudaMemcpyAsync(dH, ddH, 4 * prob->T * prob->D, cudaMemcpyDeviceToHost, st) == cudaSuccess) &&
+         cudaMemcpyAsync(statuses, dstatus, 4 * nsh, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+  // every stream is drained before returning, also after an error: no copy from
+  // or to the caller's host memory may still run on return
+  bool sync_ok = cudaStreamSynchronize(st) == cudaSuccess;
+  if (nsh > 1) sync_ok = cudaStreamSynchronize(cin.s.s) == cudaSuccess && sync_ok;
+  if (dE != nullptr) sync_ok = cudaStreamSynchronize(cout.s.s) == cudaSuccess && sync_ok;
+  if (s != CUTBCE_OK) return s;
   if (!ok || !sync_ok) return CUTBCE_ERR_CUDA;
-  return static_cast<cutbce_status>(dev_status);
+  double total = 0.0;
+  for (int k = 0; k < nsh; ++k) total += losses[k];
+  *loss = total;
+  for (int k = 0; k < nsh; ++k)
+    if (statuses[k] != 0) return static_cast<cutbce_status>(statuses[k]);
+  return CUTBCE_OK;
 }
 
 cutbce_status cutbce_topk_workspace_size(int64_t B, int64_t V, int64_t D, int k, size_t* bytes) {
