@@ -1036,10 +1036,15 @@ cutbce_status cutbce_topk(const void* Q, int64_t B, const void* E, int64_t V, in
   const unsigned mgrid = static_cast<unsigned>(ceil_div(B * 32, 256));
   {
     LaunchScope ls(CUTBCE_KERNEL_TOPK_MERGE, st);
-    if (pl.KMAX == 8)
-      k_topk_merge<8><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
-    else
-      k_topk_merge<16><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+    // many lists per query (more than 64): a block per query, else a warp per query
+    const bool per_block = pl.S * 4 > 64;
+    if (pl.KMAX == 8) {
+      if (per_block) k_topk_merge_block<8><<<static_cast<unsigned>(B), 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+      else k_topk_merge<8><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+    } else {
+      if (per_block) k_topk_merge_block<16><<<static_cast<unsigned>(B), 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+      else k_topk_merge<16><<<mgrid, 256, 0, st>>>(tp.cand_s, tp.cand_i, tp.B, pl.S, k, ids, scores);
+    }
   }
   return cudaGetLastError() == cudaSuccess ? CUTBCE_OK : CUTBCE_ERR_CUDA;
 }

@@ -294,47 +294,47 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   }
 }
 
-// One warp per query: the best k of its nsplit * 4 candidate lists (each of
-// kmax entries, sorted), by descending score and ascending id.  Each lane keeps
-// the best k of the lists it reads, then k rounds of a warp-wide argmax merge
-// them.  Empty entries (id -1) are never chosen.
+// Merge of the candidate lists (each of kmax entries, sorted) of one query, by
+// descending score and ascending id.  Lane steps: each lane keeps the best
+// kmax of the lists it reads; then k rounds of a warp-wide argmax, the lane
+// holding the best head giving it up.  Empty entries (id -1) are never chosen.
 template <int KMAX>
-__global__ void __launch_bounds__(256) k_topk_merge(const float* __restrict__ cand_s, const int* __restrict__ cand_i,
-                                                     int B, int nsplit, int k, int32_t* __restrict__ ids,
-                                                     float* __restrict__ scores) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= B) return;
-  const int qt = warp / kTileM, row = warp - qt * kTileM;
-  float ls[KMAX];
-  int li[KMAX];
+__device__ __forceinline__ void lane_take_lists(const float* __restrict__ cand_s, const int* __restrict__ cand_i,
+                                                int qt, int row, int nlists, int l0, int lstep, float (&ls)[KMAX],
+                                                int (&li)[KMAX]) {
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     ls[j] = -INFINITY;
     li[j] = 0x7fffffff;
   }
-  const int nlists = nsplit * 4;
-  for (int l = lane; l < nlists; l += 32) {
+  for (int l = l0; l < nlists; l += lstep) {
     const int64_t base = ((static_cast<int64_t>(qt) * nlists + l) * kTileM + row) * KMAX;
     for (int j = 0; j < KMAX; ++j) {
       const int v = cand_i[base + j];
       if (v < 0) break;
-      const float s = cand_s[base + j];
+      const float sc = cand_s[base + j];
       // insert by (score desc, id asc): a later list may hold a lower id with an equal score
       int pos = KMAX;
       for (int t = KMAX - 1; t >= 0; --t)
-        if (s > ls[t] || (s == ls[t] && v < li[t])) pos = t;
+        if (sc > ls[t] || (sc == ls[t] && v < li[t])) pos = t;
       if (pos < KMAX) {
         for (int t = KMAX - 1; t > pos; --t) {
           ls[t] = ls[t - 1];
           li[t] = li[t - 1];
         }
-        ls[pos] = s;
+        ls[pos] = sc;
         li[pos] = v;
       }
     }
   }
-  // k rounds: the lane holding the best head gives it up
+}
+
+// k rounds over the warp's per-lane sorted lists; lane 0 writes round r to
+// out_s[r], out_i[r] (id 0x7fffffff: no entry).
+template <int KMAX>
+__device__ __forceinline__ void warp_best_k(const float (&ls)[KMAX], const int (&li)[KMAX], int k, float* out_s,
+                                            int* out_i) {
+  const int lane = threadIdx.x & 31;
   int head = 0;
   for (int r = 0; r < k; ++r) {
     float hs = -INFINITY;
@@ -360,10 +360,58 @@ __global__ void __launch_bounds__(256) k_topk_merge(const float* __restrict__ ca
     }
     if (lane == bl && head < KMAX) ++head;
     if (lane == 0) {
-      ids[static_cast<int64_t>(warp) * k + r] = bi == 0x7fffffff ? -1 : bi;
-      scores[static_cast<int64_t>(warp) * k + r] = bs;
+      out_s[r] = bs;
+      out_i[r] = bi;
     }
   }
+}
+
+// One warp per query (few lists per query: many queries).
+template <int KMAX>
+__global__ void __launch_bounds__(256) k_topk_merge(const float* __restrict__ cand_s, const int* __restrict__ cand_i,
+                                                     int B, int nsplit, int k, int32_t* __restrict__ ids,
+                                                     float* __restrict__ scores) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= B) return;
+  const int qt = warp / kTileM, row = warp - qt * kTileM;
+  float ls[KMAX];
+  int li[KMAX];
+  lane_take_lists<KMAX>(cand_s, cand_i, qt, row, nsplit * 4, lane, 32, ls, li);
+  int32_t* oi = ids + static_cast<int64_t>(warp) * k;
+  warp_best_k<KMAX>(ls, li, k, scores + static_cast<int64_t>(warp) * k, oi);
+  __syncwarp();
+  if (lane < k && oi[lane] == 0x7fffffff) oi[lane] = -1;
+}
+
+// One block of 8 warps per query (many lists per query: few queries, many
+// vocabulary splits): warp w takes lists w * 32 + lane, + 256, ...; warp 0 then
+// merges the 8 warps' k best the same way.
+template <int KMAX>
+__global__ void __launch_bounds__(256) k_topk_merge_block(const float* __restrict__ cand_s,
+                                                           const int* __restrict__ cand_i, int B, int nsplit, int k,
+                                                           int32_t* __restrict__ ids, float* __restrict__ scores) {
+  __shared__ float ws[8][KMAX];
+  __shared__ int wi[8][KMAX];
+  const int q = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = q / kTileM, row = q - qt * kTileM;
+  float ls[KMAX];
+  int li[KMAX];
+  lane_take_lists<KMAX>(cand_s, cand_i, qt, row, nsplit * 4, warp * 32 + lane, 256, ls, li);
+  warp_best_k<KMAX>(ls, li, k, ws[warp], wi[warp]);
+  __syncthreads();
+  if (warp != 0) return;
+#pragma unroll
+  for (int t = 0; t < KMAX; ++t) {
+    const bool have = lane < 8 && t < k;
+    ls[t] = have ? ws[lane < 8 ? lane : 0][t] : -INFINITY;
+    li[t] = have ? wi[lane < 8 ? lane : 0][t] : 0x7fffffff;
+  }
+  int32_t* oi = ids + static_cast<int64_t>(q) * k;
+  warp_best_k<KMAX>(ls, li, k, scores + static_cast<int64_t>(q) * k, oi);
+  __syncwarp();
+  if (lane < k && oi[lane] == 0x7fffffff) oi[lane] = -1;
 }
 
 // hits[b] = 1 if a target id (>= 0) of query b is among its k ids.
