@@ -21,6 +21,8 @@ SHAPES = [
     dict(T=130, V=515, D=192, K=6),
     dict(T=100, V=300, D=32, K=4),      # feature width padded to 64 by the TMA box
     dict(T=129, V=640, D=96, K=3),
+    dict(T=70, V=450, D=8, K=2),        # the narrowest row: one 16-byte load per row in the column sums
+    dict(T=140, V=530, D=200, K=4),     # 25 column groups of 8: ten rows per pass in the column sums
 ]
 
 
