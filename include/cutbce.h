@@ -33,7 +33,8 @@
  *    zero dH row and contributes nothing to dE; its ids are ignored entirely.
  *  - Every output and the workspace are owned by the caller.  The library
  *    never allocates or frees device memory and keeps no state between calls
- *    apart from cached device attributes and the static scratch array of
+ *    apart from cached device attributes, a per-device pool of second streams
+ *    and events (below) and the static scratch array of
  *    cutbce_forward_fixed_scratch.
  *  - All compute calls are asynchronous on `stream`.  A call that computes the
  *    loss runs the column sums of E on a second stream of the library's own
@@ -46,7 +47,8 @@
  *    launched.  Data-dependent errors (an id out of range, a bounded wait in a
  *    kernel that ran out) are written to the workspace status word; when it is
  *    nonzero the outputs of that call are unspecified.
- *  - dH and dE are overwritten, not accumulated.  The loss is double.
+ *  - dH and dE are overwritten, not accumulated (cutbce_forward_backward_ex
+ *    can accumulate instead).  The loss is double.
  *  - Results are deterministic: no floating-point atomics are used, and every
  *    reduction runs in a fixed order that does not depend on the GPU's SM count.
  */
