@@ -175,7 +175,7 @@ def workload_config(p, n_valid, world, l2_note):
     return {"workload": p.name, "B": p.B, "N": p.N, "T": p.T, "n_valid": n_valid, "V": p.V, "D": p.D, "K": p.K,
             "tokens": "value counts all B*N positions per step, padding included; valid_tokens_per_s counts "
                       "the n_valid positions that carry work",
-            "inputs": "bf16 H, E; int32 targets; uint8 mask", "seed": 0, "l2": l2_note,
+            "inputs": f"{p.dtype} H, E; int32 targets; uint8 mask", "seed": 0, "l2": l2_note,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -282,8 +282,7 @@ def run_ours(args):
     rates = probe_rates()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     p = W.draw_config(args.workload, seed=0)
-    H = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).to(dev)
-    E = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    H, E = device_inputs(p, dev)
     tg = torch.from_numpy(p.targets).to(dev)
     m = torch.from_numpy(p.mask).to(dev)
     prob = B.make_problem(H, E, tg, m, "mean")
@@ -347,8 +346,7 @@ def run_ours(args):
     # end to end through the host-buffer entry (pinned host memory, copies inside the timed call)
     e2e = None
     if not args.no_e2e:
-        Hh = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-        Eh = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Hh, Eh = (t.pin_memory() for t in device_inputs(p, "cpu"))
         th = torch.from_numpy(p.targets).pin_memory()
         mh = torch.from_numpy(p.mask).pin_memory()
         hprob = B.make_problem(Hh, Eh, th, mh, "mean")
@@ -373,7 +371,7 @@ def run_ours(args):
             ts.append(s.elapsed_time(e))
         barrier()
         e2e_ms = max_over_ranks(statistics.mean(ts))
-        bi = Hh.numel() * 2 + Eh.numel() * 2 + th.numel() * 4 + mh.numel() + 4
+        bi = Hh.numel() * Hh.element_size() + Eh.numel() * Eh.element_size() + th.numel() * 4 + mh.numel() + 4
         bo = 8 + dHh.numel() * 4 + dEh.numel() * 4
         e2e = {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms,
@@ -381,7 +379,7 @@ def run_ours(args):
         del buf
 
     extras = measure_extras(B, p, prob, H, E, tg, loss, dH, dE, ws, flush, stream, dev) \
-        if (world == 1 and not args.no_extras) else None
+        if (world == 1 and not args.no_extras and p.dtype == "bf16") else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -396,7 +394,7 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "bf16" if p.dtype == "bf16" else "f32", "data": "synthetic",
             "config": workload_config(p, n_valid, world, "flushed before each timed step (256 MiB write)"),
             "valid_tokens_per_s": world * n_valid / (step_ms * 1e-3),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -478,6 +476,15 @@ def measure_extras(B, p, prob, H, E, tg, loss, dH, dE, ws, flush, stream, dev):
     return out
 
 
+def device_inputs(p, dev):
+    """H and E on the device in the workload's dtype (bf16 bits, or fp32 for the small fp32 check)."""
+    import torch
+    if p.dtype == "bf16":
+        return (torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).to(dev),
+                torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).to(dev))
+    return torch.from_numpy(p.H).to(dev), torch.from_numpy(p.E).to(dev)
+
+
 def run_calls_only(args):
     """N plain fused calls, no timing and no output: the command ncu captures."""
     import torch
@@ -485,8 +492,7 @@ def run_calls_only(args):
     from vocabulary_label_bce_b200 import workloads as W
     p = W.draw_config(args.workload, seed=0)
     dev = torch.device("cuda", 0)
-    H = torch.from_numpy(p.H_bits.view(np.int16)).view(torch.bfloat16).to(dev)
-    E = torch.from_numpy(p.E_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    H, E = device_inputs(p, dev)
     tg = torch.from_numpy(p.targets).to(dev)
     m = torch.from_numpy(p.mask).to(dev)
     prob = B.make_problem(H, E, tg, m, "mean")
