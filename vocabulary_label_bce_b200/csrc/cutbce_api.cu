@@ -675,7 +675,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     const float* hc = at<float>(ws, pl.o_hc);
     if (item_pass) {
       LaunchScope ls(CUTBCE_KERNEL_ITEM_PASS, st);
-      k_simt_items<<<static_cast<unsigned>(pl.n_vitems), 128, 0, st>>>(
+      k_simt_items<<<dim3(static_cast<unsigned>(pl.n_vitems), static_cast<unsigned>(ceil_div(D, 32))), 128, 0, st>>>(
           hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, wc, w.dE ? dE : nullptr,
           o.grad_bf16 ? 1 : 0, o.acc_dE ? 1 : 0, w.loss ? lpart : nullptr);
       CUTBCE_CK(cudaGetLastError());
@@ -683,7 +683,8 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     if (item_pass && after_item != nullptr) CUTBCE_CK(cudaEventRecord(after_item, st));
     if (w.dH || w.met) {
       LaunchScope ls(CUTBCE_KERNEL_POSITION_PASS, st);
-      k_simt_rows<<<static_cast<unsigned>(ceil_div(pl.Tpad, 128)), 128, 0, st>>>(
+      k_simt_rows<<<dim3(static_cast<unsigned>(ceil_div(pl.Tpad, 128)), static_cast<unsigned>(ceil_div(D, 32))), 128, 0,
+                    st>>>(
           hc, static_cast<const float*>(p->E), V, D, rowptr, pair_v, hdr, w.dH ? dhpart : nullptr, metpart);
       CUTBCE_CK(cudaGetLastError());
     }

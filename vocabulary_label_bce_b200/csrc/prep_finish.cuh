@@ -479,14 +479,19 @@ __global__ void __launch_bounds__(128) k_simt_items(const float* __restrict__ Hc
                                                     const int* __restrict__ pair_v, const WsHeader* hdr,
                                                     const float* __restrict__ wc, void* __restrict__ dE, int de_bf16,
                                                     int de_acc, double* __restrict__ loss_part) {
+  // blockIdx.y: the 32 columns of dE this thread accumulates (in registers); the
+  // loss is summed by the blocks of column group 0
   __shared__ double red[128];
   const int v = blockIdx.x * 128 + threadIdx.x;
+  const int d0 = blockIdx.y * 32;
+  const bool lead = blockIdx.y == 0;
   const int nv = hdr->n_valid;
   const float gs = hdr->grad_scale;
   double lsum = 0.0;
-  float acc[kMaxDim];
+  float acc[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
   if (v < V) {
-    for (int d = 0; d < D; ++d) acc[d] = 0.f;
     const float* e = E + static_cast<int64_t>(v) * D;
     for (int c = 0; c < nv; ++c) {
       const float* h = Hc + static_cast<int64_t>(c) * D;
@@ -495,29 +500,33 @@ __global__ void __launch_bounds__(128) k_simt_items(const float* __restrict__ Hc
       for (int d = 0; d < D; ++d) z = fmaf(h[d], e[d], z);
       float y = 0.f;
       for (int p = row_ptr[c]; p < row_ptr[c + 1]; ++p) y = pair_v[p] == v ? 1.f : y;
-      lsum += static_cast<double>(w) * static_cast<double>(fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))));
+      if (lead) lsum += static_cast<double>(w) * static_cast<double>(fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))));
       if (dE != nullptr) {
         const float g = w * (sigmoid_f32(z) - y);
-        for (int d = 0; d < D; ++d) acc[d] = fmaf(g, h[d], acc[d]);
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (d0 + k < D) acc[k] = fmaf(g, h[d0 + k], acc[k]);
       }
     }
     if (dE != nullptr) {
-      for (int d = 0; d < D; ++d) {
-        const int64_t k = static_cast<int64_t>(v) * D + d;
-        float out = __fmul_rn(acc[d], gs);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        if (d0 + k >= D) break;
+        const int64_t o_ = static_cast<int64_t>(v) * D + d0 + k;
+        float out = __fmul_rn(acc[k], gs);
         if (de_bf16) {
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dE) + k;
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dE) + o_;
           if (de_acc) out = __fadd_rn(out, __bfloat162float(*o));
           *o = __float2bfloat16_rn(out);
         } else {
-          float* o = static_cast<float*>(dE) + k;
+          float* o = static_cast<float*>(dE) + o_;
           if (de_acc) out = __fadd_rn(out, *o);
           *o = out;
         }
       }
     }
   }
-  if (loss_part != nullptr) {
+  if (loss_part != nullptr && lead) {
     // same layout as the tensor-core path: kNumEpiWarps partials per 128-item tile
     const double s = block_sum_fixed(v < V ? lsum : 0.0, red);
     if (threadIdx.x < kNumEpiWarps) loss_part[static_cast<int64_t>(blockIdx.x) * kNumEpiWarps + threadIdx.x] = threadIdx.x == 0 ? s : 0.0;
@@ -530,33 +539,57 @@ __global__ void __launch_bounds__(128) k_simt_rows(const float* __restrict__ Hc,
                                                    int V, int D, const int* __restrict__ row_ptr,
                                                    const int* __restrict__ pair_v, const WsHeader* hdr,
                                                    float* __restrict__ dh_part, int2* __restrict__ met_part) {
+  // blockIdx.y: the 32 columns of dH this thread accumulates (in registers); the
+  // metrics are counted by the blocks of column group 0
   const int c = blockIdx.x * 128 + threadIdx.x;
+  const int d0 = blockIdx.y * 32;
+  const bool lead = blockIdx.y == 0;
   if (c >= hdr->n_valid) return;
-  float acc[kMaxDim];
-  for (int d = 0; d < D; ++d) acc[d] = 0.f;
+  float acc[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
   const float* h = Hc + static_cast<int64_t>(c) * D;
   int p = row_ptr[c];
   const int pend = row_ptr[c + 1];
   int cnt = 0, tp = 0;
-  for (int v = 0; v < V; ++v) {
-    const float* e = E + static_cast<int64_t>(v) * D;
-    float z = 0.f;
-    for (int d = 0; d < D; ++d) z = fmaf(h[d], e[d], z);
-    float y = 0.f;
-    if (p < pend && pair_v[p] == v) {
-      y = 1.f;
-      ++p;
+  // four items at a time: their dot products interleave (four independent load
+  // and FMA chains); their contributions are then added in item order
+  for (int vb = 0; vb < V; vb += 4) {
+    const float* eb = E + static_cast<int64_t>(vb) * D;
+    const int nu = min(4, V - vb);
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int d = 0; d < D; ++d) {
+      const float hd = h[d];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (u < nu) z[u] = fmaf(hd, eb[u * D + d], z[u]);
     }
-    cnt += z > 0.f ? 1 : 0;
-    tp += (z > 0.f && y > 0.f) ? 1 : 0;
-    if (dh_part != nullptr) {
-      const float g = sigmoid_f32(z) - y;
-      for (int d = 0; d < D; ++d) acc[d] = fmaf(g, e[d], acc[d]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (u >= nu) break;
+      const int v = vb + u;
+      const float* e = eb + u * D;
+      float y = 0.f;
+      if (p < pend && pair_v[p] == v) {
+        y = 1.f;
+        ++p;
+      }
+      cnt += z[u] > 0.f ? 1 : 0;
+      tp += (z[u] > 0.f && y > 0.f) ? 1 : 0;
+      if (dh_part != nullptr) {
+        const float g = sigmoid_f32(z[u]) - y;
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (d0 + k < D) acc[k] = fmaf(g, e[d0 + k], acc[k]);
+      }
     }
   }
-  if (dh_part != nullptr)
-    for (int d = 0; d < D; ++d) dh_part[static_cast<int64_t>(c) * D + d] = acc[d];
-  if (met_part != nullptr) met_part[c] = make_int2(cnt, tp);
+  if (dh_part != nullptr) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      if (d0 + k < D) dh_part[static_cast<int64_t>(c) * D + d0 + k] = acc[k];
+  }
+  if (met_part != nullptr && lead) met_part[c] = make_int2(cnt, tp);
 }
 
 // Zero a float buffer (used for dE when no position is valid).
