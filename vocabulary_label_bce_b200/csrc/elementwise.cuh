@@ -16,7 +16,8 @@
 //  * passes with the loss (with or without the gradient): one tanh per logit.
 //    With t = tanh(zh): sigmoid(z) = (1 + t)/2, and w = 1 + |t| = 2 sigmoid(|z|),
 //    which is in [1, 2], so l(z, 0) = max(z, 0) + ln 2 - ln w.  The log is
-//    taken once per 32 logits of a row, as log2 of the product of their w, and
+//    taken once per tile slab of a row (up to 64 logits), as log2 of the
+//    product of their w, and
 //    max(z, 0) = z / 2 + |z| / 2: the tiles sum |z| / 2, the linear z / 2 is
 //    summed over the whole problem as one dot product of column sums.
 //  * gradient only: sigmoid(z) = (1 + tanh(z/2))/2 from one tanh, except for

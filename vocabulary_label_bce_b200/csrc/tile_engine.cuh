@@ -137,9 +137,13 @@ __device__ __forceinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity, l
   }
   return true;
 }
-// Whole-warp wait: lane 0 waits, the warp then synchronises with it (which
-// orders the other lanes after lane 0's acquire of the barrier phase).
+// Whole-warp wait.  Fast path: every lane tests the phase itself (one
+// shared-memory instruction for the warp, each lane acquiring the phase) and a
+// vote, not a shuffle, gathers the answers.  Otherwise lane 0 waits (bounded)
+// and the warp then synchronises with it, which orders the other lanes after
+// lane 0's acquire of the phase.
 __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w, int tag = 0) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, w, tag);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -275,8 +279,9 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
     for (int b = 0; b < NZ; ++b) {
       mbar_init(bar_zfull + b, 1);
-      mbar_init(bar_zfree + b, kGrad ? 1 : Cfg::GROUP_WARPS);
-      mbar_init(bar_gready + b, Cfg::GROUP_WARPS);
+      // every lane of the group's warps arrives (after its own tensor-memory wait and fence)
+      mbar_init(bar_zfree + b, kGrad ? 1 : Cfg::GROUP_WARPS * 32);
+      mbar_init(bar_gready + b, Cfg::GROUP_WARPS * 32);
     }
     mbar_init(bar_accfull, 1);
     mbar_init(bar_accempty, Cfg::GROUP_WARPS);
@@ -550,9 +555,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           win = seg + lane < seg_end ? static_cast<uint32_t>(__ldg(p.tile_pairs + seg + lane)) : 0xFFFFFFFFu;
         }
       }
-      for (int j = 0; j < n; ++j) {
+      // this group's tiles of the item: c = cnt + j with c mod groups = grp
+      const int j0 = static_cast<int>((grp + Cfg::GROUPS - cnt % Cfg::GROUPS) % Cfg::GROUPS);
+      for (int j = j0; j < n; j += Cfg::GROUPS) {
         const uint32_t c = cnt + j, bz = c % NZ;
-        if (c % Cfg::GROUPS != grp) continue;      // another group's tile
         constexpr int NCH = ZC / CH;
         uint32_t pmask[NCH];                      // item-owned pass: this row's positives per chunk
 #pragma unroll
@@ -624,6 +630,10 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         }
         tc_fence_after();
         const int key0 = kDH ? (it.x_tile0 + j) * BN : j * BN;   // key of the tile's first column
+        // loss terms of the whole tile: the product of the w of its NCH * CH / 2
+        // logits per component (each in [1, 2], so at most 2^32 per component and
+        // 2^64 for both: finite in fp32) and the sum of |z| / 2
+        float2 prod = f2(1.f, 1.f), absz = f2(0.f, 0.f);
         float tile_mx = 0.f, tile_l2 = 0.f;
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
@@ -633,8 +643,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           tmem_ld_wait();
           if (!kGrad && ch == NCH - 1) {          // no G: the buffer is free once loaded
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_zfree + bz);
+            mbar_arrive(bar_zfree + bz);          // each lane, for its own loads
           }
           const uint32_t mask = !(kGrad || kMet) ? 0u
                                 : kDH ? cursor_take_mask(rc, p.pair_v, key0 + col0)
@@ -643,12 +652,14 @@ __global__ void __launch_bounds__(kTileThreads, 1)
           float2 mcnt = f2(0.f, 0.f);             // metrics: x > 0 in this chunk (two lanes of a sum)
           float mtp = 0.f;                        // metrics: positives with x > 0 in this chunk
           uint32_t pk[CH / 2];
-          float2 prod = f2(1.f, 1.f), absz = f2(0.f, 0.f);
           // the chunk's element math; the y = 1 subtraction is compiled into a
           // separate copy taken only by chunks that hold a positive (rare), so
           // the common path has no per-element branch or bit test
           // column weights (item-owned pass with per-position weights): G = w (sigmoid - y)
-          const float* wcol = (!kDH && kGrad) ? p.wc : nullptr;
+          // (per-position weights move the loss to the position-owned pass, so
+          // only the gradient-only item-owned pass ever takes them: the pass with
+          // the loss carries no weighted copy of the element loop)
+          const float* wcol = (!kDH && kGrad && !kLoss) ? p.wc : nullptr;
           const int wcol0 = j * BN + col0;        // compacted position of this chunk's first column
           auto chunk_math = [&](auto with_y, auto with_w) {
 #pragma unroll
@@ -698,24 +709,25 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             met_cnt += static_cast<int>(mcnt.x + mcnt.y);     // exact: at most CH
             met_tp += static_cast<int>(mtp);
           }
-          if (kLoss) {
-            // CH / 2 factors in [1, 2] per component: the product stays finite;
-            // tile_l2 collects log2(1 + e^{-|z|}) = 1 - log2 w of each element (w = 2 sigmoid(|z|))
-            tile_l2 += static_cast<float>(CH) - lg2_approx(prod.x * prod.y);
-            tile_mx += absz.x + absz.y;
-          }
           // G over the first half of this warp's own (already loaded) logit columns
           if (kGrad) {
             if constexpr (CH == 32) tmem_st16(tmem_base + lane_base + bz * BN + slab * ZC + ch * (CH / 2), pk);
             else tmem_st8(tmem_base + lane_base + bz * BN + slab * ZC + ch * (CH / 2), pk);
           }
         }
+        if (kLoss) {
+          // tile_l2 collects log2(1 + e^{-|z|}) = 1 - log2 w of each element (w = 2 sigmoid(|z|)),
+          // one log for the whole tile
+          tile_l2 = static_cast<float>(NCH * CH) - lg2_approx(prod.x * prod.y);
+          tile_mx = absz.x + absz.y;
+        }
         if (!ok) break;
         if (kGrad) {
           tmem_st_wait();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_gready + bz);   // this warp's part of G is in place
+          // each lane's part of G is in place: every lane arrives for its own
+          // stores (no warp barrier, no single-lane branch)
+          mbar_arrive(bar_gready + bz);
         }
         if (kLoss) {
           if (!kDH && j == n - 1) {
