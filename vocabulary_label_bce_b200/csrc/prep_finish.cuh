@@ -392,8 +392,20 @@ __global__ void __launch_bounds__(kFinishThreads) k_finish(const FinishParams f)
       const int c = f.cidx[t];
       float out = 0.f;
       if (c >= 0) {
+        // the partials of the S splits added in split order; their loads are
+        // issued eight at a time so that they are in flight together
+        const float* src = f.dh_part + static_cast<int64_t>(c) * f.DP + d;
+        const int64_t stride = f.Tpad * f.DP;
         float acc = 0.f;
-        for (int s = 0; s < f.S; ++s) acc += f.dh_part[(static_cast<int64_t>(s) * f.Tpad + c) * f.DP + d];
+        int s = 0;
+        for (; s + 8 <= f.S; s += 8) {
+          float v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = __ldg(src + (s + k) * stride);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc += v[k];
+        }
+        for (; s < f.S; ++s) acc += __ldg(src + s * stride);
         out = __fmul_rn(acc, f.weights != nullptr ? __fmul_rn(gs, f.weights[t]) : gs);
       }
       // accumulation adds the fp32 gradient as it would be written without it
