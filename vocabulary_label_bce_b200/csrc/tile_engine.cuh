@@ -43,9 +43,8 @@
 //               MMAs and the gradient MMAs, issued by one elected lane
 //   warps 2-17  epilogue.  Warp w reads TMEM lanes 32*(w%4).. (the quarter its
 //               sub-partition may access) and one column slab of the tile.
-//               Item-owned pass: two groups of 8 take alternate tiles (64-
-//               column slabs); position-owned pass: all 16 take every tile
-//               (32-column slabs).
+//               Two groups of 8 take alternate tiles (64-column slabs, or
+//               32 with 64-row streamed tiles).
 //
 // Tensor memory holds NZ = 3 fp32 logit buffers, the gradient accumulator and,
 // where it fits, a copy of the stationary tile (the logit MMA's A operand, so
