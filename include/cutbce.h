@@ -255,13 +255,15 @@ cutbce_status cutbce_host_buffer_size(const cutbce_problem* prob, size_t* bytes)
  * copies the results out and synchronises; on return the host outputs are
  * valid and the returned status includes the device status word.
  * Overlap: with a bf16 item table of more than 32 MiB, the call works in up to
- * four vocabulary shards of whole 128-item tiles (the shard options of
- * cutbce_forward_backward_ex): shard s + 1 of E is copied in on a second stream
- * while shard s is computed on `stream`, and each shard's dE rows are copied
- * out on a third stream as soon as its item-owned pass ends, while its dH pass
- * and the next shard run.  The shards' losses are added on the host and their
- * dH on the device, in shard order, so the results are deterministic and equal
- * those of cutbce_forward_backward to rounding (bit for bit with one shard).
+ * four vocabulary shards (whole vocabulary splits of the dH pass, on whole
+ * 128-item tiles).  It compacts the rows and orders the pairs once (that reads
+ * no E).  Then, as shard s of E lands (copied in on a second stream while shard
+ * s - 1 is computed on `stream`), it runs the two tile passes over that shard's
+ * item tiles and splits only; the shard's dE rows are copied out on a third
+ * stream as soon as its item-owned pass ends.  The sparse correction, the
+ * column sums and the finish run once at the end.  Every tile and split is
+ * computed exactly as by cutbce_forward_backward and summed by the same finish,
+ * so loss, dH and dE are its bits.
  * The streams and events come from a per-device pool, created by the first
  * such calls and kept for the rest of the process; every stream the call used
  * is synchronised before it returns. */

@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <climits>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -54,7 +55,15 @@ struct Opts {
   bool grad_bf16 = false, acc_dH = false, acc_dE = false;
   int64_t v_off = 0, V_total = 0;   // V_total resolved: the problem's V when not sharded
   bool one_stream = false;           // everything on the caller's stream (no pooled second stream)
+  // A call in parts (the host-buffer entry, tensor-core path): kPhasePrep
+  // compacts the rows and orders the pairs (no E read), kPhasePasses runs the
+  // two tile passes over item tiles [tile_begin, tile_end) and vocabulary
+  // splits [split_begin, split_end), kPhaseFinish sums the sparse correction
+  // and the column sums and finishes.  All three in one call is the plain call.
+  int phases = 7;
+  int tile_begin = 0, tile_end = INT_MAX, split_begin = 0, split_end = INT_MAX;
 };
+constexpr int kPhasePrep = 1, kPhasePasses = 2, kPhaseFinish = 4;
 
 cutbce_status resolve_opts(const cutbce_problem* p, const cutbce_options* o, Opts& out) {
   out = Opts{};
@@ -523,10 +532,13 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   // the column sums of E depend on E alone: a second stream computes them while
   // the prep kernels run, and the column-sum kernel of H_c waits for it
   // (the fixed-scratch entry keeps to one stream: it runs them in order)
+  const bool ph_prep = (o.phases & kPhasePrep) != 0, ph_passes = (o.phases & kPhasePasses) != 0,
+             ph_finish = (o.phases & kPhaseFinish) != 0;
+  if (!bf16 && o.phases != (kPhasePrep | kPhasePasses | kPhaseFinish)) return CUTBCE_ERR_UNSUPPORTED;
   SideStreamLease side;
-  if (bf16 && w.loss) {
+  if (bf16 && w.loss && ph_finish) {
     cudaStream_t cs = st;
-    if (!o.one_stream) {
+    if (!o.one_stream && ph_prep) {
       if ((s = take_side_stream(side.s)) != CUTBCE_OK) return s;
       side.held = true;
       CUTBCE_CK(cudaEventRecord(side.s.ev, st));
@@ -540,6 +552,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     CUTBCE_CK(cudaGetLastError());
     if (side.held) CUTBCE_CK(cudaEventRecord(side.s.ev2, side.s.s));
   }
+  if (ph_prep) {
   CUTBCE_CK(cudaMemsetAsync(hdr, 0, 256, st));
   {
   LaunchScope ls(CUTBCE_KERNEL_PREP_ROWS, st);
@@ -553,24 +566,29 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
                                           orig, rowptr, hdr);
   CUTBCE_CK(cudaGetLastError());
   }
-  {
-  LaunchScope ls(CUTBCE_KERNEL_PREP_GATHER, st);
-  if (bf16) {
-    k_prep_gather<__nv_bfloat16><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(p->H), static_cast<const __nv_bfloat16*>(p->E), D, pl.DP, K, pl.Tpad,
-        orig, ids, rowcnt, rowptr, hdr, o.weights, wc, at<__nv_bfloat16>(ws, pl.o_hc), pair_t, pair_v, cpart);
-  } else {
-    k_prep_gather<float><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
-        static_cast<const float*>(p->H), static_cast<const float*>(p->E), D, pl.DP, K, pl.Tpad, orig, ids, rowcnt,
-        rowptr, hdr, o.weights, wc, at<float>(ws, pl.o_hc), pair_t, pair_v, cpart);
   }
-  CUTBCE_CK(cudaGetLastError());
-  }
+  // the gather: the rows and pairs with the prep, the sparse correction (which
+  // reads E) with the finish; one launch when the call has both
+  auto gather = [&](int mode) -> cudaError_t {
+    LaunchScope ls(CUTBCE_KERNEL_PREP_GATHER, st);
+    if (bf16) {
+      k_prep_gather<__nv_bfloat16><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(p->H), static_cast<const __nv_bfloat16*>(p->E), D, pl.DP, K, pl.Tpad,
+          orig, ids, rowcnt, rowptr, hdr, o.weights, wc, at<__nv_bfloat16>(ws, pl.o_hc), pair_t, pair_v, cpart, mode);
+    } else {
+      k_prep_gather<float><<<static_cast<unsigned>(pl.n_gather_blocks), 256, 0, st>>>(
+          static_cast<const float*>(p->H), static_cast<const float*>(p->E), D, pl.DP, K, pl.Tpad, orig, ids, rowcnt,
+          rowptr, hdr, o.weights, wc, at<float>(ws, pl.o_hc), pair_t, pair_v, cpart, mode);
+    }
+    return cudaGetLastError();
+  };
+  if (ph_prep) CUTBCE_CK(gather(kGatherRows | (ph_finish ? kGatherCorrection : 0)));
+  else if (ph_finish) CUTBCE_CK(gather(kGatherCorrection));
 
   // With per-position weights the tensor-core path sums the loss in the
   // position-owned pass (one weight per row there); the item-owned pass then
   // computes dE only.  The fp32 path sums it per item with the column weights.
-  if (bf16 && w.loss) {
+  if (bf16 && w.loss && ph_finish) {
     if (side.held) CUTBCE_CK(cudaStreamWaitEvent(st, side.s.ev2, 0));
     LaunchScope ls(CUTBCE_KERNEL_COL_SUMS, st);
     k_col_sums<<<static_cast<unsigned>(pl.csum_nbH), kColSumThreads, 0, st>>>(
@@ -586,7 +604,11 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
   if (bf16) {
     const int* srt_key = pair_v;
     const int* srt_val = pair_t;
-    if (w.dE) {
+    if (w.dE && !ph_prep) {
+      // ordered by an earlier part of the call: the last radix pass's output
+      srt_val = at<int>(ws, pl.o_srt[2 * ((pl.radix_passes - 1) & 1) + 1]);
+    }
+    if (w.dE && ph_prep) {
       // pairs grouped by item tile, ascending position inside a group: stable LSD
       // radix sort of (item tile, packed row/position) starting from (position, item) order
       LaunchScope ls(CUTBCE_KERNEL_PAIR_SORT, st);
@@ -609,7 +631,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
       }
       CUTBCE_CK(cudaGetLastError());
     }
-    if (w.dE) {
+    if (w.dE && ph_prep) {
       LaunchScope ls(CUTBCE_KERNEL_CSC_OFFSETS, st);
       const int nkeys = static_cast<int>(pl.n_vitems);
       k_key_offsets<<<static_cast<unsigned>(ceil_div(nkeys + 1, 256)), 256, 0, st>>>(srt_key, hdr, nkeys, cscoff);
@@ -635,12 +657,18 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     tp.tiles_per_split = pl.tps;
     tp.n_item_tiles_bn = pl.n_vtiles_bn;
     tp.timeout_ns = kDefaultTimeoutNs;
+    tp.range_begin = o.tile_begin;
+    tp.range_end = o.tile_end;
     const __nv_bfloat16* hc = at<__nv_bfloat16>(ws, pl.o_hc);
-    if (item_pass) {
+    const int64_t tiles_in_range =
+        std::max<int64_t>(0, std::min<int64_t>(o.tile_end, pl.n_vitems) - std::min<int64_t>(o.tile_begin, pl.n_vitems));
+    const int64_t splits_in_range =
+        std::max<int64_t>(0, std::min<int64_t>(o.split_end, pl.S) - std::min<int64_t>(o.split_begin, pl.S));
+    if (ph_passes && item_pass && tiles_in_range > 0) {
       CUtensorMap ms, mx;
       if (!make_map(&ms, p->E, D, V, D, kTileM) || !make_map(&mx, hc, pl.DP, pl.Tpad, pl.DP, pl.BN))
         return CUTBCE_ERR_CUDA;
-      const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(dev.sms), pl.n_vitems,
+      const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(dev.sms), tiles_in_range,
                                                            static_cast<int64_t>(kMaxCtas)}));
       cudaError_t e;
       LaunchScope ls(CUTBCE_KERNEL_ITEM_PASS, st);
@@ -649,12 +677,14 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
       else e = launch_tile_dp<false, true, false>(pl.DP, grid, ms, mx, tp, st);
       CUTBCE_CK(e);
     }
-    if (item_pass && after_item != nullptr) CUTBCE_CK(cudaEventRecord(after_item, st));
-    if (pos_pass) {
+    if (ph_passes && item_pass && after_item != nullptr) CUTBCE_CK(cudaEventRecord(after_item, st));
+    tp.range_begin = o.split_begin;
+    tp.range_end = o.split_end;
+    if (ph_passes && pos_pass && splits_in_range > 0) {
       CUtensorMap ms, mx;
       if (!make_map(&ms, hc, pl.DP, pl.Tpad, pl.DP, kTileM) || !make_map(&mx, p->E, D, V, D, pl.BN))
         return CUTBCE_ERR_CUDA;
-      const int64_t items_max = static_cast<int64_t>(pl.S) * ceil_div(T, kTileM);
+      const int64_t items_max = splits_in_range * ceil_div(T, kTileM);
       const int grid = static_cast<int>(
           std::min<int64_t>({static_cast<int64_t>(dev.sms), items_max, static_cast<int64_t>(kMaxCtas)}));
       LaunchScope ls(CUTBCE_KERNEL_POSITION_PASS, st);
@@ -689,7 +719,7 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
       CUTBCE_CK(cudaGetLastError());
     }
   }
-  if (w.loss || w.dH || w.met) {
+  if (ph_finish && (w.loss || w.dH || w.met)) {
     const unsigned grid = static_cast<unsigned>(finish_grid(T, D));
     FinishParams fp{};
     fp.T = T;
@@ -727,12 +757,13 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
 
 // Host-buffer entry: layout of the caller's device buffer.
 struct HostLayout {
-  size_t o_H, o_E, o_tg, o_mask, o_loss, o_status, o_grad, o_dH, o_dE, o_ws, total;
+  size_t o_H, o_E, o_tg, o_mask, o_loss, o_grad, o_dH, o_dE, o_ws, total;
 };
 
 // The host-buffer entry runs a large item table in up to kMaxHostShards
-// vocabulary shards of whole 128-item tiles, so that copying shard s + 1 in and
-// shard s - 1's dE out overlap the computation of shard s.
+// vocabulary shards (whole splits of the position-owned pass, on whole 128-item
+// tiles), so that copying shard s + 1 in and shard s - 1's dE out overlap the
+// computation of shard s.
 constexpr int kMaxHostShards = 4;
 constexpr int64_t kHostShardBytes = int64_t(32) << 20;
 
@@ -743,16 +774,22 @@ int host_shards(const cutbce_problem* p) {
   return static_cast<int>(std::max<int64_t>(1, n));
 }
 
-// Items [v0, v1) of shard k of n, in whole tiles.  The first and the last shard
-// are the smaller ones: the first one's copy in and the last one's copy out are
-// the only copies nothing overlaps.  Cumulative shares in 1/20 of the tiles.
-void host_shard_bounds(int64_t V, int n, int k, int64_t& v0, int64_t& v1) {
+// Shard k of n in vocabulary splits of the position-owned pass: splits
+// [s0, s1), which cover the items [v0, v1) and, since the boundaries fall on
+// whole 128-item tiles, the item tiles [v0 / 128, ceil(v1 / 128)).
+void host_shard_splits(const Plan& pl, int n, int k, int& s0, int& s1, int64_t& v0, int64_t& v1) {
   static const int kCum[kMaxHostShards + 1][kMaxHostShards + 1] = {
       {0, 0, 0, 0, 0}, {0, 20, 0, 0, 0}, {0, 10, 20, 0, 0}, {0, 5, 15, 20, 0}, {0, 3, 10, 17, 20}};
-  const int64_t tiles = ceil_div(V, kTileM);
-  const int64_t t0 = tiles * kCum[n][k] / 20, t1 = tiles * kCum[n][k + 1] / 20;
-  v0 = std::min(V, t0 * kTileM);
-  v1 = std::min(V, t1 * kTileM);
+  const int64_t rows_per_split = static_cast<int64_t>(pl.tps) * pl.BN;
+  s0 = static_cast<int>(int64_t(pl.S) * kCum[n][k] / 20);
+  s1 = static_cast<int>(int64_t(pl.S) * kCum[n][k + 1] / 20);
+  if (rows_per_split % kTileM != 0) {   // 64-row splits of odd length: boundaries at even splits
+    s0 &= ~1;
+    s1 &= ~1;
+  }
+  if (k + 1 == n) s1 = pl.S;
+  v0 = std::min<int64_t>(pl.V, s0 * rows_per_split);
+  v1 = k + 1 == n ? pl.V : std::min<int64_t>(pl.V, s1 * rows_per_split);
 }
 
 void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
@@ -766,8 +803,7 @@ void host_layout(const cutbce_problem* p, const Plan& pl, HostLayout& hl) {
   hl.o_E = take(pl.elem * p->V * p->D);
   hl.o_tg = take(4 * p->T * p->K);
   hl.o_mask = take(p->T);
-  hl.o_loss = take(8 * kMaxHostShards);       // one loss per shard, summed on the host in shard order
-  hl.o_status = take(4 * kMaxHostShards);     // the status word of each shard's call
+  hl.o_loss = take(8);
   hl.o_grad = take(4);
   hl.o_dH = take(4 * p->T * p->D);
   hl.o_dE = take(4 * p->V * p->D);
@@ -904,11 +940,23 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   HostLayout hl;
   host_layout(prob, pl, hl);
   if (dev_bytes < hl.total) return CUTBCE_ERR_WORKSPACE;
-  const int nsh = host_shards(prob);
+  const Want w{true, dE != nullptr, dH != nullptr, false};
+  Plan plw;
+  make_plan(prob, w, plw);           // the plan of the call's parts (splits, tile sizes, header offset)
+  int nsh = host_shards(prob);
+  nsh = std::min(nsh, std::max(1, plw.S / 2));
   // Streams (per-device pool, created on first use): E's shards are copied in on
   // `cin`, the computation runs on `st`, and each shard's dE is copied out on
   // `cout` as soon as its item-owned pass ends (dE is final then), while the
   // dH pass and the next shard run on `st`.
+  //
+  // With more than one shard the call runs in parts on one workspace: the prep
+  // and the pair order once (they read no E), then each shard's two tile
+  // passes as soon as its rows of E are in, over the item tiles and the
+  // vocabulary splits it covers, then the sparse correction, the column sums
+  // and the finish once.  Every tile and split is computed exactly as by the
+  // one-call path and the partials are summed by the same finish, so the
+  // results are the same bits.
   SideStreamLease cin, cout;
   if (nsh > 1) {
     if ((s = take_side_stream(cin.s)) != CUTBCE_OK) return s;
@@ -931,47 +979,60 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
             cudaMemcpyAsync(b + hl.o_grad, &grad_loss, 4, cudaMemcpyHostToDevice, st) == cudaSuccess;
   cutbce_problem dp = *prob;
   dp.H = b + hl.o_H;
+  dp.E = b + hl.o_E;
   dp.targets = reinterpret_cast<const int32_t*>(b + hl.o_tg);
   dp.mask = prob->mask != nullptr ? reinterpret_cast<const uint8_t*>(b + hl.o_mask) : nullptr;
   float* ddH = dH ? reinterpret_cast<float*>(b + hl.o_dH) : nullptr;
   float* ddE = dE ? reinterpret_cast<float*>(b + hl.o_dE) : nullptr;
   double* dloss = reinterpret_cast<double*>(b + hl.o_loss);
-  int32_t* dstatus = reinterpret_cast<int32_t*>(b + hl.o_status);
-  for (int k = 0; k < nsh && ok && s == CUTBCE_OK; ++k) {
-    int64_t v0 = 0, v1 = prob->V;
-    if (nsh > 1) host_shard_bounds(prob->V, nsh, k, v0, v1);   // never empty: nsh > 1 needs V D > 16 Mi
-    if (v1 <= v0) {
-      s = CUTBCE_ERR_INVALID_ARG;
-      break;
+  const float* dgrad = reinterpret_cast<const float*>(b + hl.o_grad);
+  void* dws = b + hl.o_ws;
+  cudaEvent_t after_item = dE != nullptr ? cout.s.ev : nullptr;
+  // the rows [v0, v1) of dE are final once the item-owned pass over them has run
+  auto copy_dE_out = [&](int64_t v0, int64_t v1) {
+    return dE == nullptr ||
+           (cudaStreamWaitEvent(cout.s.s, cout.s.ev, 0) == cudaSuccess &&
+            cudaMemcpyAsync(dE + v0 * prob->D, ddE + v0 * prob->D, 4 * (v1 - v0) * prob->D, cudaMemcpyDeviceToHost,
+                            cout.s.s) == cudaSuccess);
+  };
+  if (ok && nsh == 1) {
+    ok = cudaMemcpyAsync(b + hl.o_E, prob->E, prob->V * rowE, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    if (ok) s = run(&dp, dgrad, dloss, ddH, ddE, w, dws, pl.total, st, after_item);
+    if (ok && s == CUTBCE_OK) ok = copy_dE_out(0, prob->V);
+  } else if (ok) {
+    Opts part{};
+    part.phases = kPhasePrep;
+    s = run(&dp, dgrad, dloss, ddH, ddE, w, dws, pl.total, st, nullptr, part);
+    for (int k = 0; k < nsh && ok && s == CUTBCE_OK; ++k) {
+      int s0 = 0, s1 = 0;
+      int64_t v0 = 0, v1 = 0;
+      host_shard_splits(plw, nsh, k, s0, s1, v0, v1);
+      if (v1 <= v0) continue;               // an empty shard (few splits): nothing to copy or compute
+      ok = cudaMemcpyAsync(b + hl.o_E + v0 * rowE, static_cast<const uint8_t*>(prob->E) + v0 * rowE,
+                           (v1 - v0) * rowE, cudaMemcpyHostToDevice, in) == cudaSuccess &&
+           cudaEventRecord(cin.s.ev, in) == cudaSuccess && cudaStreamWaitEvent(st, cin.s.ev, 0) == cudaSuccess;
+      if (!ok) break;
+      part = Opts{};
+      part.phases = kPhasePasses;
+      part.tile_begin = static_cast<int>(v0 / kTileM);
+      part.tile_end = static_cast<int>(ceil_div(v1, kTileM));
+      part.split_begin = s0;
+      part.split_end = s1;
+      s = run(&dp, dgrad, dloss, ddH, ddE, w, dws, pl.total, st, after_item, part);
+      if (s == CUTBCE_OK) ok = copy_dE_out(v0, v1);
     }
-    ok = cudaMemcpyAsync(b + hl.o_E + v0 * rowE, static_cast<const uint8_t*>(prob->E) + v0 * rowE,
-                         (v1 - v0) * rowE, cudaMemcpyHostToDevice, in) == cudaSuccess;
-    if (ok && nsh > 1)
-      ok = cudaEventRecord(cin.s.ev, in) == cudaSuccess && cudaStreamWaitEvent(st, cin.s.ev, 0) == cudaSuccess;
-    if (!ok) break;
-    cutbce_problem sp = dp;
-    sp.E = b + hl.o_E + v0 * rowE;
-    sp.V = v1 - v0;
-    Opts o{};
-    o.v_off = v0;
-    o.V_total = prob->V;
-    o.acc_dH = k > 0;                        // the shards' dH add up, in shard order
-    s = run(&sp, reinterpret_cast<const float*>(b + hl.o_grad), dloss + k, ddH,
-            ddE ? ddE + v0 * prob->D : nullptr, Want{true, dE != nullptr, dH != nullptr, false}, b + hl.o_ws,
-            pl.total, st, dE != nullptr ? cout.s.ev : nullptr, o);
-    if (s != CUTBCE_OK) break;
-    ok = cudaMemcpyAsync(dstatus + k, b + hl.o_ws + pl.o_hdr, 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
-    if (ok && dE != nullptr)
-      ok = cudaStreamWaitEvent(cout.s.s, cout.s.ev, 0) == cudaSuccess &&
-           cudaMemcpyAsync(dE + v0 * prob->D, ddE + v0 * prob->D, 4 * (v1 - v0) * prob->D, cudaMemcpyDeviceToHost,
-                           cout.s.s) == cudaSuccess;
+    if (ok && s == CUTBCE_OK) {
+      part = Opts{};
+      part.phases = kPhaseFinish;
+      s = run(&dp, dgrad, dloss, ddH, ddE, w, dws, pl.total, st, nullptr, part);
+    }
   }
-  double losses[kMaxHostShards] = {};
-  int32_t statuses[kMaxHostShards] = {};
+  double loss_h = 0.0;
+  int32_t status_h = 0;
   if (ok && s == CUTBCE_OK)
-    ok = cudaMemcpyAsync(losses, dloss, 8 * nsh, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
+    ok = cudaMemcpyAsync(&loss_h, dloss, 8, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
          (!dH || cudaMemcpyAsync(dH, ddH, 4 * prob->T * prob->D, cudaMemcpyDeviceToHost, st) == cudaSuccess) &&
-         cudaMemcpyAsync(statuses, dstatus, 4 * nsh, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+         cudaMemcpyAsync(&status_h, b + hl.o_ws + plw.o_hdr, 4, cudaMemcpyDeviceToHost, st) == cudaSuccess;
   // every stream is drained before returning, also after an error: no copy from
   // or to the caller's host memory may still run on return
   bool sync_ok = cudaStreamSynchronize(st) == cudaSuccess;
@@ -979,12 +1040,8 @@ cutbce_status cutbce_forward_backward_host(const cutbce_problem* prob, float gra
   if (dE != nullptr) sync_ok = cudaStreamSynchronize(cout.s.s) == cudaSuccess && sync_ok;
   if (s != CUTBCE_OK) return s;
   if (!ok || !sync_ok) return CUTBCE_ERR_CUDA;
-  double total = 0.0;
-  for (int k = 0; k < nsh; ++k) total += losses[k];
-  *loss = total;
-  for (int k = 0; k < nsh; ++k)
-    if (statuses[k] != 0) return static_cast<cutbce_status>(statuses[k]);
-  return CUTBCE_OK;
+  *loss = loss_h;
+  return status_h != 0 ? static_cast<cutbce_status>(status_h) : CUTBCE_OK;
 }
 
 cutbce_status cutbce_topk_workspace_size(int64_t B, int64_t V, int64_t D, int k, size_t* bytes) {

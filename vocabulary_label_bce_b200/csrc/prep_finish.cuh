@@ -177,8 +177,14 @@ __global__ void __launch_bounds__(kScanThreads) k_prep_scan(const uint8_t* __res
 // target correction sum_{v in P_t} w_t h_t . e_v of Eq. (2) in fp32 per pair, in
 // a fixed order, into one double per block.
 // bf16 H_c (the tensor-core path) holds h / 2; fp32 H_c (the SIMT path) holds h.
+// `mode` selects the work: kGatherRows (H_c, the compacted weights and the pair
+// lists, which need no E), kGatherCorrection (the correction partials, which
+// read E), or both.  Split in two, the same blocks sum the same pairs in the
+// same order: the partials are bit-identical to one launch doing both.
 template <typename TIn>
 constexpr bool kHalveHc = sizeof(TIn) == 2;
+constexpr int kGatherRows = 1;
+constexpr int kGatherCorrection = 2;
 
 template <typename TIn>
 __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, const TIn* __restrict__ E,
@@ -188,7 +194,9 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
                                                      const int* __restrict__ row_ptr, const WsHeader* hdr,
                                                      const float* __restrict__ weights, float* __restrict__ wc,
                                                      TIn* __restrict__ Hc, int* __restrict__ pair_t,
-                                                     int* __restrict__ pair_v, double* __restrict__ corr_part) {
+                                                     int* __restrict__ pair_v, double* __restrict__ corr_part,
+                                                     int mode) {
+  const bool rows = (mode & kGatherRows) != 0, corr = (mode & kGatherCorrection) != 0;
   __shared__ double wsum[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t c = static_cast<int64_t>(blockIdx.x) * 8 + warp;
@@ -196,32 +204,36 @@ __global__ void __launch_bounds__(256) k_prep_gather(const TIn* __restrict__ H, 
   double acc = 0.0;
   if (c < Tpad) {
     TIn* dst = Hc + c * DP;
-    if (wc != nullptr && lane == 0) wc[c] = c < nv ? weights[orig[c]] : 0.f;
+    if (rows && wc != nullptr && lane == 0) wc[c] = c < nv ? weights[orig[c]] : 0.f;
     if (c < nv) {
       const int t = orig[c];
       const double wt = weights != nullptr ? static_cast<double>(weights[t]) : 1.0;
       const TIn* src = H + static_cast<int64_t>(t) * D;
-      for (int d = lane; d < DP; d += 32)
-        dst[d] = d < D ? (kHalveHc<TIn> ? TIn(0.5f * static_cast<float>(src[d])) : src[d]) : TIn(0.0f);
+      if (rows)
+        for (int d = lane; d < DP; d += 32)
+          dst[d] = d < D ? (kHalveHc<TIn> ? TIn(0.5f * static_cast<float>(src[d])) : src[d]) : TIn(0.0f);
       const int p0 = row_ptr[c];
       const int n = row_cnt[t];
       for (int k = 0; k < n; ++k) {
         const int v = ids[static_cast<int64_t>(t) * K + k];
-        if (lane == 0) {
+        if (rows && lane == 0) {
           pair_t[p0 + k] = static_cast<int>(c);
           pair_v[p0 + k] = v;
         }
-        const TIn* e = E + static_cast<int64_t>(v) * D;
-        float z = 0.f;
-        for (int d = lane; d < D; d += 32) z = fmaf(static_cast<float>(src[d]), static_cast<float>(e[d]), z);
+        if (corr) {
+          const TIn* e = E + static_cast<int64_t>(v) * D;
+          float z = 0.f;
+          for (int d = lane; d < D; d += 32) z = fmaf(static_cast<float>(src[d]), static_cast<float>(e[d]), z);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-        acc += wt * static_cast<double>(z);
+          for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+          acc += wt * static_cast<double>(z);
+        }
       }
-    } else {
+    } else if (rows) {
       for (int d = lane; d < DP; d += 32) dst[d] = TIn(0.0f);
     }
   }
+  if (!corr) return;
   if (lane == 0) wsum[warp] = acc;
   __syncthreads();
   if (threadIdx.x == 0) {

@@ -89,6 +89,9 @@ struct TileParams {
   int nsplit;                  // position-owned pass: vocabulary splits S
   int tiles_per_split;         // streamed item tiles per split
   int n_item_tiles_bn;         // ceil(V / BN)
+  int range_begin, range_end;  // the launch's share of the work: item tiles [begin, end) of the
+                               // item-owned pass, vocabulary splits [begin, end) of the position-owned
+                               // pass (the whole of it: 0 and INT_MAX)
   long long timeout_ns;
 };
 
@@ -248,12 +251,16 @@ __global__ void __launch_bounds__(kTileThreads, 1)
   __syncthreads();
   if (s_status != 0) return;  // an earlier step failed
   const int n_valid = s_nvalid;
-  const int n_items = kDH ? p.nsplit * static_cast<int>(ceil_div(n_valid, kTileM))
-                          : static_cast<int>(ceil_div(p.V, kTileM));
+  // work items: item tiles (item-owned pass) or (split, position tile) pairs,
+  // split-major (position-owned pass); this launch takes [i_lo, n_items)
+  const int n_pos_tiles = static_cast<int>(ceil_div(n_valid, kTileM));
+  const int i_lo = kDH ? min(p.range_begin, p.nsplit) * n_pos_tiles : min(p.range_begin, static_cast<int>(ceil_div(p.V, kTileM)));
+  const int n_items = kDH ? min(p.range_end, p.nsplit) * n_pos_tiles
+                          : min(p.range_end, static_cast<int>(ceil_div(p.V, kTileM)));
 
   if (!kDH && n_valid == 0) {
     // no valid position: dE = 0 and every item's loss is 0
-    for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
+    for (int i = i_lo + static_cast<int>(blockIdx.x); i < n_items; i += gridDim.x) {
       if (kLoss && threadIdx.x < kNumEpiWarps) p.loss_part[static_cast<int64_t>(i) * kNumEpiWarps + threadIdx.x] = 0.0;
       if (kGrad && p.dE != nullptr && !p.de_acc) {
         const int64_t r0 = static_cast<int64_t>(i) * kTileM;
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
     return;
   }
-  if (static_cast<int>(blockIdx.x) >= n_items) return;
+  if (i_lo + static_cast<int>(blockIdx.x) >= n_items) return;
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -303,7 +310,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     // ============================================================ TMA producer
     if (lane == 0) {
       uint32_t ic = 0, xc = 0;
-      for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++ic) {
+      for (int i = i_lo + static_cast<int>(blockIdx.x); i < n_items; i += gridDim.x, ++ic) {
         const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
         if (!wait_bar(bar_sempty, (ic & 1) ^ 1, wc, wait_tag(1, 1, ic))) break;
         mbar_arrive_expect_tx(bar_sfull, S_BYTES);
@@ -357,7 +364,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
       const uint64_t dXk = smem_desc_sw128(smem_u32(sX), 16, 1024);    // streamed tile as K-major B
       const uint64_t dXmn = smem_desc_sw128(smem_u32(sX), BN * 128, 1024);  // streamed tile as MN-major B
       const uint32_t tZ = tmem_base, tAcc = tmem_base + ACC_COL, tS = tmem_base + Cfg::S_COL;
-      int zi = blockIdx.x, zj = 0, gi = blockIdx.x, gj = 0;
+      int zi = i_lo + static_cast<int>(blockIdx.x), zj = 0, gi = zi, gj = 0;
       uint32_t zic = 0, cz = 0, gic = 0, cg = 0;
       uint32_t zst = 0, zph = 0, zoff = 0;        // ring stage of the next logit tile, its phase, its offset
       uint32_t gst = 0, goff = 0;                 // ring stage of the next gradient MMA, its offset
@@ -532,7 +539,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     __syncwarp();
     uint32_t cnt = 0, ic = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ic) {
+    for (int i = i_lo + static_cast<int>(blockIdx.x); i < n_items && ok; i += gridDim.x, ++ic) {
       const ItemInfo it = item_info<DP, kDH>(i, n_valid, p);
       const int n = it.n_x;
       double item_acc = 0.0;
