@@ -553,19 +553,19 @@ cutbce_status run(const cutbce_problem* p, const float* grad_loss, double* loss,
     if (side.held) CUTBCE_CK(cudaEventRecord(side.s.ev2, side.s.s));
   }
   if (ph_prep) {
-  CUTBCE_CK(cudaMemsetAsync(hdr, 0, 256, st));
-  {
-  LaunchScope ls(CUTBCE_KERNEL_PREP_ROWS, st);
-  k_prep_rows<<<static_cast<unsigned>(ceil_div(T, 128)), 128, 0, st>>>(p->targets, p->mask, o.weights, T, K, V,
-                                                                        o.v_off, o.V_total, ids, rowcnt, hdr);
-  CUTBCE_CK(cudaGetLastError());
-  }
-  {
-  LaunchScope ls(CUTBCE_KERNEL_PREP_SCAN, st);
-  k_prep_scan<<<1, kScanThreads, 0, st>>>(p->mask, o.weights, rowcnt, T, o.V_total, p->reduction, grad_loss, cidx,
-                                          orig, rowptr, hdr);
-  CUTBCE_CK(cudaGetLastError());
-  }
+    CUTBCE_CK(cudaMemsetAsync(hdr, 0, 256, st));
+    {
+      LaunchScope ls(CUTBCE_KERNEL_PREP_ROWS, st);
+      k_prep_rows<<<static_cast<unsigned>(ceil_div(T, 128)), 128, 0, st>>>(p->targets, p->mask, o.weights, T, K, V,
+                                                                            o.v_off, o.V_total, ids, rowcnt, hdr);
+      CUTBCE_CK(cudaGetLastError());
+    }
+    {
+      LaunchScope ls(CUTBCE_KERNEL_PREP_SCAN, st);
+      k_prep_scan<<<1, kScanThreads, 0, st>>>(p->mask, o.weights, rowcnt, T, o.V_total, p->reduction, grad_loss,
+                                              cidx, orig, rowptr, hdr);
+      CUTBCE_CK(cudaGetLastError());
+    }
   }
   // the gather: the rows and pairs with the prep, the sparse correction (which
   // reads E) with the finish; one launch when the call has both
